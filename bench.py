@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the OrbitQuant rotate-then-quantize linear layer on B200.
+
+One step = the whole per-token hot path over one batch: the fused RPBH
+rotate + norm split + Lloyd-Max quantise kernel on the activations, then the
+codebook-decode tcgen05 GEMM (weights were quantised offline, before timing).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle as the reference arm
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+M tokens against a replicated packed weight -- the path has no exchange, so
+there is no data-path collective (weak scaling); only the timing is reduced
+(max over ranks).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "qlinear tokens/s and TFLOP/s (% bf16 peak); RPBH+quant GB/s (% HBM peak)"
+DEFAULT_WORKLOAD = "flux_qkv_w4a4"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def committed_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if one exists for
+    this kernel and workload (null otherwise)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    return j.get(kernel, {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed loop runs."""
+
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 10:
+                self.rows.append((time.time(), parts))
+
+    def mark(self, which):
+        if which == "start":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mine = [p for (t, p) in self.rows if (not self.uuid or self.uuid in p[1])]
+        inside = [p for (t, p) in self.rows if self.t0 and self.t0 - 0.05 <= t <= self.t1 + 0.05 and
+                  (not self.uuid or self.uuid in p[1])]
+        use = inside if inside else mine[-5:]
+        if not use:
+            return None
+        sm = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
+        mx = [float(p[3]) for p in use if p[3].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in use:
+            for n, v in zip(names, p[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def rpbh_bytes(w):
+    esize = 4 if w.x_dtype == "f32" else 2
+    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+    return w.M * (w.d * esize + packed + 4)
+
+
+def cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, max_rows):
+    """Times the oracle on `rows` tokens: rotate + quantise each row, then its
+    full output row of the quantised product.  Returns (tokens/s, rows, s, threads)."""
+    import numpy as np
+
+    import oracle
+
+    perm, sign = oracle.plan(w.d, w.h, w.plan_seed)
+    ca, ta = oracle.codebook(w.d, w.bits_a)
+    cw, _ = oracle.codebook(w.d, w.bits_w)
+    ca16 = oracle.round_bf16(ca)[1]
+    cw16 = oracle.round_bf16(cw)[1]
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+
+    iw = B.unpack_indices(w_idx_cpu, w.d, w.bits_w).numpy()
+    r64 = w_r_cpu.float().numpy().astype(np.float64)
+
+    def run(rows):
+        xs = x_cpu[:rows].float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        q = oracle.quantize_rows(xs, w.h, perm, sign, ta, decision=32)
+        oracle.qlinear(q["idx"], q["s"], iw, r64, ca16, cw16)
+        return time.perf_counter() - t0
+
+    rows = 2
+    dt = run(rows)
+    while dt < target_s * 0.5 and rows < max_rows:
+        rows = min(max_rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
+        dt = run(rows)
+    return rows / dt, rows, dt, oracle.num_threads()
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on bounded samples."""
+    from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+
+    w = I.WORKLOADS[args.workload]
+    perm, sign = oracle.plan(w.d, w.h, w.plan_seed)
+    ca, ta = oracle.codebook(w.d, w.bits_a)
+    cw, tw = oracle.codebook(w.d, w.bits_w)
+    ca16, cw16 = oracle.round_bf16(ca)[1], oracle.round_bf16(cw)[1]
+    # offline weight pass (untimed): the oracle's own quantisation of W
+    t_w = time.perf_counter()
+    Wq = oracle.quantize_rows(I.make_w(w).float().numpy().astype(np.float64), w.h, perm, sign, tw, decision=32)
+    t_w = time.perf_counter() - t_w
+    rows_per_step = max(1, min(w.M, 8))
+    x = I.make_x(w, rows=np.arange(rows_per_step)).float().numpy().astype(np.float64)
+
+    def step():
+        q = oracle.quantize_rows(x, w.h, perm, sign, ta, decision=32)
+        return oracle.qlinear(q["idx"], q["s"], Wq["idx"], Wq["s"], ca16, cw16)
+
+    t = time.perf_counter()
+    step()
+    one = time.perf_counter() - t
+    budget = 150.0
+    while rows_per_step > 1 and one * (args.steps + args.warmup) > budget:
+        rows_per_step //= 2
+        x = x[:rows_per_step]
+        t = time.perf_counter()
+        step()
+        one = time.perf_counter() - t
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t) / args.steps
+    tok_s = rows_per_step / dt
+    out = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "tokens_per_step": rows_per_step, "M": w.M, "d": w.d, "N": w.N, "h": w.h,
+                      "bits_w": w.bits_w, "bits_a": w.bits_a, "parallelism": "replicas"},
+           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": f"{rows_per_step} tokens per step of {w.name} (rotate+quantise the rows, "
+                                      f"then their full {w.N}-wide output rows); offline weight pass "
+                                      f"{t_w:.1f} s untimed"},
+           "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+    from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CPU oracle is the reference arm: --impl reference)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    B.lib()
+
+    w = I.WORKLOADS[args.workload]
+    x_cpu = I.make_x(w)
+    W_cpu = I.make_w(w)
+    plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
+    cb_a, cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
+    x = x_cpu.to(dev)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W_cpu.to(dev))  # offline pass, untimed
+    ws = torch.empty(B.qlinear_workspace(w.M, w.d, w.bits_a), dtype=torch.uint8, device=dev)
+    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+    a_idx = ws[: w.M * packed].view(w.M, packed)
+    s_off = (w.M * packed + 255) // 256 * 256
+    s = ws[s_off: s_off + 4 * w.M].view(torch.float32)
+    y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
+        B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("start")
+    for i in range(args.steps):
+        flush.zero_()  # cold L2 for every step (outside the events)
+        ev[i][0].record(stream)
+        B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
+        ev[i][1].record(stream)
+        B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler.mark("stop")
+    clocks = sampler.stop()
+    if B.device_status() != 0:
+        raise SystemExit("a kernel reported a timeout")
+
+    t_rpbh = [e[0].elapsed_time(e[1]) for e in ev]
+    t_gemm = [e[1].elapsed_time(e[2]) for e in ev]
+    t_step = [e[0].elapsed_time(e[2]) for e in ev]
+    ms = float(np.mean(t_step))
+    ms_rpbh = float(np.mean(t_rpbh))
+    ms_gemm = float(np.mean(t_gemm))
+    if world > 1:
+        tt = torch.tensor([ms, ms_rpbh, ms_gemm], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, ms_rpbh, ms_gemm = [float(v) for v in tt.tolist()]
+
+    # end to end through the public one-call API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_cpu.pin_memory()
+        y_pin = torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory()
+        ws2 = torch.empty_like(ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for it in range(max(3, args.warmup) + args.steps):
+            if it == max(3, args.warmup):
+                torch.cuda.synchronize()
+                if world > 1:
+                    dist.barrier()
+                e0.record(stream)
+            x.copy_(x_pin, non_blocking=True)
+            B.qlinear(plan, cb_a, cb_w, x, w_idx, w_r, y=y, workspace=ws2, stream=stream)
+            y_pin.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": world * w.M / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(x_cpu.numel() * x_cpu.element_size()),
+               "d2h_bytes_per_step": int(y.numel() * y.element_size()), "ms_per_step": e2e_ms}
+
+    peaks = measured_peaks()
+    flops = 2.0 * w.M * w.N * w.d
+    gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
+    step_tflops = flops / (ms * 1e-3) / 1e12
+    rb = rpbh_bytes(w)
+    rpbh_gbs = rb / (ms_rpbh * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": world * w.M / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "d": w.d, "N": w.N, "h": w.h, "bits_w": w.bits_w,
+                   "bits_a": w.bits_a, "x_dtype": w.x_dtype, "tokens_per_gpu": w.M, "global_batch": world * w.M,
+                   "parallelism": f"dp{world} (replicated packed W, no collective)",
+                   "l2": "flushed (256 MB write) before every timed step, outside the events"},
+        "tflops": step_tflops,
+        "breakdown": {"rpbh_quant_ms": ms_rpbh, "qgemm_ms": ms_gemm, "qgemm_tflops": gemm_tflops,
+                      "rpbh_quant_gbs": rpbh_gbs},
+        "roofline": {"bound": "tensor", "kernel": "qgemm", "achieved": gemm_tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops"],
+                     "traffic": committed_traffic("qgemm", w.name), "peak_source": peaks["source"] + " (burst)",
+                     "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
+        "roofline_rpbh": {"bound": "hbm", "kernel": "rpbh_quant", "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": rpbh_gbs / peaks["hbm_gbs"],
+                          "traffic": committed_traffic("rpbh_quant", w.name),
+                          "algorithmic": f"M*(d*in_bytes + packed + 4) = {rb} B per launch"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, rows, dt, thr = cpu_oracle_sample(w, x_cpu, w_idx.cpu(), w_r.cpu(), args.cpu_seconds, w.M)
+        out["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                               "sample": f"{rows} tokens of {w.name}: rotate+quantise each row, then its full "
+                                         f"{w.N}-wide output row ({dt:.1f} s)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * oq.h -- C ABI of liboq: OrbitQuant-style rotate-then-quantize linear layers
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method: "OrbitQuant" paper summary (hyper.ai, papers 2607.02461), section
+ * 方法 (Method).  A linear layer with input dimension d shares one rotation
+ * Pi_d between its weights and its activations:
+ *   offline:  W' = W Pi_d^T; each row w'_n = r_n * w~'_n with r_n = ||w'_n||_2
+ *             stored as BF16; w~'_n is quantised with the Lloyd-Max codebook
+ *             C_d of b_w bits.
+ *   online:   x' = Pi_d x; s = ||x'||_2; x~' = x' / (s + eps) quantised with
+ *             C_d of b_a bits; y = (W^' x^') with no inverse rotation.
+ *   RPBH:     Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) P_pi.
+ *   C_d:      Lloyd-Max quantiser of the marginal f_d of one coordinate of a
+ *             rotated unit vector, built once per (d, bits), data-free.
+ *
+ * Conventions for every call:
+ *   - Status codes are returned; nothing throws and nothing exits.
+ *   - Tensor buffers are owned by the caller.  "device" pointers must be
+ *     CUDA device memory of the device that is current on the calling
+ *     thread (the device the plan was created on); "host" pointers are
+ *     ordinary host memory.  Device pointers must be 16-byte aligned
+ *     (OQ_ERR_ALIGNMENT otherwise).
+ *   - Plan and codebook handles are owned by the library and released with
+ *     their free functions.  A plan holds device tables on the device that
+ *     was current when it was created.
+ *   - Device work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous: the library never synchronises.
+ *     Launch failures are reported as OQ_ERR_CUDA.  A kernel that gives up a
+ *     bounded wait records OQ_ERR_TIMEOUT in a device flag read by
+ *     oq_device_status().
+ *   - Layouts are row-major.  Packed indices are K-major rows, LSB-first:
+ *     bits = 4: two indices per byte (index k in bits 4*(k%2) of byte k/2);
+ *     bits = 2: four per byte (bits 2*(k%4) of byte k/4);
+ *     bits = 6: one index per byte (low 6 bits).
+ *     Index j means centroid c_j of C_d sorted ascending (0 = most negative).
+ *   - eps = 1e-12 on both the weight and the activation side.
+ */
+#ifndef OQ_H
+#define OQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    OQ_OK = 0,
+    OQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, mismatched handles */
+    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,4,6}, d % 64 != 0 */
+    OQ_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned */
+    OQ_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
+    OQ_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see oq_device_status) */
+    OQ_ERR_OOM = 6,         /* a library-owned allocation failed, or the workspace is too small */
+    OQ_ERR_NO_CONVERGENCE = 7 /* the codebook solver did not converge */
+} oq_status;
+
+typedef enum { OQ_BF16 = 0, OQ_F32 = 1 } oq_dtype;
+
+typedef struct oq_codebook_s oq_codebook_t;
+typedef struct oq_plan_s oq_plan_t;
+
+/* Human-readable name of a status code (static string). */
+const char* oq_status_str(oq_status s);
+
+/* ---------------------------------------------------------------------- */
+/* A0. Codebook C_d  [OrbitQuant, Method: "Lloyd-Max run offline on f_d,   */
+/*     one codebook per dimension"].                                       */
+/* Builds the 2^bits-level Lloyd-Max quantiser of                          */
+/*   f_d(t) = c_d (1 - t^2)^((d-3)/2),  t in [-1, 1]                        */
+/* on the host in fp64 (Newton iteration on the Lloyd-Max conditions, cell */
+/* masses from the regularised incomplete beta function), then derives the */
+/* fp32 thresholds, bf16 centroids and the quantiser lookup table the      */
+/* kernels use.  Host-only: needs no GPU.                                  */
+/*   d    >= 3;  bits in {1..6} (the quantising calls accept {2, 4, 6}).   */
+/*   out  receives a library-owned handle (free with oq_codebook_free).    */
+oq_status oq_codebook(int d, int bits, oq_codebook_t** out);
+
+/* Copies the fp64 codebook: centroids[2^bits] ascending and               */
+/* thresholds[2^bits - 1] (midpoints of adjacent centroids; the middle one */
+/* is exactly 0).  Host pointers; either may be NULL.                       */
+oq_status oq_codebook_values(const oq_codebook_t* cb, double* centroids, double* thresholds);
+
+/* Copies the bf16 bit patterns of the centroids as the product uses them  */
+/* (round-to-nearest-even of the fp64 values).  Host pointer, 2^bits.      */
+oq_status oq_codebook_bf16(const oq_codebook_t* cb, uint16_t* centroids_bf16);
+
+/* (d, bits) of a codebook.  Host pointers; either may be NULL. */
+oq_status oq_codebook_shape(const oq_codebook_t* cb, int* d, int* bits);
+
+void oq_codebook_free(oq_codebook_t* cb);
+
+/* ---------------------------------------------------------------------- */
+/* RPBH plan  [OrbitQuant, Method: Pi_d = blkdiag(H_h D_1..H_h D_{d/h}) P_pi, */
+/*            P_pi a uniformly random permutation, D_i Rademacher signs].   */
+/* pi and the signs come from SplitMix64(seed): a Fisher-Yates shuffle of  */
+/* the identity (i = d-1..1, j = next() mod (i+1)), then d signs           */
+/* sigma_k = (next() >> 63) ? -1 : +1.  (P_pi x)_k = x[pi(k)]; sigma_k     */
+/* multiplies post-permutation coordinate k; H_h is Sylvester-ordered and  */
+/* scaled by 1/sqrt(h).                                                     */
+/*   d % h == 0, h a power of two in [16, 128], d <= 32768.                */
+/* Uploads the plan's gather table to the current device.                  */
+oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out);
+
+/* Host copy of the plan: perm[d] (int32, (P_pi x)_k = x[perm[k]]) and     */
+/* sign[d] (int8, +-1).  Either may be NULL.                               */
+oq_status oq_rpbh_plan_export(const oq_plan_t* plan, int32_t* perm, int8_t* sign);
+
+/* Host-only plan generation (no device tables): same arrays as above. */
+oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign);
+
+/* (d, h) of a plan.  Host pointers; either may be NULL. */
+oq_status oq_plan_shape(const oq_plan_t* plan, int* d, int* h);
+
+void oq_plan_free(oq_plan_t* plan);
+
+/* ---------------------------------------------------------------------- */
+/* Offline weight pass  [OrbitQuant, Method: offline weight stage].         */
+/* Row n of W' = W Pi_d^T is Pi_d w_n, so the same rotate-split-quantise   */
+/* kernel runs on the rows of W:                                            */
+/*   w'_n = Pi_d w_n;  r_n = ||w'_n||_2;  idx = Q_bw(w'_n / (r_n + eps)).   */
+/*   W       device, [N, d] of `dtype` (bf16 or fp32), row-major.          */
+/*   N       rows (> 0).                                                    */
+/*   idx_out device, [N, d*bits/8] bytes (bits 6: [N, d]), packed as above. */
+/*   r_out   device, [N] bf16 bit patterns: r_n rounded to nearest even.    */
+oq_status oq_quantize_weights(const oq_plan_t* plan, const oq_codebook_t* cb_w, const void* W, oq_dtype dtype, int N,
+                              uint8_t* idx_out, uint16_t* r_out, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Online activation pass  [OrbitQuant, Method: online activation stage].  */
+/*   x' = Pi_d x;  s = ||x'||_2 (fp32);  idx = Q_ba(x' / (s + eps)).        */
+/*   x       device, [M, d] of `dtype`, row-major.  M >= 0 (0: no work).    */
+/*   idx_out device, [M, d*bits/8] bytes (bits 6: [M, d]).                  */
+/*   s_out   device, [M] fp32.                                              */
+/* The decision v >= t_j is taken in fp32 (v = x'_k / (s + eps) rounded to */
+/* fp32, t_j the fp32-rounded thresholds).  Rows whose norm is not finite  */
+/* are quantised to the middle cell (index 2^(bits-1)) with s stored as is. */
+oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype, int M,
+                           uint8_t* idx_out, float* s_out, void* stream);
+
+/* Test hook: steps A1-A4 only (permute, sign, block WHT, norm).           */
+/*   x_rot   device, [M, d] fp32: x' = Pi_d x.   norm_out device, [M] fp32. */
+oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, int M, float* x_rot, float* norm_out,
+                        void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Codebook-decode GEMM  [OrbitQuant, Method: W^' x^' ~ W x, no inverse     */
+/* rotation at run time].                                                   */
+/*   y[m, n] = r_n * s_m * sum_k  C_w[iw[n, k]] * C_a[ia[m, k]]  (+ bias_n)  */
+/* with C_w, C_a the bf16 centroid values, fp32 accumulation, bf16 output.  */
+/*   a_idx   device, [M, d*ba/8] packed activation indices; s device [M] f32. */
+/*   w_idx   device, [N, d*bw/8] packed weight indices; w_r device [N] bf16. */
+/*   bias    device [N] bf16 or NULL.   y device [M, N] bf16.              */
+/*   d % 64 == 0; bits_w, bits_a in {2, 4, 6}.  M >= 0, N > 0.              */
+oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                   const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                   void* stream);
+
+/* Bytes of workspace oq_qlinear needs for M rows (packed activation       */
+/* indices plus their norms, 256-byte aligned sections).                   */
+size_t oq_qlinear_workspace(int M, int d, int bits_a);
+
+/* Full layer x -> y: oq_quantize_acts into `workspace`, then oq_qgemm.     */
+/*   x device [M, d] of dtype; w_idx / w_r from oq_quantize_weights with the */
+/*   same plan; workspace device, >= oq_qlinear_workspace(M, d, bits_a)     */
+/*   bytes, 256-byte aligned (OQ_ERR_OOM if too small).  Other arguments as */
+/*   in oq_qgemm.                                                           */
+oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
+                     oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
+                     uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Device status: reads (and, if `clear`, resets) the current device's     */
+/* error flag that kernels set when a bounded wait runs out.  Synchronises */
+/* `stream`.  *out receives OQ_OK or OQ_ERR_TIMEOUT.                        */
+oq_status oq_device_status(int clear, int* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OQ_H */

@@ -1,0 +1,264 @@
+"""Thin ctypes binding over liboq's C ABI (include/oq.h).
+
+Argument marshalling only: every step of the path runs in liboq's kernels.
+PyTorch supplies device memory and streams.  The calls keep the C names
+without the ``oq_`` prefix.  Calls whose output buffers are omitted allocate
+them with torch first (``quantize_acts(plan, cb, x)``).
+
+If liboq.so is missing, the first call raises; there is no other
+implementation behind these functions.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liboq.so")
+
+OQ_OK = 0
+OQ_BF16, OQ_F32 = 0, 1
+_STATUS = {0: "OQ_OK", 1: "OQ_ERR_INVALID_ARG", 2: "OQ_ERR_UNSUPPORTED", 3: "OQ_ERR_ALIGNMENT", 4: "OQ_ERR_CUDA",
+           5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE"}
+
+# every symbol include/oq.h declares
+EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf16", "oq_codebook_shape",
+           "oq_codebook_free", "oq_rpbh_plan", "oq_rpbh_plan_export", "oq_rpbh_plan_host", "oq_plan_shape",
+           "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
+           "oq_qlinear_workspace", "oq_qlinear", "oq_device_status"]
+
+
+class OQError(RuntimeError):
+    def __init__(self, status, call):
+        self.status = status
+        super().__init__(f"{call} failed: {_STATUS.get(status, status)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """Load liboq.so (fails loudly if it was not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"liboq.so not found at {LIB_PATH}; build it with "
+                                       "`python -m rotation_bit_quantization_rpbh_b200.build`")
+                L = ctypes.CDLL(LIB_PATH)
+                P, I, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+                sig = {
+                    "oq_status_str": ([I], ctypes.c_char_p),
+                    "oq_codebook": ([I, I, P], I),
+                    "oq_codebook_values": ([P, P, P], I),
+                    "oq_codebook_bf16": ([P, P], I),
+                    "oq_codebook_shape": ([P, P, P], I),
+                    "oq_codebook_free": ([P], None),
+                    "oq_rpbh_plan": ([I, I, U64, P], I),
+                    "oq_rpbh_plan_export": ([P, P, P], I),
+                    "oq_rpbh_plan_host": ([I, I, U64, P, P], I),
+                    "oq_plan_shape": ([P, P, P], I),
+                    "oq_plan_free": ([P], None),
+                    "oq_quantize_weights": ([P, P, P, I, I, P, P, P], I),
+                    "oq_quantize_acts": ([P, P, P, I, I, P, P, P], I),
+                    "oq_rpbh_apply": ([P, P, I, I, P, P, P], I),
+                    "oq_qgemm": ([P, P, I, I, P, P, P, P, P, P, P], I),
+                    "oq_qlinear_workspace": ([I, I, I], SZ),
+                    "oq_qlinear": ([P, P, P, P, I, I, P, P, I, P, P, P, SZ, P], I),
+                    "oq_device_status": ([I, P, P], I),
+                }
+                for name, (args, res) in sig.items():
+                    f = getattr(L, name)
+                    f.argtypes = args
+                    f.restype = res
+                _lib = L
+    return _lib
+
+
+def _check(status, call):
+    if status != OQ_OK:
+        raise OQError(status, call)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return OQ_BF16
+    if t.dtype == torch.float32:
+        return OQ_F32
+    raise TypeError(f"unsupported input dtype {t.dtype} (bf16 or fp32)")
+
+
+def packed_row_bytes(d, bits):
+    return d if bits == 6 else d * bits // 8
+
+
+class Codebook:
+    """Lloyd-Max codebook C_d (library-owned handle)."""
+
+    def __init__(self, d, bits):
+        h = ctypes.c_void_p()
+        _check(lib().oq_codebook(d, bits, ctypes.byref(h)), "oq_codebook")
+        self._h = h
+        self.d, self.bits, self.L = d, bits, 1 << bits
+
+    @property
+    def handle(self):
+        return self._h
+
+    def values(self):
+        import numpy as np
+
+        c = np.zeros(self.L)
+        t = np.zeros(max(self.L - 1, 1))
+        _check(lib().oq_codebook_values(self._h, c.ctypes.data_as(ctypes.c_void_p),
+                                        t.ctypes.data_as(ctypes.c_void_p)), "oq_codebook_values")
+        return c, t[: self.L - 1]
+
+    def bf16_bits(self):
+        import numpy as np
+
+        b = np.zeros(self.L, dtype=np.uint16)
+        _check(lib().oq_codebook_bf16(self._h, b.ctypes.data_as(ctypes.c_void_p)), "oq_codebook_bf16")
+        return b
+
+    def __del__(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.oq_codebook_free(self._h)
+            self._h = None
+
+
+class Plan:
+    """RPBH plan (library-owned handle with device tables on the current device)."""
+
+    def __init__(self, d, h, seed):
+        hp = ctypes.c_void_p()
+        _check(lib().oq_rpbh_plan(d, h, ctypes.c_uint64(seed), ctypes.byref(hp)), "oq_rpbh_plan")
+        self._h = hp
+        self.d, self.h, self.seed = d, h, seed
+
+    @property
+    def handle(self):
+        return self._h
+
+    def export(self):
+        import numpy as np
+
+        perm = np.zeros(self.d, dtype=np.int32)
+        sign = np.zeros(self.d, dtype=np.int8)
+        _check(lib().oq_rpbh_plan_export(self._h, perm.ctypes.data_as(ctypes.c_void_p),
+                                         sign.ctypes.data_as(ctypes.c_void_p)), "oq_rpbh_plan_export")
+        return perm, sign
+
+    def __del__(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.oq_plan_free(self._h)
+            self._h = None
+
+
+def codebook(d, bits):
+    return Codebook(d, bits)
+
+
+def rpbh_plan(d, h, seed):
+    return Plan(d, h, seed)
+
+
+def rpbh_plan_host(d, h, seed):
+    import numpy as np
+
+    perm = np.zeros(d, dtype=np.int32)
+    sign = np.zeros(d, dtype=np.int8)
+    _check(lib().oq_rpbh_plan_host(d, h, ctypes.c_uint64(seed), perm.ctypes.data_as(ctypes.c_void_p),
+                                   sign.ctypes.data_as(ctypes.c_void_p)), "oq_rpbh_plan_host")
+    return perm, sign
+
+
+def quantize_weights(plan, cb_w, W, idx_out=None, r_out=None, stream=None):
+    N, d = W.shape
+    if idx_out is None:
+        idx_out = torch.empty((N, packed_row_bytes(d, cb_w.bits)), dtype=torch.uint8, device=W.device)
+    if r_out is None:
+        r_out = torch.empty(N, dtype=torch.bfloat16, device=W.device)
+    _check(lib().oq_quantize_weights(plan.handle, cb_w.handle, _ptr(W), _dtype_code(W), N, _ptr(idx_out),
+                                     _ptr(r_out), _stream(stream)), "oq_quantize_weights")
+    return idx_out, r_out
+
+
+def quantize_acts(plan, cb_a, x, idx_out=None, s_out=None, stream=None):
+    M, d = x.shape
+    if idx_out is None:
+        idx_out = torch.empty((M, packed_row_bytes(d, cb_a.bits)), dtype=torch.uint8, device=x.device)
+    if s_out is None:
+        s_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().oq_quantize_acts(plan.handle, cb_a.handle, _ptr(x), _dtype_code(x), M, _ptr(idx_out), _ptr(s_out),
+                                  _stream(stream)), "oq_quantize_acts")
+    return idx_out, s_out
+
+
+def rpbh_apply(plan, x, x_rot=None, norm_out=None, stream=None):
+    M, d = x.shape
+    if x_rot is None:
+        x_rot = torch.empty((M, d), dtype=torch.float32, device=x.device)
+    if norm_out is None:
+        norm_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().oq_rpbh_apply(plan.handle, _ptr(x), _dtype_code(x), M, _ptr(x_rot), _ptr(norm_out),
+                               _stream(stream)), "oq_rpbh_apply")
+    return x_rot, norm_out
+
+
+def qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
+    M, N = a_idx.shape[0], w_idx.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_idx.device)
+    _check(lib().oq_qgemm(cb_a.handle, cb_w.handle, M, N, _ptr(a_idx), _ptr(s), _ptr(w_idx), _ptr(w_r), _ptr(bias),
+                          _ptr(y), _stream(stream)), "oq_qgemm")
+    return y
+
+
+def qlinear_workspace(M, d, bits_a):
+    return int(lib().oq_qlinear_workspace(M, d, bits_a))
+
+
+def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None):
+    M, d = x.shape
+    N = w_idx.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = qlinear_workspace(M, d, cb_a.bits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(lib().oq_qlinear(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
+                            _ptr(w_r), N, _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "oq_qlinear")
+    return y
+
+
+def device_status(clear=True, stream=None):
+    out = ctypes.c_int(0)
+    _check(lib().oq_device_status(int(clear), ctypes.byref(out), _stream(stream)), "oq_device_status")
+    return out.value
+
+
+def unpack_indices(packed, d, bits):
+    """Unpack LSB-first packed indices [rows, bytes] to one index per byte
+    [rows, d] (a layout conversion for tests and callers, on any device)."""
+    p = packed.to(torch.int32)
+    if bits == 6:
+        return (p & 63).to(torch.uint8)
+    per = 8 // bits
+    shifts = torch.arange(per, device=p.device, dtype=torch.int32) * bits
+    v = (p.unsqueeze(-1) >> shifts) & ((1 << bits) - 1)
+    return v.reshape(p.shape[0], -1)[:, :d].to(torch.uint8)

@@ -1,0 +1,341 @@
+// C ABI of liboq (declared in include/oq.h): argument checks, handle
+// management, lazy per-device uploads and kernel dispatch.
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <new>
+
+#include "device_util.cuh"
+#include "oq_internal.h"
+#include "qgemm.cuh"
+#include "rpbh_quant.cuh"
+
+namespace oq {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int device_sms() {
+    static int count[kMaxDevices] = {0};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+    return count[dev] > 0 ? count[dev] : 148;
+}
+
+bool quant_bits_ok(int bits) { return bits == 2 || bits == 4 || bits == 6; }
+
+int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }
+
+// Launch the fused rotate/quantise kernel in one of its three modes.
+oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_dtype dtype, int M, int mode,
+                   uint8_t* idx_out, float* s_out, uint16_t* r_out, float* y_out, float* norm_out, cudaStream_t st) {
+    if (!plan || !x || M < 0) return OQ_ERR_INVALID_ARG;
+    if (dtype != OQ_BF16 && dtype != OQ_F32) return OQ_ERR_INVALID_ARG;
+    if (mode != 2) {
+        if (!cb || !idx_out) return OQ_ERR_INVALID_ARG;
+        if (cb->d != plan->d) return OQ_ERR_INVALID_ARG;
+        if (!quant_bits_ok(cb->bits)) return OQ_ERR_UNSUPPORTED;
+        if (packed_row_bytes(plan->d, cb->bits) % 4 != 0) return OQ_ERR_UNSUPPORTED;
+        if (!aligned16(idx_out)) return OQ_ERR_ALIGNMENT;
+    }
+    if (mode == 0 && (!s_out || !aligned16(s_out))) return s_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
+    if (mode == 1 && (!r_out || !aligned16(r_out))) return r_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
+    if (mode == 2 && (!y_out || !norm_out)) return OQ_ERR_INVALID_ARG;
+    if (mode == 2 && (!aligned16(y_out) || !aligned16(norm_out))) return OQ_ERR_ALIGNMENT;
+    if (!aligned16(x)) return OQ_ERR_ALIGNMENT;
+    if (current_device() != plan->device) return OQ_ERR_INVALID_ARG;
+    if (M == 0) return OQ_OK;
+
+    const DeviceCodebook* dcb = nullptr;
+    if (mode != 2) {
+        oq_status s = codebook_device(cb, &dcb);
+        if (s != OQ_OK) return s;
+    }
+    const int d = plan->d, h = plan->h, nb = d / h;
+    const int esize = dtype == OQ_BF16 ? 2 : 4;
+    RpbhParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = x;
+    p.M = M;
+    p.d = d;
+    p.nb = nb;
+    p.row_bytes = d * esize;
+    p.srow = d * esize + 16;
+    int R = 1;
+    while (R < 32 && 2 * R * nb <= 256 && 2 * (2 * R) * p.srow <= 160 * 1024) R *= 2;
+    p.R = R;
+    p.T = (nb * R + 31) / 32 * 32;
+    if (p.T > 1024) return OQ_ERR_UNSUPPORTED;
+    p.ntiles = (M + R - 1) / R;
+    p.gtab = plan->dev.gtab;
+    if (mode != 2) {
+        p.lut = dcb->lut;
+        p.lut_n = (int)cb->lut.size();
+        p.lut_off = -(int)kLutMagicBits - cb->kmin;
+        p.G = cb->G;
+        p.L = cb->L;
+        p.out_row_bytes = packed_row_bytes(d, cb->bits);
+    }
+    p.idx_out = idx_out;
+    p.s_out = s_out;
+    p.r_out = r_out;
+    p.y_out = y_out;
+    p.norm_out = norm_out;
+    p.rsqrt_h = (float)(1.0 / std::sqrt((double)h));
+    p.eps_h = (float)(kEps * std::sqrt((double)h));
+    if (rpbh_smem_bytes(p) > 227 * 1024) return OQ_ERR_UNSUPPORTED;
+    const int grid = p.ntiles < device_sms() ? p.ntiles : device_sms();
+    cudaError_t e = launch_rpbh_quant(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, grid, st);
+    return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
+}
+
+}  // namespace
+
+oq_status codebook_device(oq_codebook_t* cb, const DeviceCodebook** out) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return OQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(cb->mu);
+    DeviceCodebook& dc = cb->dev[dev];
+    if (!dc.lut) {
+        void* ptr = nullptr;
+        const size_t bytes = cb->lut.size() * sizeof(LutEntry);
+        if (cudaMalloc(&ptr, bytes) != cudaSuccess) return OQ_ERR_OOM;
+        if (cudaMemcpy(ptr, cb->lut.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+            cudaFree(ptr);
+            return OQ_ERR_CUDA;
+        }
+        dc.lut = static_cast<LutEntry*>(ptr);
+    }
+    *out = &dc;
+    return OQ_OK;
+}
+
+}  // namespace oq
+
+using namespace oq;
+
+extern "C" {
+
+const char* oq_status_str(oq_status s) {
+    switch (s) {
+        case OQ_OK: return "OQ_OK";
+        case OQ_ERR_INVALID_ARG: return "OQ_ERR_INVALID_ARG";
+        case OQ_ERR_UNSUPPORTED: return "OQ_ERR_UNSUPPORTED";
+        case OQ_ERR_ALIGNMENT: return "OQ_ERR_ALIGNMENT";
+        case OQ_ERR_CUDA: return "OQ_ERR_CUDA";
+        case OQ_ERR_TIMEOUT: return "OQ_ERR_TIMEOUT";
+        case OQ_ERR_OOM: return "OQ_ERR_OOM";
+        case OQ_ERR_NO_CONVERGENCE: return "OQ_ERR_NO_CONVERGENCE";
+    }
+    return "OQ_ERR_UNKNOWN";
+}
+
+oq_status oq_codebook(int d, int bits, oq_codebook_t** out) {
+    if (!out) return OQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (d < 3 || bits < 1 || bits > 6) return OQ_ERR_UNSUPPORTED;
+    oq_codebook_t* cb = new (std::nothrow) oq_codebook_s();
+    if (!cb) return OQ_ERR_OOM;
+    oq_status s = build_codebook(d, bits, cb);
+    if (s != OQ_OK) {
+        delete cb;
+        return s;
+    }
+    *out = cb;
+    return OQ_OK;
+}
+
+oq_status oq_codebook_values(const oq_codebook_t* cb, double* centroids, double* thresholds) {
+    if (!cb) return OQ_ERR_INVALID_ARG;
+    if (centroids) std::memcpy(centroids, cb->c.data(), sizeof(double) * cb->L);
+    if (thresholds) std::memcpy(thresholds, cb->t.data(), sizeof(double) * (cb->L - 1));
+    return OQ_OK;
+}
+
+oq_status oq_codebook_bf16(const oq_codebook_t* cb, uint16_t* centroids_bf16) {
+    if (!cb || !centroids_bf16) return OQ_ERR_INVALID_ARG;
+    std::memcpy(centroids_bf16, cb->c_bf16.data(), sizeof(uint16_t) * cb->L);
+    return OQ_OK;
+}
+
+oq_status oq_codebook_shape(const oq_codebook_t* cb, int* d, int* bits) {
+    if (!cb) return OQ_ERR_INVALID_ARG;
+    if (d) *d = cb->d;
+    if (bits) *bits = cb->bits;
+    return OQ_OK;
+}
+
+void oq_codebook_free(oq_codebook_t* cb) {
+    if (!cb) return;
+    for (int i = 0; i < kMaxDevices; ++i)
+        if (cb->dev[i].lut) cudaFree(cb->dev[i].lut);
+    delete cb;
+}
+
+static oq_status check_plan_args(int d, int h) {
+    if (d <= 0 || h <= 0) return OQ_ERR_INVALID_ARG;
+    if ((h & (h - 1)) != 0 || h < 16 || h > 128 || d % h != 0 || d > 32767 || d % 8 != 0) return OQ_ERR_UNSUPPORTED;
+    return OQ_OK;
+}
+
+oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign) {
+    oq_status s = check_plan_args(d, h);
+    if (s != OQ_OK) return s;
+    std::vector<int32_t> pv(d);
+    std::vector<int8_t> sv(d);
+    make_plan(d, h, seed, pv.data(), sv.data());
+    if (perm) std::memcpy(perm, pv.data(), sizeof(int32_t) * d);
+    if (sign) std::memcpy(sign, sv.data(), d);
+    return OQ_OK;
+}
+
+oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out) {
+    if (!out) return OQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    oq_status s = check_plan_args(d, h);
+    if (s != OQ_OK) return s;
+    const int dev = current_device();
+    if (dev < 0) return OQ_ERR_CUDA;
+    oq_plan_t* p = new (std::nothrow) oq_plan_s();
+    if (!p) return OQ_ERR_OOM;
+    p->d = d;
+    p->h = h;
+    p->seed = seed;
+    p->device = dev;
+    p->perm.resize(d);
+    p->sign.resize(d);
+    make_plan(d, h, seed, p->perm.data(), p->sign.data());
+    build_gather_table(p, p->gtab_host);
+    void* ptr = nullptr;
+    if (cudaMalloc(&ptr, sizeof(uint16_t) * d) != cudaSuccess) {
+        delete p;
+        return OQ_ERR_OOM;
+    }
+    if (cudaMemcpy(ptr, p->gtab_host.data(), sizeof(uint16_t) * d, cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(ptr);
+        delete p;
+        return OQ_ERR_CUDA;
+    }
+    p->dev.gtab = static_cast<uint16_t*>(ptr);
+    *out = p;
+    return OQ_OK;
+}
+
+oq_status oq_rpbh_plan_export(const oq_plan_t* plan, int32_t* perm, int8_t* sign) {
+    if (!plan) return OQ_ERR_INVALID_ARG;
+    if (perm) std::memcpy(perm, plan->perm.data(), sizeof(int32_t) * plan->d);
+    if (sign) std::memcpy(sign, plan->sign.data(), plan->d);
+    return OQ_OK;
+}
+
+oq_status oq_plan_shape(const oq_plan_t* plan, int* d, int* h) {
+    if (!plan) return OQ_ERR_INVALID_ARG;
+    if (d) *d = plan->d;
+    if (h) *h = plan->h;
+    return OQ_OK;
+}
+
+void oq_plan_free(oq_plan_t* plan) {
+    if (!plan) return;
+    if (plan->dev.gtab) cudaFree(plan->dev.gtab);
+    delete plan;
+}
+
+oq_status oq_quantize_weights(const oq_plan_t* plan, const oq_codebook_t* cb_w, const void* W, oq_dtype dtype, int N,
+                              uint8_t* idx_out, uint16_t* r_out, void* stream) {
+    if (N <= 0) return OQ_ERR_INVALID_ARG;
+    return run_rpbh(plan, const_cast<oq_codebook_t*>(cb_w), W, dtype, N, 1, idx_out, nullptr, r_out, nullptr, nullptr,
+                    static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype, int M,
+                           uint8_t* idx_out, float* s_out, void* stream) {
+    return run_rpbh(plan, const_cast<oq_codebook_t*>(cb_a), x, dtype, M, 0, idx_out, s_out, nullptr, nullptr, nullptr,
+                    static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, int M, float* x_rot, float* norm_out,
+                        void* stream) {
+    return run_rpbh(plan, nullptr, x, dtype, M, 2, nullptr, nullptr, nullptr, x_rot, norm_out,
+                    static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                   const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                   void* stream) {
+    if (!cb_a || !cb_w || !a_idx || !s || !w_idx || !w_r || !y || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
+    if (cb_a->d != cb_w->d) return OQ_ERR_INVALID_ARG;
+    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % 64 != 0) return OQ_ERR_UNSUPPORTED;
+    if (!aligned16(a_idx) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
+        (bias && !aligned16(bias)))
+        return OQ_ERR_ALIGNMENT;
+    if (M == 0) return OQ_OK;
+    QgemmArgs a;
+    a.M = M;
+    a.N = N;
+    a.K = cb_a->d;
+    a.bits_a = cb_a->bits;
+    a.bits_w = cb_w->bits;
+    a.a_idx = a_idx;
+    a.w_idx = w_idx;
+    a.s = s;
+    a.w_r = w_r;
+    a.bias = bias;
+    a.y = y;
+    a.ca_bf16 = cb_a->c_bf16.data();
+    a.cw_bf16 = cb_w->c_bf16.data();
+    cudaError_t e = launch_qgemm(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
+}
+
+size_t oq_qlinear_workspace(int M, int d, int bits_a) {
+    if (M <= 0 || d <= 0 || !quant_bits_ok(bits_a)) return 0;
+    const size_t idx = (size_t)M * (size_t)packed_row_bytes(d, bits_a);
+    const size_t idx_al = (idx + 255) / 256 * 256;
+    return idx_al + ((size_t)M * sizeof(float) + 255) / 256 * 256;
+}
+
+oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
+                     oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
+                     uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+    if (!plan || !cb_a || !cb_w || !workspace) return OQ_ERR_INVALID_ARG;
+    if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
+    if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
+    if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
+    if (M == 0) return OQ_OK;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return OQ_ERR_ALIGNMENT;
+    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
+    if (ws_bytes < need) return OQ_ERR_OOM;
+    uint8_t* a_idx = static_cast<uint8_t*>(workspace);
+    const size_t idx_al = ((size_t)M * packed_row_bytes(plan->d, cb_a->bits) + 255) / 256 * 256;
+    float* s = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + idx_al);
+    oq_status st = oq_quantize_acts(plan, cb_a, x, dtype, M, a_idx, s, stream);
+    if (st != OQ_OK) return st;
+    return oq_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream);
+}
+
+oq_status oq_device_status(int clear, int* out, void* stream) {
+    if (!out) return OQ_ERR_INVALID_ARG;
+    int v = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyFromSymbolAsync(&v, g_error_flag, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return OQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return OQ_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbolAsync(g_error_flag, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return OQ_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return OQ_ERR_CUDA;
+    }
+    *out = v ? OQ_ERR_TIMEOUT : OQ_OK;
+    return OQ_OK;
+}
+
+}  // extern "C"

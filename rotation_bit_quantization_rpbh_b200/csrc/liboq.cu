@@ -1,0 +1,5 @@
+// Single translation unit for the device side of liboq, so that the kernels
+// and the C ABI share the device error flag without relocatable device code.
+#include "rpbh_quant.cu"
+#include "qgemm.cu"
+#include "api.cu"

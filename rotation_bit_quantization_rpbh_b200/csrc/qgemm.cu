@@ -1,0 +1,524 @@
+// Codebook-decode GEMM on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Method: "OrbitQuant" paper summary (hyper.ai, papers 2607.02461), section
+// 方法 (Method): W^' = diag(r') Q_bw(W~'), x^' = s Q_ba(x~'), and the layer
+// computes W^' x^' ~ W x with no inverse rotation.  Per output element
+//   y[m, n] = r_n * s_m * sum_k C_w[iw[n, k]] * C_a[ia[m, k]]
+// with the centroids taken as bf16 values, fp32 accumulation, bf16 output.
+//
+// Structure (one persistent CTA per SM, 128 x 256 output tiles, K step 64):
+//   warp 0      TMA producer: 2-D tensor loads of the packed index tiles
+//               (A: 128 rows, W: 256 rows) into a 4-stage ring;
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32
+//               accumulators) and issues tcgen05.mma (one thread);
+//   warps 2-9   decoders: expand each packed tile to bf16 centroid values
+//               (register byte-permute lookups; 6-bit codes via a 64-entry
+//               shared table) and write them in the canonical 128-byte
+//               swizzled K-major layout the MMA descriptors name;
+//   warps 10-13 epilogue: tcgen05.ld of the accumulator, scale by s_m r_n
+//               (+ bias) in fp32, round to bf16, store.
+// Every mbarrier wait is bounded: on a timeout the kernel raises the device
+// error flag, drains its own TMA loads and frees its TMEM before returning.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "device_util.cuh"
+#include "qgemm.cuh"
+
+namespace oq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int P_MAX = 4;     // packed ring depth (3 when the packed stage is large)
+constexpr int D_STAGES = 3;  // decoded ring
+constexpr int NDEC_WARPS = 8;
+constexpr int NTHREADS = (2 + NDEC_WARPS + 4) * 32;
+constexpr int DEC_A = BM * 128, DEC_B = BN * 128, DEC_STAGE = DEC_A + DEC_B;
+
+__host__ __device__ constexpr int pk_row_bytes(int bits) { return bits == 6 ? BK : BK * bits / 8; }
+__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw) { return BM * pk_row_bytes(ba) + BN * pk_row_bytes(bw); }
+__host__ __device__ constexpr int p_stages(int ba, int bw) {
+    return D_STAGES * DEC_STAGE + P_MAX * pk_stage_bytes(ba, bw) + 2048 <= 227 * 1024 ? P_MAX : P_MAX - 1;
+}
+
+struct QgemmParams {
+    CUtensorMap tmA;
+    CUtensorMap tmB;
+    int M, N, KB, num_m, num_tiles;
+    const float* s;
+    const uint16_t* w_r;
+    const uint16_t* bias;
+    uint16_t* y;
+    uint32_t tab_a[4], tab_w[4];  // 4-bit path: magnitude hi bytes (2 words), lo bytes (2 words)
+    uint16_t c6a[64], c6w[64];    // 6-bit path tables
+};
+
+// ----------------------------------------------------------------------------
+// tcgen05 / TMA wrappers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), version 1 (sm_100), leading offset unused (1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)1u << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major,
+// M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+#define OQ_TMEM_LD32(taddr, v)                                                                                        \
+    asm volatile(                                                                                                     \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19," \
+        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                                    \
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), \
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),     \
+          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),    \
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])                 \
+        : "r"(taddr))
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Bounded wait that also gives up when another role has already aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicExch(&g_error_flag, kErrTimeout);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// ----------------------------------------------------------------------------
+// Decoding packed indices to bf16 centroid values.
+// The codebooks are symmetric (c_{L-1-j} = -c_j), so a 4-bit index j maps to
+// magnitude m = (j & 7) ^ (j < 8 ? 7 : 0) of the positive half and a sign.
+// One byte-permute picks the 4 high bytes, one the 4 low bytes, a third
+// (with its sign-replicate mode) marks the negative lanes.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint4 decode8_nibbles(uint32_t w, const uint32_t tab[4]) {
+    const uint32_t S = (w >> 3) & 0x11111111u;                  // bit 3 of each nibble (1: upper half)
+    const uint32_t mw = ~(w ^ (S * 7u)) & 0x77777777u;           // magnitude index per nibble
+    uint32_t out[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint32_t sel = half ? (mw >> 16) : mw;
+        const uint32_t wh = half ? (w >> 16) : w;
+        uint32_t hi = prmt(tab[0], tab[1], sel);
+        const uint32_t lo = prmt(tab[2], tab[3], sel);
+        const uint32_t neg = prmt(0x7f7f7f7fu, 0x7f7f7f7fu, wh);  // 0x7f where j < 8, 0x00 where j >= 8
+        hi ^= (neg << 7) & 0x80808080u;
+        out[2 * half] = prmt(lo, hi, 0x5140u);
+        out[2 * half + 1] = prmt(lo, hi, 0x7362u);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// 2-bit codes: spread each 2-bit field into a nibble and offset it by 6, so
+// codes 0..3 land on entries 6..9 of a symmetric 16-entry table whose middle
+// four entries are the 4-level codebook.
+__device__ __forceinline__ uint4 decode8_2bit(uint32_t w16, const uint32_t tab[4]) {
+    uint32_t x = w16 & 0xffffu;
+    x = (x | (x << 8)) & 0x00ff00ffu;
+    x = (x | (x << 4)) & 0x0f0f0f0fu;
+    x = (x | (x << 2)) & 0x33333333u;
+    return decode8_nibbles(x + 0x66666666u, tab);
+}
+
+__device__ __forceinline__ uint4 decode8_6bit(uint2 w, const uint16_t* tab) {
+    const uint32_t a = w.x, b = w.y;
+    const uint32_t e0 = tab[a & 63], e1 = tab[(a >> 8) & 63], e2 = tab[(a >> 16) & 63], e3 = tab[(a >> 24) & 63];
+    const uint32_t e4 = tab[b & 63], e5 = tab[(b >> 8) & 63], e6 = tab[(b >> 16) & 63], e7 = tab[(b >> 24) & 63];
+    return make_uint4(e0 | (e1 << 16), e2 | (e3 << 16), e4 | (e5 << 16), e6 | (e7 << 16));
+}
+
+template <int BITS>
+__device__ __forceinline__ uint4 decode_unit(const uint8_t* src, const uint32_t tab[4], const uint16_t* tab6) {
+    if constexpr (BITS == 4) return decode8_nibbles(*reinterpret_cast<const uint32_t*>(src), tab);
+    else if constexpr (BITS == 2) return decode8_2bit(*reinterpret_cast<const uint16_t*>(src), tab);
+    else return decode8_6bit(*reinterpret_cast<const uint2*>(src), tab6);
+}
+
+// Decode a ROWS x 64 tile: unit u = (row, chunk of 8 codes), written to the
+// 128-byte-swizzled K-major position (chunk ^ (row & 7)).
+template <int BITS, int ROWS>
+__device__ __forceinline__ void decode_tile(const uint8_t* pk, uint8_t* dst, int t, const uint32_t tab[4],
+                                            const uint16_t* tab6) {
+    constexpr int UB = BITS == 6 ? 8 : BITS;  // packed bytes per 8 codes
+#pragma unroll 4
+    for (int u = t; u < ROWS * 8; u += NDEC_WARPS * 32) {
+        const int row = u >> 3, c = u & 7;
+        const uint4 v = decode_unit<BITS>(pk + row * pk_row_bytes(BITS) + c * UB, tab, tab6);
+        *reinterpret_cast<uint4*>(dst + (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4)) = v;
+    }
+}
+
+// ----------------------------------------------------------------------------
+template <int BA, int BW>
+__global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constant__ QgemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int PKA = BM * pk_row_bytes(BA);
+    constexpr int PK_STAGE = pk_stage_bytes(BA, BW);
+    constexpr int P_STAGES = p_stages(BA, BW);
+    uint8_t* dec = smem;
+    uint8_t* pk = smem + D_STAGES * DEC_STAGE;
+    uint16_t* t6 = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(t6 + 128);
+    uint64_t* pk_full = bars;
+    uint64_t* pk_empty = bars + P_STAGES;
+    uint64_t* dec_full = bars + 2 * P_STAGES;
+    uint64_t* dec_empty = dec_full + D_STAGES;
+    uint64_t* acc_full = dec_empty + D_STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int i = 0; i < P_STAGES; ++i) {
+            mbar_init(&pk_full[i], 1);
+            mbar_init(&pk_empty[i], NDEC_WARPS);
+        }
+        for (int i = 0; i < D_STAGES; ++i) {
+            mbar_init(&dec_full[i], NDEC_WARPS);
+            mbar_init(&dec_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (tid < 64) t6[tid] = p.c6a[tid];
+    else if (tid < 128) t6[tid] = p.c6w[tid - 64];
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512u));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            int step = 0;
+            int last_step[P_MAX];
+            for (int i = 0; i < P_STAGES; ++i) last_step[i] = -1;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+                const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+                for (int kb = 0; kb < p.KB; ++kb, ++step) {
+                    const int s = step % P_STAGES;
+                    if (!wait_or_abort(&pk_empty[s], ((step / P_STAGES) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&pk_full[s], PK_STAGE);
+                    uint8_t* dst = pk + s * PK_STAGE;
+                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA), m0, &pk_full[s]);
+                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW), n0, &pk_full[s]);
+                    last_step[s] = step;
+                }
+            }
+            // the loads this thread issued must land before shared memory goes away
+            for (int i = 0; i < P_STAGES; ++i)
+                if (last_step[i] >= 0) mbar_wait_bounded(&pk_full[i], (last_step[i] / P_STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            int step = 0, acc_it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++acc_it) {
+                const int a = acc_it & 1;
+                if (!wait_or_abort(&acc_empty[a], ((acc_it >> 1) & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+                for (int kb = 0; kb < p.KB; ++kb, ++step) {
+                    const int ds = step % D_STAGES;
+                    if (!wait_or_abort(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(dec + ds * DEC_STAGE), b_base = a_base + DEC_A;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k), kIdesc,
+                               (kb | k) != 0 ? 1u : 0u);
+                    tc_commit(&dec_empty[ds]);
+                }
+                if (ok) tc_commit(&acc_full[a]);
+            }
+        }
+    } else if (warp < 2 + NDEC_WARPS) {
+        // ------------------------------ decoders ----------------------------------
+        const int t = tid - 64;
+        int step = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+            for (int kb = 0; kb < p.KB; ++kb, ++step) {
+                const int ps = step % P_STAGES, ds = step % D_STAGES;
+                if (!wait_or_abort(&pk_full[ps], (step / P_STAGES) & 1, abort_flag) ||
+                    !wait_or_abort(&dec_empty[ds], ((step / D_STAGES) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* pa = pk + ps * PK_STAGE;
+                uint8_t* da = dec + ds * DEC_STAGE;
+                decode_tile<BA, BM>(pa, da, t, p.tab_a, t6);
+                decode_tile<BW, BN>(pa + PKA, da + DEC_A, t, p.tab_w, t6 + 64);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&pk_empty[ps]);
+                    mbar_arrive(&dec_full[ds]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ----------------------------------
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        int acc_it = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++acc_it) {
+            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            const int a = acc_it & 1;
+            if (!wait_or_abort(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const int row = m0 + q * 32 + lane;
+            const bool row_ok = row < p.M;
+            const float sm = row_ok ? p.s[row] : 0.f;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                OQ_TMEM_LD32(taddr + c0, v);
+                tmem_wait_ld();
+                const int n = n0 + c0;
+                if (row_ok && n < p.N) {
+                    uint16_t* yrow = p.y + (size_t)row * p.N + n;
+                    if (n + 32 <= p.N) {
+                        uint32_t rr[16];
+                        const uint4* rp = reinterpret_cast<const uint4*>(p.w_r + n);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 t4 = __ldg(rp + i);
+                            rr[4 * i] = t4.x;
+                            rr[4 * i + 1] = t4.y;
+                            rr[4 * i + 2] = t4.z;
+                            rr[4 * i + 3] = t4.w;
+                        }
+                        uint32_t bb[16];
+                        if (p.bias) {
+                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint4 t4 = __ldg(bp + i);
+                                bb[4 * i] = t4.x;
+                                bb[4 * i + 1] = t4.y;
+                                bb[4 * i + 2] = t4.z;
+                                bb[4 * i + 3] = t4.w;
+                            }
+                        }
+                        uint32_t o[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float r0 = __uint_as_float(rr[j] << 16), r1 = __uint_as_float(rr[j] & 0xffff0000u);
+                            float y0 = __uint_as_float(v[2 * j]) * sm * r0;
+                            float y1 = __uint_as_float(v[2 * j + 1]) * sm * r1;
+                            if (p.bias) {
+                                y0 += __uint_as_float(bb[j] << 16);
+                                y1 += __uint_as_float(bb[j] & 0xffff0000u);
+                            }
+                            o[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
+                                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y1)) << 16);
+                        }
+                        if ((p.N & 7) == 0) {
+                            uint4* yp = reinterpret_cast<uint4*>(yrow);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) yp[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                yrow[2 * j] = (uint16_t)(o[j] & 0xffffu);
+                                yrow[2 * j + 1] = (uint16_t)(o[j] >> 16);
+                            }
+                        }
+                    } else {
+                        for (int j = 0; j < 32 && n + j < p.N; ++j) {
+                            float yv = __uint_as_float(v[j]) * sm * __uint_as_float((uint32_t)p.w_r[n + j] << 16);
+                            if (p.bias) yv += __uint_as_float((uint32_t)p.bias[n + j] << 16);
+                            yrow[j] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u));
+    }
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 4-bit-path tables from a symmetric 16-entry bf16 codebook c16 (c16[8+m] =
+// magnitude m): high bytes of magnitudes 0..7, then low bytes.
+void nibble_tables(const uint16_t* c16, uint32_t tab[4]) {
+    tab[0] = tab[1] = tab[2] = tab[3] = 0;
+    for (int m = 0; m < 8; ++m) {
+        const uint32_t v = c16[8 + m];
+        tab[m / 4] |= ((v >> 8) & 0xffu) << (8 * (m % 4));
+        tab[2 + m / 4] |= (v & 0xffu) << (8 * (m % 4));
+    }
+}
+
+void fill_tables(int bits, const uint16_t* cb, uint32_t tab[4], uint16_t* c6) {
+    uint16_t c16[16] = {0};
+    std::memset(c6, 0, 64 * sizeof(uint16_t));
+    if (bits == 4) {
+        for (int j = 0; j < 16; ++j) c16[j] = cb[j];
+    } else if (bits == 2) {
+        for (int j = 0; j < 4; ++j) c16[6 + j] = cb[j];
+    } else {
+        for (int j = 0; j < 64; ++j) c6[j] = cb[j];
+    }
+    nibble_tables(c16, tab);
+}
+
+template <int BA, int BW>
+cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
+    auto k = qgemm_kernel<BA, BW>;
+    const int smem = D_STAGES * DEC_STAGE + p_stages(BA, BW) * pk_stage_bytes(BA, BW) + 256 + 256 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, NTHREADS, smem, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+int qgemm_sm_count() {
+    static int count[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+    return count[dev] > 0 ? count[dev] : 148;
+}
+
+}  // namespace
+
+cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
+    QgemmParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a), BM) ||
+        !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w), BN))
+        return cudaErrorInvalidValue;
+    prm.M = a.M;
+    prm.N = a.N;
+    prm.KB = a.K / BK;
+    prm.num_m = (a.M + BM - 1) / BM;
+    prm.num_tiles = prm.num_m * ((a.N + BN - 1) / BN);
+    prm.s = a.s;
+    prm.w_r = a.w_r;
+    prm.bias = a.bias;
+    prm.y = a.y;
+    fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
+    fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
+    const int grid = prm.num_tiles < qgemm_sm_count() ? prm.num_tiles : qgemm_sm_count();
+#define OQ_CASE(X, Y) \
+    if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y>(prm, grid, stream);
+    OQ_CASE(4, 4)
+    OQ_CASE(4, 2)
+    OQ_CASE(6, 4)
+    OQ_CASE(2, 2)
+    OQ_CASE(2, 4)
+    OQ_CASE(4, 6)
+    OQ_CASE(6, 2)
+    OQ_CASE(2, 6)
+    OQ_CASE(6, 6)
+#undef OQ_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace oq

@@ -1,0 +1,305 @@
+// Fused RPBH rotate -> norm/direction split -> Lloyd-Max quantise -> pack.
+//
+// Method: "OrbitQuant" paper summary (hyper.ai, papers 2607.02461), section
+// 方法 (Method):
+//   x' = Pi_d x,  Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) P_pi;
+//   s = ||x'||_2;  x~' = x' / (s + eps);  index = Q_b(x~') under C_d.
+// The weight side runs the same kernel on the rows of W (row n of
+// W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
+//
+// Design (sm_100a, HBM-bound):
+//   - persistent CTAs, one per SM; a CTA owns R rows at a time and stages
+//     them in shared memory with 1-D bulk copies (cp.async.bulk), double
+//     buffered on two mbarriers so the next tile streams in while this one
+//     is computed;
+//   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
+//     x[pi(k)] from the staged row (the sign D is folded into the gather
+//     table's top bit), runs the whole Walsh-Hadamard butterfly in registers
+//     (packed f32x2 adds), and adds its block's sum of squares into the row
+//     norm (warp shuffles, then one shared-memory pass);
+//   - quantisation needs no search: bin(v) = rint(v G) (one fmaf with a
+//     magic constant) indexes a small table holding, per bin, the count of
+//     thresholds below it and the one threshold inside it, so
+//     index = base + (v >= T) -- exactly #{ j : t_j <= v } in fp32;
+//   - indices are packed LSB-first and written with 16-byte stores.
+#include <cfloat>
+#include <cuda_bf16.h>
+
+#include "device_util.cuh"
+#include "oq_internal.h"
+#include "rpbh_quant.cuh"
+
+namespace oq {
+
+
+namespace {
+
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+struct SmemLayout {
+    int gtab, lut, stage, red, bar, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
+    SmemLayout L;
+    L.gtab = 0;
+    L.lut = align_up(p.d * 2, 16);
+    L.stage = align_up(L.lut + p.lut_n * 8, 128);
+    L.red = L.stage + 2 * p.R * p.srow;
+    L.bar = align_up(L.red + (p.T / 32) * p.R * 4, 8);
+    L.total = L.bar + 16;
+    return L;
+}
+
+
+template <typename InT, int H, int BITS, int MODE>
+__global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const SmemLayout L = smem_layout(p);
+    const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
+    const LutEntry* s_lut = reinterpret_cast<const LutEntry*>(smem + L.lut);
+    uint8_t* s_stage = smem + L.stage;
+    float* s_red = reinterpret_cast<float*>(smem + L.red);
+    uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x;
+    const int R = p.R, nb = p.nb;
+    const int r = tid & (R - 1);
+    const int b = tid / R;
+    const bool active = b < nb;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = p.T >> 5;
+
+    if (tid == 0) {
+        mbar_init(&s_bar[0], 1);
+        mbar_init(&s_bar[1], 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    {
+        const uint4* g = reinterpret_cast<const uint4*>(p.gtab);
+        uint4* s = reinterpret_cast<uint4*>(smem + L.gtab);
+        for (int i = tid; i < p.d / 8; i += blockDim.x) s[i] = g[i];
+        LutEntry* sl = reinterpret_cast<LutEntry*>(smem + L.lut);
+        for (int i = tid; i < p.lut_n; i += blockDim.x) sl[i] = p.lut[i];
+    }
+    __syncthreads();
+
+    auto issue = [&](int tile, int st) {
+        const int row0 = tile * R;
+        const int rows = min(R, p.M - row0);
+        mbar_arrive_expect_tx(&s_bar[st], (uint32_t)(rows * p.row_bytes));
+        const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
+        uint8_t* dst = s_stage + st * R * p.srow;
+        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &s_bar[st]);
+    };
+
+    int tile = blockIdx.x;
+    if (tid == 0 && tile < p.ntiles) issue(tile, 0);
+    int pending_other = 0;  // tid 0: a copy into the other stage is in flight
+
+    const float2 G2 = make_float2(p.G, p.G);
+    const float2 M2 = make_float2(kLutMagic, kLutMagic);
+    const int lut_off = p.lut_off;  // -(magic bits) - kmin, as an index offset
+    constexpr int L2H = H / 2;
+
+    for (int it = 0; tile < p.ntiles; tile += gridDim.x, ++it) {
+        const int st = it & 1;
+        const int next = tile + gridDim.x;
+        pending_other = 0;
+        if (tid == 0 && next < p.ntiles) {
+            issue(next, st ^ 1);
+            pending_other = 1;
+        }
+        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort = 1;
+        __syncthreads();
+        if (s_abort) {
+            // give the prefetch into the other stage (bounded) time to land
+            // before this CTA's shared memory goes away
+            if (tid == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
+            break;
+        }
+
+        const int row = tile * R + r;
+        const bool valid = active && row < p.M;
+
+        // ---- A1 + A2: gather x[pi(k)] with the sign D folded in --------------
+        float2 v2[L2H];
+        if (valid) {
+            const uint8_t* rowp = s_stage + st * R * p.srow + r * p.srow;
+#pragma unroll
+            for (int c = 0; c < H / 8; ++c) {
+                const uint4 ch = reinterpret_cast<const uint4*>(s_gtab)[c * nb + b];
+                const uint32_t w[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const uint32_t e0 = w[e >> 1] & 0xffffu, e1 = w[e >> 1] >> 16;
+                    float f0, f1;
+                    if constexpr (sizeof(InT) == 2) {
+                        const uint32_t r0 = reinterpret_cast<const uint16_t*>(rowp)[e0 & 0x7fffu];
+                        const uint32_t r1 = reinterpret_cast<const uint16_t*>(rowp)[e1 & 0x7fffu];
+                        f0 = __uint_as_float((r0 ^ (e0 & 0x8000u)) << 16);
+                        f1 = __uint_as_float((r1 ^ (e1 & 0x8000u)) << 16);
+                    } else {
+                        const uint32_t r0 = reinterpret_cast<const uint32_t*>(rowp)[e0 & 0x7fffu];
+                        const uint32_t r1 = reinterpret_cast<const uint32_t*>(rowp)[e1 & 0x7fffu];
+                        f0 = __uint_as_float(r0 ^ ((e0 & 0x8000u) << 16));
+                        f1 = __uint_as_float(r1 ^ ((e1 & 0x8000u) << 16));
+                    }
+                    v2[c * 4 + (e >> 1)] = make_float2(f0, f1);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < L2H; ++j) v2[j] = make_float2(0.f, 0.f);
+        }
+
+        // ---- A3: unnormalised Walsh-Hadamard butterflies, Sylvester order ------
+#pragma unroll
+        for (int j = 0; j < L2H; ++j) {
+            const float a = v2[j].x, c = v2[j].y;
+            v2[j] = make_float2(a + c, a - c);
+        }
+#pragma unroll
+        for (int hl = 1; hl < L2H; hl <<= 1) {
+#pragma unroll
+            for (int j = 0; j < L2H; ++j) {
+                if ((j & hl) == 0) {
+                    const float2 a = v2[j], c = v2[j + hl];
+                    v2[j] = f2add(a, c);
+                    v2[j + hl] = f2sub(a, c);
+                }
+            }
+        }
+
+        // ---- A4: row norm (sum of squares of the block, then across blocks) ----
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < L2H; ++j) acc = f2fma(v2[j], v2[j], acc);
+        float ss = acc.x + acc.y;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+            if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane < R) s_red[warp * R + lane] = ss;
+        __syncthreads();
+        float su = 0.f;
+        for (int w = 0; w < nwarps; ++w) su += s_red[w * R + r];
+
+        if (valid) {
+            const float s = su * p.rsqrt_h;  // ||x'|| with the 1/sqrt(h) of H_h applied
+            if (b == 0) {
+                if constexpr (MODE == 0) p.s_out[row] = s;
+                if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+                if constexpr (MODE == 2) p.norm_out[row] = s;
+            }
+            if constexpr (MODE == 2) {
+                float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + b * H);
+                const float2 sc = make_float2(p.rsqrt_h, p.rsqrt_h);
+#pragma unroll
+                for (int j = 0; j < L2H; j += 2) {
+                    const float2 a = f2mul(v2[j], sc), c = f2mul(v2[j + 1], sc);
+                    yo[j >> 1] = make_float4(a.x, a.y, c.x, c.y);
+                }
+            } else {
+                // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
+                constexpr int NB = BITS == 6 ? H : H * BITS / 8;  // packed bytes per h-block
+                constexpr int NW = NB / 4;
+                uint32_t words[NW];
+#pragma unroll
+                for (int i = 0; i < NW; ++i) words[i] = 0u;
+                const bool finite = su <= FLT_MAX;  // false for inf and NaN
+                if (finite) {
+                    const float inv = 1.0f / (su + p.eps_h);
+                    const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+                    for (int j = 0; j < L2H; ++j) {
+                        const float2 q = f2mul(v2[j], inv2);
+                        const float2 z = f2fma(q, G2, M2);
+                        const LutEntry t0 = s_lut[(int)__float_as_uint(z.x) + lut_off];
+                        const LutEntry t1 = s_lut[(int)__float_as_uint(z.y) + lut_off];
+                        const uint32_t i0 = (uint32_t)(t0.base + (q.x >= t0.T ? 1 : 0));
+                        const uint32_t i1 = (uint32_t)(t1.base + (q.y >= t1.T ? 1 : 0));
+                        const int k = 2 * j;
+                        if constexpr (BITS == 4) {
+                            words[k >> 3] |= (i0 | (i1 << 4)) << (4 * (k & 7));
+                        } else if constexpr (BITS == 2) {
+                            words[k >> 4] |= (i0 | (i1 << 2)) << (2 * (k & 15));
+                        } else {
+                            words[k >> 2] |= (i0 | (i1 << 8)) << (8 * (k & 3));
+                        }
+                    }
+                } else {
+                    const uint32_t mid = (uint32_t)(p.L >> 1);
+#pragma unroll
+                    for (int k = 0; k < H; ++k) {
+                        if constexpr (BITS == 4) words[k >> 3] |= mid << (4 * (k & 7));
+                        else if constexpr (BITS == 2) words[k >> 4] |= mid << (2 * (k & 15));
+                        else words[k >> 2] |= mid << (8 * (k & 3));
+                    }
+                }
+                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
+                if constexpr (NB % 16 == 0) {
+#pragma unroll
+                    for (int i = 0; i < NW; i += 4)
+                        reinterpret_cast<uint4*>(dst)[i >> 2] = make_uint4(words[i], words[i + 1], words[i + 2], words[i + 3]);
+                } else if constexpr (NB % 8 == 0) {
+#pragma unroll
+                    for (int i = 0; i < NW; i += 2) reinterpret_cast<uint2*>(dst)[i >> 1] = make_uint2(words[i], words[i + 1]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < NW; ++i) reinterpret_cast<uint32_t*>(dst)[i] = words[i];
+                }
+            }
+        }
+        __syncthreads();  // s_red and this stage are free for reuse
+    }
+}
+
+template <typename InT, int H, int BITS, int MODE>
+cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
+    auto k = rpbh_quant_kernel<InT, H, BITS, MODE>;
+    const int smem = smem_layout(p).total;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, p.T, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename InT, int H, int MODE>
+cudaError_t launch_bits(const RpbhParams& p, int bits, int grid, cudaStream_t stream) {
+    switch (bits) {
+        case 2: return launch_rpbh_t<InT, H, 2, MODE>(p, grid, stream);
+        case 4: return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
+        case 6: return launch_rpbh_t<InT, H, 6, MODE>(p, grid, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename InT, int MODE>
+cudaError_t launch_h(const RpbhParams& p, int h, int bits, int grid, cudaStream_t stream) {
+    switch (h) {
+        case 16: return launch_bits<InT, 16, MODE>(p, bits, grid, stream);
+        case 32: return launch_bits<InT, 32, MODE>(p, bits, grid, stream);
+        case 64: return launch_bits<InT, 64, MODE>(p, bits, grid, stream);
+        case 128: return launch_bits<InT, 128, MODE>(p, bits, grid, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int rpbh_smem_bytes(const RpbhParams& p) { return smem_layout(p).total; }
+
+cudaError_t launch_rpbh_quant(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
+                              cudaStream_t stream) {
+    if (in_bf16) {
+        if (mode == 0) return launch_h<__nv_bfloat16, 0>(p, h, bits, grid, stream);
+        if (mode == 1) return launch_h<__nv_bfloat16, 1>(p, h, bits, grid, stream);
+        return launch_h<__nv_bfloat16, 2>(p, h, 4, grid, stream);
+    }
+    if (mode == 0) return launch_h<float, 0>(p, h, bits, grid, stream);
+    if (mode == 1) return launch_h<float, 1>(p, h, bits, grid, stream);
+    return launch_h<float, 2>(p, h, 4, grid, stream);
+}
+
+}  // namespace oq

@@ -1,0 +1,38 @@
+// Launch interface of the fused RPBH + quantise kernel (rpbh_quant.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "oq_internal.h"
+
+namespace oq {
+
+struct RpbhParams {
+    const void* x;        // [M, d] rows, bf16 or fp32
+    int M, d, nb;         // rows, dimension, h-blocks per row (d / h)
+    int R, T;             // rows per tile (power of two), threads per CTA
+    int row_bytes, srow;  // bytes per input row; shared-memory row stride
+    int ntiles;
+    const uint16_t* gtab;  // device gather table (chunked, see host.cpp)
+    const LutEntry* lut;   // device quantiser lookup table
+    int lut_n, lut_off;    // entries; index offset = -(magic bits) - kmin
+    float G;               // lookup-table bins per unit of v
+    int L;                 // levels (2^bits)
+    uint8_t* idx_out;      // packed indices
+    int out_row_bytes;
+    float* s_out;          // activations: s (fp32)
+    uint16_t* r_out;       // weights: r (bf16)
+    float* y_out;          // test hook: x' (fp32)
+    float* norm_out;       // test hook: ||x'||
+    float rsqrt_h;         // 1/sqrt(h)
+    float eps_h;           // eps * sqrt(h) (the split's eps in unnormalised units)
+};
+
+int rpbh_smem_bytes(const RpbhParams& p);
+
+// mode 0: activations (s fp32), 1: weights (r bf16), 2: rotation only (x', norm)
+cudaError_t launch_rpbh_quant(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
+                              cudaStream_t stream);
+
+}  // namespace oq

@@ -1,0 +1,99 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-side logic (codebook solver, plan generator, argument
+checks) agrees with the oracle.  No GPU compute is called here."""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from rotation_bit_quantization_rpbh_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "oq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(oq_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = B.lib()
+    syms = header_symbols()
+    assert len(syms) >= 18
+    for s in syms:
+        assert hasattr(L, s), s
+    assert sorted(B.EXPORTS) == syms
+
+
+def test_status_strings():
+    L = B.lib()
+    assert L.oq_status_str(0) == b"OQ_OK"
+    assert L.oq_status_str(5) == b"OQ_ERR_TIMEOUT"
+
+
+@pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (12288, 4), (4096, 2), (4096, 4), (1536, 4), (1536, 6),
+                                    (64, 2), (64, 4), (64, 6), (512, 2), (8, 2)])
+def test_library_codebook_matches_oracle(d, bits):
+    """Two independent solvers (library: Newton on the Lloyd-Max conditions
+    with incomplete-beta cell masses; oracle: Lloyd iteration with
+    Gauss-Legendre quadrature) land on the same C_d."""
+    cb = B.codebook(d, bits)
+    c, t = cb.values()
+    co, to = oracle.codebook(d, bits)
+    assert np.max(np.abs(c - co)) * math.sqrt(d) < 1e-10
+    np.testing.assert_array_equal(t.astype(np.float32), to.astype(np.float32))
+    assert t[len(t) // 2] == 0.0
+    np.testing.assert_array_equal(c, -c[::-1])
+    np.testing.assert_array_equal(cb.bf16_bits(), oracle.round_bf16(co)[0])
+
+
+@pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (3072, 128, 1), (12288, 128, 2), (4096, 128, 3), (1536, 128, 4),
+                                      (64, 16, 99)])
+def test_library_plan_matches_oracle(d, h, seed):
+    p1, s1 = B.rpbh_plan_host(d, h, seed)
+    p2, s2 = oracle.plan(d, h, seed)
+    np.testing.assert_array_equal(p1, p2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_argument_checks_on_host_calls():
+    L = B.lib()
+    import ctypes
+
+    h = ctypes.c_void_p()
+    assert L.oq_codebook(256, 7, ctypes.byref(h)) == 2  # UNSUPPORTED
+    assert L.oq_codebook(2, 4, ctypes.byref(h)) == 2
+    assert L.oq_codebook(256, 4, None) == 1  # INVALID_ARG
+    perm = np.zeros(300, dtype=np.int32)
+    sign = np.zeros(300, dtype=np.int8)
+    P = perm.ctypes.data_as(ctypes.c_void_p)
+    S = sign.ctypes.data_as(ctypes.c_void_p)
+    assert L.oq_rpbh_plan_host(300, 128, 0, P, S) == 2  # d % h != 0
+    assert L.oq_rpbh_plan_host(256, 96, 0, P, S) == 2  # h not a power of two
+    assert L.oq_rpbh_plan_host(256, 256, 0, P, S) == 2  # h beyond the in-register block
+    assert L.oq_rpbh_plan_host(0, 64, 0, P, S) == 1
+    assert L.oq_rpbh_plan_host(256, 64, 0, P, S) == 0
+
+
+def test_workspace_size():
+    ws = B.qlinear_workspace(4096, 3072, 4)
+    assert ws >= 4096 * 1536 + 4096 * 4 and ws % 256 == 0
+    assert B.qlinear_workspace(32760, 1536, 6) >= 32760 * 1536 + 32760 * 4
+    assert B.qlinear_workspace(0, 1536, 4) == 0
+    assert B.qlinear_workspace(10, 1536, 3) == 0
+
+
+def test_unpack_layout():
+    import torch
+
+    # two 4-bit codes per byte, LSB first; four 2-bit codes per byte
+    p4 = torch.tensor([[0x21, 0x43]], dtype=torch.uint8)
+    assert B.unpack_indices(p4, 4, 4).tolist() == [[1, 2, 3, 4]]
+    p2 = torch.tensor([[0b11100100]], dtype=torch.uint8)
+    assert B.unpack_indices(p2, 4, 2).tolist() == [[0, 1, 2, 3]]
+    p6 = torch.tensor([[63, 5]], dtype=torch.uint8)
+    assert B.unpack_indices(p6, 2, 6).tolist() == [[63, 5]]

@@ -1,0 +1,112 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs -- multi-tile ragged cases checked in full, the five
+workload shapes at full size checked on sampled rows and columns.
+
+Tolerances are stated in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rotation_bit_quantization_rpbh_b200 import binding as B
+from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+from parity import (GEMM_TOL, check_quantized_rows, check_rotation, gemm_reference, rel_frob, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_idx=1024, n_rows_gemm=128,
+               n_cols_gemm=64, bias=False):
+    rng = np.random.default_rng(seed + 7)
+    plan = B.rpbh_plan(d, h, seed)
+    perm, sign = oracle.plan(d, h, seed)
+    pe, se = plan.export()
+    np.testing.assert_array_equal(pe, perm)
+    np.testing.assert_array_equal(se, sign)
+    cb_a, cb_w = B.codebook(d, ba), B.codebook(d, bw)
+    ocb_a, ocb_w = oracle.codebook(d, ba), oracle.codebook(d, bw)
+
+    xg, Wg = x_cpu.to(dev), W_cpu.to(dev)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, Wg)
+    a_idx, s = B.quantize_acts(plan, cb_a, xg)
+    bias_t = None
+    if bias:
+        bias_t = (torch.randn(N, generator=torch.Generator().manual_seed(seed)) * 0.1).to(torch.bfloat16).to(dev)
+    y = B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=bias_t)
+    y2 = B.qlinear(plan, cb_a, cb_w, xg, w_idx, w_r, bias=bias_t)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    # the one-call layer is the two calls it is made of
+    assert torch.equal(y, y2)
+
+    rows_a = np.arange(M) if full_check else np.sort(rng.choice(M, min(M, n_rows_idx), replace=False))
+    rows_w = np.arange(N) if full_check else np.sort(rng.choice(N, min(N, n_rows_idx), replace=False))
+    rot_rows = rows_a if full_check else rows_a[:64]
+    check_rotation(plan, x_cpu, rot_rows, h, perm, sign, dev)
+    nb_a, _ = check_quantized_rows(a_idx, s, x_cpu, rows_a, h, perm, sign, cb_a, ocb_a, "acts")
+    nb_w, n_ulp = check_quantized_rows(w_idx, w_r, W_cpu, rows_w, h, perm, sign, cb_w, ocb_w, "weights")
+
+    # product: oracle fp64 on the GPU's indices, norms and the bf16 centroid values
+    ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
+    iw = B.unpack_indices(w_idx, d, bw).cpu().numpy()
+    s64 = s.cpu().numpy().astype(np.float64)
+    r64 = w_r.cpu().to(torch.float32).numpy().astype(np.float64)
+    ca = oracle.round_bf16(ocb_a[0])[1]
+    cw = oracle.round_bf16(ocb_w[0])[1]
+    np.testing.assert_array_equal(oracle.round_bf16(ocb_a[0])[0], cb_a.bf16_bits())
+    yg = y.cpu().to(torch.float32).numpy().astype(np.float64)
+    b64 = None if bias_t is None else bias_t.cpu().to(torch.float32).numpy().astype(np.float64)
+    if full_check:
+        ref = gemm_reference(ia, s64, iw, r64, ca, cw)
+        if b64 is not None:
+            ref = ref + b64[None, :]
+        err = rel_frob(yg, ref)
+        assert err <= GEMM_TOL, err
+    else:
+        rr = np.sort(rng.choice(M, min(M, n_rows_gemm), replace=False))
+        cc = np.sort(rng.choice(N, min(N, n_cols_gemm), replace=False))
+        ref_r = gemm_reference(ia, s64, iw, r64, ca, cw, rows=rr)
+        ref_c = gemm_reference(ia, s64, iw, r64, ca, cw, cols=cc)
+        if b64 is not None:
+            ref_r = ref_r + b64[None, :]
+            ref_c = ref_c + b64[None, cc]
+        err = max(rel_frob(yg[rr], ref_r), rel_frob(yg[:, cc], ref_c))
+        assert err <= GEMM_TOL, err
+    return {"band_a": nb_a, "band_w": nb_w, "r_ulp": n_ulp, "gemm_rel": err}
+
+
+# multi-tile cases with ragged edges, checked in full
+SMALL = [
+    # M,   d,   N,  h, bw, ba, dtype, seed, bias
+    (300, 512, 520, 128, 4, 4, "bf16", 11, False),   # 3 M tiles (ragged), 3 N tiles (ragged), 8 K steps
+    (129, 256, 200, 64, 2, 4, "f32", 12, True),     # ragged M by one row, N below one tile
+    (77, 384, 264, 128, 4, 6, "bf16", 13, False),   # 6-bit activations, 1 byte per code
+    (1, 64, 8, 16, 2, 2, "bf16", 14, False),        # a single row, one K step, tiny N
+    (260, 1024, 256, 32, 6, 2, "f32", 15, True),    # 6-bit weights, 2-bit activations, h = 32
+    (513, 768, 272, 128, 2, 6, "bf16", 16, False),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[f"M{c[0]}_d{c[1]}_N{c[2]}_h{c[3]}_W{c[4]}A{c[5]}_{c[6]}" for c in SMALL])
+def test_small_layers_match_oracle_in_full(cuda_device, case):
+    M, d, N, h, bw, ba, dt, seed, bias = case
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))
+    x[:, torch.randint(0, d, (3,), generator=g)] *= 30.0
+    W = torch.randn(N, d, generator=g) * 0.02
+    dtype = torch.bfloat16 if dt == "bf16" else torch.float32
+    _run_layer(cuda_device, M, d, N, h, bw, ba, x.to(dtype), W.to(dtype), seed, full_check=True, bias=bias)
+
+
+@pytest.mark.parametrize("name", I.ORDER)
+def test_workload_at_full_size(cuda_device, name):
+    w = I.WORKLOADS[name]
+    x = I.make_x(w)
+    W = I.make_w(w)
+    full = name == "tiny_w4a4"
+    stats = _run_layer(cuda_device, w.M, w.d, w.N, w.h, w.bits_w, w.bits_a, x, W, w.plan_seed, full_check=full)
+    print(name, stats)
