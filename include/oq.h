@@ -131,7 +131,8 @@ oq_status oq_quantize_weights(const oq_plan_t* plan, const oq_codebook_t* cb_w, 
 /* ---------------------------------------------------------------------- */
 /* Online activation pass  [OrbitQuant, Method: online activation stage].  */
 /*   x' = Pi_d x;  s = ||x'||_2 (fp32);  idx = Q_ba(x' / (s + eps)).        */
-/*   x       device, [M, d] of `dtype`, row-major.  M >= 0 (0: no work).    */
+/*   x       device, [M, d] of `dtype`, row-major.  M >= 0 (0: no work; the */
+/*           buffers may then be NULL).                                    */
 /*   idx_out device, [M, d*bits/8] bytes (bits 6: [M, d]).                  */
 /*   s_out   device, [M] fp32.                                              */
 /* The decision v >= t_j is taken in fp32 (v = x'_k / (s + eps) rounded to */

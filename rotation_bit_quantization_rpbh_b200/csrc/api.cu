@@ -36,10 +36,14 @@ int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }
 // Launch the fused rotate/quantise kernel in one of its three modes.
 oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_dtype dtype, int M, int mode,
                    uint8_t* idx_out, float* s_out, uint16_t* r_out, float* y_out, float* norm_out, cudaStream_t st) {
-    if (!plan || !x || M < 0) return OQ_ERR_INVALID_ARG;
+    if (!plan || M < 0) return OQ_ERR_INVALID_ARG;
     if (dtype != OQ_BF16 && dtype != OQ_F32) return OQ_ERR_INVALID_ARG;
+    if (mode != 2 && (!cb || cb->d != plan->d)) return OQ_ERR_INVALID_ARG;
+    if (mode != 2 && !quant_bits_ok(cb->bits)) return OQ_ERR_UNSUPPORTED;
+    if (M == 0) return OQ_OK;  // an empty batch: buffers may be null
+    if (!x) return OQ_ERR_INVALID_ARG;
     if (mode != 2) {
-        if (!cb || !idx_out) return OQ_ERR_INVALID_ARG;
+        if (!idx_out) return OQ_ERR_INVALID_ARG;
         if (cb->d != plan->d) return OQ_ERR_INVALID_ARG;
         if (!quant_bits_ok(cb->bits)) return OQ_ERR_UNSUPPORTED;
         if (packed_row_bytes(plan->d, cb->bits) % 4 != 0) return OQ_ERR_UNSUPPORTED;
@@ -51,7 +55,6 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     if (mode == 2 && (!aligned16(y_out) || !aligned16(norm_out))) return OQ_ERR_ALIGNMENT;
     if (!aligned16(x)) return OQ_ERR_ALIGNMENT;
     if (current_device() != plan->device) return OQ_ERR_INVALID_ARG;
-    if (M == 0) return OQ_OK;
 
     const DeviceCodebook* dcb = nullptr;
     if (mode != 2) {
@@ -270,13 +273,14 @@ oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, in
 oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
                    const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                    void* stream) {
-    if (!cb_a || !cb_w || !a_idx || !s || !w_idx || !w_r || !y || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
+    if (!cb_a || !cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != cb_w->d) return OQ_ERR_INVALID_ARG;
     if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % 64 != 0) return OQ_ERR_UNSUPPORTED;
+    if (M == 0) return OQ_OK;  // an empty batch: activation and output buffers may be null
+    if (!a_idx || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
     if (!aligned16(a_idx) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
         (bias && !aligned16(bias)))
         return OQ_ERR_ALIGNMENT;
-    if (M == 0) return OQ_OK;
     QgemmArgs a;
     a.M = M;
     a.N = N;
@@ -305,11 +309,12 @@ size_t oq_qlinear_workspace(int M, int d, int bits_a) {
 oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
                      oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
-    if (!plan || !cb_a || !cb_w || !workspace) return OQ_ERR_INVALID_ARG;
+    if (!plan || !cb_a || !cb_w) return OQ_ERR_INVALID_ARG;
     if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
     if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
+    if (!workspace) return OQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return OQ_ERR_ALIGNMENT;
     const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
     if (ws_bytes < need) return OQ_ERR_OOM;

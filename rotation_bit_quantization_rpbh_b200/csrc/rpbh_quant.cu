@@ -182,8 +182,9 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
             if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (lane < R) s_red[warp * R + lane] = ss;
         __syncthreads();
-        float su = 0.f;
-        for (int w = 0; w < nwarps; ++w) su += s_red[w * R + r];
+        float ssum = 0.f;
+        for (int w = 0; w < nwarps; ++w) ssum += s_red[w * R + r];
+        const float su = __fsqrt_rn(ssum);  // ||H u|| before the 1/sqrt(h) of H_h
 
         if (valid) {
             const float s = su * p.rsqrt_h;  // ||x'|| with the 1/sqrt(h) of H_h applied
