@@ -6,19 +6,29 @@
 //   y[m, n] = r_n * s_m * sum_k C_w[iw[n, k]] * C_a[ia[m, k]]
 // with the centroids taken as bf16 values, fp32 accumulation, bf16 output.
 //
-// Structure (one persistent CTA per SM, 128 x 256 output tiles, K step 64):
-//   warp 0      TMA producer: 2-D tensor loads of the packed index tiles
-//               (A: 128 rows, W: 256 rows) into a 4-stage ring;
-//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32
-//               accumulators) and issues tcgen05.mma (one thread);
-//   warps 2-9   decoders: expand each packed tile to bf16 centroid values
-//               (register byte-permute lookups; 6-bit codes via a 64-entry
-//               shared table) and write them in the canonical 128-byte
-//               swizzled K-major layout the MMA descriptors name;
-//   warps 10-13 epilogue: tcgen05.ld of the accumulator, scale by s_m r_n
-//               (+ bias) in fp32, round to bf16, store.
-// Every mbarrier wait is bounded: on a timeout the kernel raises the device
-// error flag, drains its own TMA loads and frees its TMEM before returning.
+// Structure: clusters of two CTAs on an SM pair share one 256 x 256 output
+// tile through tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16 per
+// instruction).  CTA r of the pair owns A rows [128r, 128r + 128) and W rows
+// [128r, 128r + 128) of the tile, so each SM expands 256 rows of codes per
+// K step for a 128 x 256 share of the output (a 1-SM 128 x 256 tile would
+// expand 384).  Per CTA:
+//   warp 0      TMA producer: 2-D tensor loads of this CTA's packed index
+//               tiles into a ring (no multicast: each CTA reads its own rows);
+//   warp 1      TMEM: 512 columns = two 128 x 256 fp32 accumulators; in the
+//               leader CTA one thread issues the pair's MMAs;
+//   warps 2-9   decoders: expand packed codes to bf16 centroid values
+//               (register byte-permute lookups, 64-entry shared table for
+//               6-bit codes) in the 128-byte-swizzled K-major layout, then
+//               arrive on their CTA's "stage full" barrier; in the peer CTA
+//               one thread of warp 1 forwards each full stage to the leader
+//               (one cluster-scope release per stage instead of one per warp);
+//   warps 10-13 epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
+//               scale by s_m r_n (+ bias) in fp32, round to bf16, store, and
+//               release the accumulator to the leader.
+// The leader's MMA completions are multicast (tcgen05.commit) to the
+// barriers of both CTAs.  Every mbarrier wait is bounded: on a timeout the
+// kernel raises the device error flag, drains its own TMA loads, leaves the
+// cluster together with its peer and frees its TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -32,17 +42,23 @@
 namespace oq {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int P_MAX = 4;     // packed ring depth (3 when the packed stage is large)
-constexpr int D_STAGES = 3;  // decoded ring
+constexpr int TM = 256, TN = 256, BK = 64;  // pair tile and K step
+constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one CTA
+constexpr int D_STAGES = 4;                 // decoded ring
+constexpr int P_MAX = 6;                    // packed ring depth (fewer when the packed stage is large)
 constexpr int NDEC_WARPS = 8;
 constexpr int NTHREADS = (2 + NDEC_WARPS + 4) * 32;
-constexpr int DEC_A = BM * 128, DEC_B = BN * 128, DEC_STAGE = DEC_A + DEC_B;
+constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 
 __host__ __device__ constexpr int pk_row_bytes(int bits) { return bits == 6 ? BK : BK * bits / 8; }
-__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw) { return BM * pk_row_bytes(ba) + BN * pk_row_bytes(bw); }
+__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw) { return HM * pk_row_bytes(ba) + HN * pk_row_bytes(bw); }
 __host__ __device__ constexpr int p_stages(int ba, int bw) {
-    return D_STAGES * DEC_STAGE + P_MAX * pk_stage_bytes(ba, bw) + 2048 <= 227 * 1024 ? P_MAX : P_MAX - 1;
+    return (227 * 1024 - D_STAGES * DEC_STAGE - 2048) / pk_stage_bytes(ba, bw) < P_MAX
+               ? (227 * 1024 - D_STAGES * DEC_STAGE - 2048) / pk_stage_bytes(ba, bw)
+               : P_MAX;
+}
+__host__ __device__ constexpr int smem_bytes(int ba, int bw) {
+    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 256 + 256 + 1024;
 }
 
 struct QgemmParams {
@@ -58,8 +74,41 @@ struct QgemmParams {
 };
 
 // ----------------------------------------------------------------------------
-// tcgen05 / TMA wrappers
+// cluster / tcgen05 / TMA wrappers
 // ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -71,15 +120,22 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+// arrive (once the pair's issued MMAs complete) on the barrier at this
+// offset in both CTAs of the pair
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(mask)
+        : "memory");
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
@@ -94,8 +150,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major,
-// M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// M = 256 (the CTA pair), N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
 
 #define OQ_TMEM_LD32(taddr, v)                                                                                        \
     asm volatile(                                                                                                     \
@@ -115,11 +171,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-// Bounded wait that also gives up when another role has already aborted.
+// Bounded wait that also gives up when another role of this CTA aborted.
+template <bool CLUSTER_SCOPE>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto test = [&]() { return CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (test()) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!test()) {
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             atomicExch(&g_error_flag, kErrTimeout);
@@ -138,8 +196,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // (with its sign-replicate mode) marks the negative lanes.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ uint4 decode8_nibbles(uint32_t w, const uint32_t tab[4]) {
-    const uint32_t S = (w >> 3) & 0x11111111u;                  // bit 3 of each nibble (1: upper half)
-    const uint32_t mw = ~(w ^ (S * 7u)) & 0x77777777u;           // magnitude index per nibble
+    const uint32_t S = (w >> 3) & 0x11111111u;         // bit 3 of each nibble (1: upper half)
+    const uint32_t mw = ~(w ^ (S * 7u)) & 0x77777777u;  // magnitude index per nibble
     uint32_t out[4];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -180,26 +238,28 @@ __device__ __forceinline__ uint4 decode_unit(const uint8_t* src, const uint32_t 
     else return decode8_6bit(*reinterpret_cast<const uint2*>(src), tab6);
 }
 
-// Decode a ROWS x 64 tile: unit u = (row, chunk of 8 codes), written to the
-// 128-byte-swizzled K-major position (chunk ^ (row & 7)).
-template <int BITS, int ROWS>
-__device__ __forceinline__ void decode_tile(const uint8_t* pk, uint8_t* dst, int t, const uint32_t tab[4],
-                                            const uint16_t* tab6) {
-    constexpr int UB = BITS == 6 ? 8 : BITS;  // packed bytes per 8 codes
-#pragma unroll 4
-    for (int u = t; u < ROWS * 8; u += NDEC_WARPS * 32) {
-        const int row = u >> 3, c = u & 7;
-        const uint4 v = decode_unit<BITS>(pk + row * pk_row_bytes(BITS) + c * UB, tab, tab6);
-        *reinterpret_cast<uint4*>(dst + (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4)) = v;
+// Decode one CTA's 128 x 64 share of a tile: thread t owns units
+// (row = t/8 + 32 i, chunk = t % 8), i = 0..3, written at the 128-byte
+// swizzled K-major position (chunk ^ (row & 7)) of its row.
+template <int BITS>
+__device__ __forceinline__ void decode_rows(const uint8_t* pk, uint8_t* dst, int src_off, int dst_off,
+                                            const uint32_t tab[4], const uint16_t* tab6) {
+    constexpr int PKR = pk_row_bytes(BITS);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = decode_unit<BITS>(pk + src_off + i * 32 * PKR, tab, tab6);
+        *reinterpret_cast<uint4*>(dst + dst_off + i * 4096) = v;
     }
 }
 
 // ----------------------------------------------------------------------------
 template <int BA, int BW>
-__global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constant__ QgemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    qgemm_kernel(const __grid_constant__ QgemmParams p) {
     extern __shared__ uint8_t smem_raw[];
+    // the same offset in both CTAs (dynamic shared memory starts at the same address)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int PKA = BM * pk_row_bytes(BA);
+    constexpr int PKA = HM * pk_row_bytes(BA);
     constexpr int PK_STAGE = pk_stage_bytes(BA, BW);
     constexpr int P_STAGES = p_stages(BA, BW);
     uint8_t* dec = smem;
@@ -208,14 +268,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(t6 + 128);
     uint64_t* pk_full = bars;
     uint64_t* pk_empty = bars + P_STAGES;
-    uint64_t* dec_full = bars + 2 * P_STAGES;
-    uint64_t* dec_empty = dec_full + D_STAGES;
-    uint64_t* acc_full = dec_empty + D_STAGES;
-    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* dec_full = pk_empty + P_STAGES;   // leader's counts both CTAs' decoders
+    uint64_t* dec_empty = dec_full + D_STAGES;  // arrived by the leader's multicast commit
+    uint64_t* acc_full = dec_empty + D_STAGES;  // arrived by the leader's multicast commit
+    uint64_t* acc_empty = acc_full + 2;         // leader's counts both CTAs' epilogues
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (tid == 0) {
         for (int i = 0; i < P_STAGES; ++i) {
@@ -223,12 +286,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
             mbar_init(&pk_empty[i], NDEC_WARPS);
         }
         for (int i = 0; i < D_STAGES; ++i) {
-            mbar_init(&dec_full[i], NDEC_WARPS);
+            // leader: its own decoder warps plus the peer's relay; peer: its decoder warps
+            mbar_init(&dec_full[i], NDEC_WARPS + (leader ? 1 : 0));
             mbar_init(&dec_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], 2 * 4);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -236,12 +300,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
     if (tid < 64) t6[tid] = p.c6a[tid];
     else if (tid < 128) t6[tid] = p.c6w[tid - 64];
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(512u));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -250,13 +314,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
         if (lane == 0) {
             int step = 0;
             int last_step[P_MAX];
-            for (int i = 0; i < P_STAGES; ++i) last_step[i] = -1;
+            for (int i = 0; i < P_MAX; ++i) last_step[i] = -1;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-                const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+                const int m0 = (tile % p.num_m) * TM + (int)rank * HM;
+                const int n0 = (tile / p.num_m) * TN + (int)rank * HN;
                 for (int kb = 0; kb < p.KB; ++kb, ++step) {
                     const int s = step % P_STAGES;
-                    if (!wait_or_abort(&pk_empty[s], ((step / P_STAGES) & 1) ^ 1, abort_flag)) {
+                    if (!wait_or_abort<false>(&pk_empty[s], ((step / P_STAGES) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -272,18 +337,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
                 if (last_step[i] >= 0) mbar_wait_bounded(&pk_full[i], (last_step[i] / P_STAGES) & 1);
         }
     } else if (warp == 1) {
-        // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0) {
-            int step = 0, acc_it = 0;
+        // ------------------------------ relay (peer CTA) --------------------------
+        // The peer's decoder warps arrive on their own CTA's barrier (a cheap
+        // CTA-scope release); one thread forwards each completed stage to the
+        // leader with a single cluster-scope release.
+        if (!leader && lane == 0) {
+            const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
+            int step = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++acc_it) {
-                const int a = acc_it & 1;
-                if (!wait_or_abort(&acc_empty[a], ((acc_it >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 for (int kb = 0; kb < p.KB; ++kb, ++step) {
                     const int ds = step % D_STAGES;
-                    if (!wait_or_abort(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
+                    if (!wait_or_abort<false>(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_remote(dec_full_leader + (uint32_t)(ds * sizeof(uint64_t)));
+                }
+            }
+        }
+        // ------------------------------ MMA issuer (leader) -----------------------
+        if (leader && lane == 0) {
+            int step = 0, acc_it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++acc_it) {
+                const int a = acc_it & 1;
+                if (!wait_or_abort<true>(&acc_empty[a], ((acc_it >> 1) & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(a * TN);
+                for (int kb = 0; kb < p.KB; ++kb, ++step) {
+                    const int ds = step % D_STAGES;
+                    if (!wait_or_abort<true>(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -291,30 +375,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
                     const uint32_t a_base = smem_u32(dec + ds * DEC_STAGE), b_base = a_base + DEC_A;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k), kIdesc,
-                               (kb | k) != 0 ? 1u : 0u);
-                    tc_commit(&dec_empty[ds]);
+                        tc_mma_pair(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k), kIdesc,
+                                    (kb | k) != 0 ? 1u : 0u);
+                    tc_commit_pair(&dec_empty[ds]);
                 }
-                if (ok) tc_commit(&acc_full[a]);
+                if (ok) tc_commit_pair(&acc_full[a]);
             }
         }
     } else if (warp < 2 + NDEC_WARPS) {
         // ------------------------------ decoders ----------------------------------
         const int t = tid - 64;
+        const int row = t >> 3, c = t & 7;
+        const int dst_off = (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4);
+        const int srcA = row * pk_row_bytes(BA) + c * (BA == 6 ? 8 : BA);
+        const int srcB = row * pk_row_bytes(BW) + c * (BW == 6 ? 8 : BW);
+        const uint32_t tab_a[4] = {p.tab_a[0], p.tab_a[1], p.tab_a[2], p.tab_a[3]};
+        const uint32_t tab_w[4] = {p.tab_w[0], p.tab_w[1], p.tab_w[2], p.tab_w[3]};
         int step = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
             for (int kb = 0; kb < p.KB; ++kb, ++step) {
                 const int ps = step % P_STAGES, ds = step % D_STAGES;
-                if (!wait_or_abort(&pk_full[ps], (step / P_STAGES) & 1, abort_flag) ||
-                    !wait_or_abort(&dec_empty[ds], ((step / D_STAGES) & 1) ^ 1, abort_flag)) {
+                if (!wait_or_abort<false>(&pk_full[ps], (step / P_STAGES) & 1, abort_flag) ||
+                    !wait_or_abort<false>(&dec_empty[ds], ((step / D_STAGES) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const uint8_t* pa = pk + ps * PK_STAGE;
                 uint8_t* da = dec + ds * DEC_STAGE;
-                decode_tile<BA, BM>(pa, da, t, p.tab_a, t6);
-                decode_tile<BW, BN>(pa + PKA, da + DEC_A, t, p.tab_w, t6 + 64);
+                decode_rows<BA>(pa, da, srcA, dst_off, tab_a, t6);
+                decode_rows<BW>(pa + PKA, da + DEC_A, srcB, dst_off, tab_w, t6 + 64);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -326,18 +416,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const uint32_t acc_empty_leader = map_to_rank(&acc_empty[0], 0);
         int acc_it = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++acc_it) {
-            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++acc_it) {
+            const int m0 = (tile % p.num_m) * TM + (int)rank * HM, n0 = (tile / p.num_m) * TN;
             const int a = acc_it & 1;
-            if (!wait_or_abort(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
+            if (!wait_or_abort<false>(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const int row = m0 + q * 32 + lane;
             const bool row_ok = row < p.M;
             const float sm = row_ok ? p.s[row] : 0.f;
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * TN);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+            for (int c0 = 0; c0 < TN; c0 += 32) {
                 uint32_t v[32];
                 OQ_TMEM_LD32(taddr + c0, v);
                 tmem_wait_ld();
@@ -392,25 +483,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) qgemm_kernel(const __grid_constan
                             }
                         }
                     } else {
-                        for (int j = 0; j < 32 && n + j < p.N; ++j) {
-                            float yv = __uint_as_float(v[j]) * sm * __uint_as_float((uint32_t)p.w_r[n + j] << 16);
-                            if (p.bias) yv += __uint_as_float((uint32_t)p.bias[n + j] << 16);
-                            yrow[j] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {  // unrolled: v stays in registers
+                            if (n + j < p.N) {
+                                float yv = __uint_as_float(v[j]) * sm * __uint_as_float((uint32_t)p.w_r[n + j] << 16);
+                                if (p.bias) yv += __uint_as_float((uint32_t)p.bias[n + j] << 16);
+                                yrow[j] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+                            }
                         }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[a]);
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader + (uint32_t)(a * sizeof(uint64_t)));
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // the peer no longer touches this CTA's barriers or shared memory
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u));
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u));
     }
 }
 
@@ -470,7 +565,7 @@ void fill_tables(int bits, const uint16_t* cb, uint32_t tab[4], uint16_t* c6) {
 template <int BA, int BW>
 cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
     auto k = qgemm_kernel<BA, BW>;
-    const int smem = D_STAGES * DEC_STAGE + p_stages(BA, BW) * pk_stage_bytes(BA, BW) + 256 + 256 + 1024;
+    const int smem = smem_bytes(BA, BW);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k<<<grid, NTHREADS, smem, stream>>>(prm);
@@ -491,23 +586,24 @@ int qgemm_sm_count() {
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     QgemmParams prm;
     std::memset(&prm, 0, sizeof(prm));
-    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a), BM) ||
-        !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w), BN))
+    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a), HM) ||
+        !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w), HN))
         return cudaErrorInvalidValue;
     prm.M = a.M;
     prm.N = a.N;
     prm.KB = a.K / BK;
-    prm.num_m = (a.M + BM - 1) / BM;
-    prm.num_tiles = prm.num_m * ((a.N + BN - 1) / BN);
+    prm.num_m = (a.M + TM - 1) / TM;
+    prm.num_tiles = prm.num_m * ((a.N + TN - 1) / TN);
     prm.s = a.s;
     prm.w_r = a.w_r;
     prm.bias = a.bias;
     prm.y = a.y;
     fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
     fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
-    const int grid = prm.num_tiles < qgemm_sm_count() ? prm.num_tiles : qgemm_sm_count();
+    const int pairs_max = qgemm_sm_count() / 2;
+    const int pairs = prm.num_tiles < pairs_max ? prm.num_tiles : pairs_max;
 #define OQ_CASE(X, Y) \
-    if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y>(prm, grid, stream);
+    if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y>(prm, 2 * pairs, stream);
     OQ_CASE(4, 4)
     OQ_CASE(4, 2)
     OQ_CASE(6, 4)
