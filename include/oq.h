@@ -54,7 +54,8 @@ typedef enum {
     OQ_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
     OQ_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see oq_device_status) */
     OQ_ERR_OOM = 6,         /* a library-owned allocation failed, or the workspace is too small */
-    OQ_ERR_NO_CONVERGENCE = 7 /* the codebook solver did not converge */
+    OQ_ERR_NO_CONVERGENCE = 7, /* the codebook solver did not converge */
+    OQ_ERR_TOO_LARGE = 8       /* the request does not fit the fixed scratch of oq_qlinear_noalloc */
 } oq_status;
 
 typedef enum { OQ_BF16 = 0, OQ_F32 = 1 } oq_dtype;
@@ -171,6 +172,35 @@ size_t oq_qlinear_workspace(int M, int d, int bits_a);
 oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
                      oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* The full layer without any device allocation.  The paper has no        */
+/* counterpart to this call: it exists for callers that may not allocate  */
+/* device memory once they are running -- serving processes that reserve  */
+/* all device memory at start-up and forbid cudaMalloc/cudaFree on the    */
+/* request path (an allocation there can block, fragment the reserve or   */
+/* fail under memory pressure), and host code that cannot hold a torch    */
+/* allocator.                                                              */
+/*   Same arguments and results as oq_qlinear, minus the workspace: the   */
+/*   packed activation codes and their norms go to a scratch array that   */
+/*   the library reserves statically on every device that loads it        */
+/*   (OQ_NOALLOC_SCRATCH_BYTES, 64 MiB, held until the process exits).    */
+/*   Requests needing more than that (oq_qlinear_workspace(M, d, bits_a)  */
+/*   > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE before any work. */
+/*   Nothing is allocated here: the plan and both codebooks must already  */
+/*   have their tables on this device (a plan gets them when created; a   */
+/*   codebook on its first oq_quantize_acts / oq_quantize_weights /       */
+/*   oq_qlinear call on the device), else OQ_ERR_INVALID_ARG.             */
+/*   The first call on a device looks up the scratch array's device       */
+/*   address (once per device); make that first call before any stream   */
+/*   capture.  All calls share the one array and it keeps the last call's */
+/*   contents; every call overwrites the part it reads, so nothing needs  */
+/*   clearing.  Calls whose kernels overlap on the GPU (other streams,    */
+/*   other host threads) race on the array: order them on one stream.    */
+#define OQ_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
+                             const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
+                             const uint16_t* bias, uint16_t* y, void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* Device status: reads (and, if `clear`, resets) the current device's     */

@@ -20,13 +20,14 @@ LIB_PATH = os.path.join(_HERE, "liboq.so")
 OQ_OK = 0
 OQ_BF16, OQ_F32 = 0, 1
 _STATUS = {0: "OQ_OK", 1: "OQ_ERR_INVALID_ARG", 2: "OQ_ERR_UNSUPPORTED", 3: "OQ_ERR_ALIGNMENT", 4: "OQ_ERR_CUDA",
-           5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE"}
+           5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE", 8: "OQ_ERR_TOO_LARGE"}
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 # every symbol include/oq.h declares
 EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf16", "oq_codebook_shape",
            "oq_codebook_free", "oq_rpbh_plan", "oq_rpbh_plan_export", "oq_rpbh_plan_host", "oq_plan_shape",
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
-           "oq_qlinear_workspace", "oq_qlinear", "oq_device_status"]
+           "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status"]
 
 
 class OQError(RuntimeError):
@@ -68,6 +69,7 @@ def lib():
                     "oq_qgemm": ([P, P, I, I, P, P, P, P, P, P, P], I),
                     "oq_qlinear_workspace": ([I, I, I], SZ),
                     "oq_qlinear": ([P, P, P, P, I, I, P, P, I, P, P, P, SZ, P], I),
+                    "oq_qlinear_noalloc": ([P, P, P, P, I, I, P, P, I, P, P, P], I),
                     "oq_device_status": ([I, P, P], I),
                 }
                 for name, (args, res) in sig.items():
@@ -243,6 +245,20 @@ def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, 
     _check(lib().oq_qlinear(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
                             _ptr(w_r), N, _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
            "oq_qlinear")
+    return y
+
+
+def qlinear_noalloc(plan, cb_a, cb_w, x, w_idx, w_r, y, bias=None, stream=None):
+    """oq_qlinear without any device allocation inside the call, for callers
+    that may not allocate device memory on their request path (a serving
+    process that reserved all device memory at start-up).  The caller passes
+    the output ``y``; the packed activation codes go to the library's fixed
+    64 MiB per-device scratch array, shared by all calls: calls that overlap
+    on the GPU race on it, so keep them on one stream."""
+    M, d = x.shape
+    N = w_idx.shape[0]
+    _check(lib().oq_qlinear_noalloc(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
+                                    _ptr(w_r), N, _ptr(bias), _ptr(y), _stream(stream)), "oq_qlinear_noalloc")
     return y
 
 

@@ -136,6 +136,7 @@ const char* oq_status_str(oq_status s) {
         case OQ_ERR_TIMEOUT: return "OQ_ERR_TIMEOUT";
         case OQ_ERR_OOM: return "OQ_ERR_OOM";
         case OQ_ERR_NO_CONVERGENCE: return "OQ_ERR_NO_CONVERGENCE";
+        case OQ_ERR_TOO_LARGE: return "OQ_ERR_TOO_LARGE";
     }
     return "OQ_ERR_UNKNOWN";
 }
@@ -324,6 +325,55 @@ oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_
     oq_status st = oq_quantize_acts(plan, cb_a, x, dtype, M, a_idx, s, stream);
     if (st != OQ_OK) return st;
     return oq_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream);
+}
+
+// ---------------------------------------------------------------------------
+// oq_qlinear without device allocation (no counterpart in the paper).
+// Scratch for the packed activation codes and norms lives in this fixed,
+// file-scope device array; its device address is looked up once per device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[OQ_NOALLOC_SCRATCH_BYTES];
+
+static oq_status noalloc_scratch_ptr(void** out) {
+    static std::mutex mu;
+    static void* ptrs[kMaxDevices] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return OQ_ERR_CUDA;
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return OQ_OK;
+}
+
+static bool codebook_resident(oq_codebook_t* cb) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lk(cb->mu);
+    return cb->dev[dev].lut != nullptr;
+}
+
+oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
+                             const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
+                             const uint16_t* bias, uint16_t* y, void* stream) {
+    if (!plan || !cb_a || !cb_w) return OQ_ERR_INVALID_ARG;
+    if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
+    if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
+    if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
+    if (M == 0) return OQ_OK;
+    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
+    if (need > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE;
+    if (current_device() != plan->device) return OQ_ERR_INVALID_ARG;
+    // the activation codebook's tables must already be here (its upload would allocate)
+    if (!codebook_resident(const_cast<oq_codebook_t*>(cb_a))) return OQ_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    oq_status st = noalloc_scratch_ptr(&scratch);
+    if (st != OQ_OK) return st;
+    return oq_qlinear(plan, cb_a, cb_w, x, dtype, M, w_idx, w_r, N, bias, y, scratch, OQ_NOALLOC_SCRATCH_BYTES,
+                      stream);
 }
 
 oq_status oq_device_status(int clear, int* out, void* stream) {
