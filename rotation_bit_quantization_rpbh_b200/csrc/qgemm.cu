@@ -16,13 +16,14 @@
 //               tiles into a ring (no multicast: each CTA reads its own rows);
 //   warp 1      TMEM: 512 columns = two 128 x 256 fp32 accumulators; in the
 //               leader CTA one thread issues the pair's MMAs;
-//   warps 2-9   decoders: expand packed codes to bf16 centroid values
+//   warps 2-17  decoders: expand packed codes to bf16 centroid values
 //               (register byte-permute lookups, 64-entry shared table for
 //               6-bit codes) in the 128-byte-swizzled K-major layout, then
-//               arrive on their CTA's "stage full" barrier; in the peer CTA
-//               one thread of warp 1 forwards each full stage to the leader
-//               (one cluster-scope release per stage instead of one per warp);
-//   warps 10-13 epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
+//               signal the leader's "stage full" barrier: the leader's own
+//               warps arrive, the peer's warps complete transaction bytes on
+//               it with st.async (asynchronous, cluster-scope release), so no
+//               decoder thread waits on a cluster-wide release;
+//   warps 18-21 epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
 //               scale by s_m r_n (+ bias) in fp32, round to bf16, store, and
 //               release the accumulator to the leader.
 // The leader's MMA completions are multicast (tcgen05.commit) to the
@@ -46,7 +47,9 @@ constexpr int TM = 256, TN = 256, BK = 64;  // pair tile and K step
 constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one CTA
 constexpr int D_STAGES = 4;                 // decoded ring
 constexpr int P_MAX = 6;                    // packed ring depth (fewer when the packed stage is large)
-constexpr int NDEC_WARPS = 8;
+constexpr int NDEC_WARPS = 16;
+constexpr int DEC_ROWS = NDEC_WARPS * 4;    // rows one pass of the decoders covers (8 units of 8 codes per row)
+constexpr int DEC_UNITS = HM / DEC_ROWS;   // units per decoder thread and operand per K step
 constexpr int NTHREADS = (2 + NDEC_WARPS + 4) * 32;
 constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 
@@ -95,6 +98,15 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Asynchronous 4-byte store into the peer's shared memory that completes
+// 4 transaction bytes on the peer's mbarrier with cluster-scope release
+// semantics; the issuing thread does not wait for it.
+__device__ __forceinline__ void st_async_complete_tx(uint32_t cluster_dst, uint32_t value, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(cluster_dst),
+                 "r"(value), "r"(cluster_bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -153,14 +165,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 // M = 256 (the CTA pair), N = 256.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
 
-#define OQ_TMEM_LD32(taddr, v)                                                                                        \
-    asm volatile(                                                                                                     \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19," \
-        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                                    \
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), \
-          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),     \
-          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),    \
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])                 \
+#define OQ_TMEM_LD16(taddr, v)                                                                                  \
+    asm volatile(                                                                                               \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),      \
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])  \
         : "r"(taddr))
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -231,24 +240,64 @@ __device__ __forceinline__ uint4 decode8_6bit(uint2 w, const uint16_t* tab) {
     return make_uint4(e0 | (e1 << 16), e2 | (e3 << 16), e4 | (e5 << 16), e6 | (e7 << 16));
 }
 
+// Packed codes of one unit (8 indices): 4-bit -> one word, 2-bit -> the low
+// half of a word, 6-bit (a byte each) -> two words.
 template <int BITS>
-__device__ __forceinline__ uint4 decode_unit(const uint8_t* src, const uint32_t tab[4], const uint16_t* tab6) {
-    if constexpr (BITS == 4) return decode8_nibbles(*reinterpret_cast<const uint32_t*>(src), tab);
-    else if constexpr (BITS == 2) return decode8_2bit(*reinterpret_cast<const uint16_t*>(src), tab);
-    else return decode8_6bit(*reinterpret_cast<const uint2*>(src), tab6);
+struct Packed8 {
+    uint32_t a, b;
+};
+
+template <int BITS>
+__device__ __forceinline__ Packed8<BITS> load_unit(const uint8_t* src) {
+    Packed8<BITS> u;
+    if constexpr (BITS == 4) {
+        u.a = *reinterpret_cast<const uint32_t*>(src);
+        u.b = 0;
+    } else if constexpr (BITS == 2) {
+        u.a = *reinterpret_cast<const uint16_t*>(src);
+        u.b = 0;
+    } else {
+        const uint2 t = *reinterpret_cast<const uint2*>(src);
+        u.a = t.x;
+        u.b = t.y;
+    }
+    return u;
 }
 
-// Decode one CTA's 128 x 64 share of a tile: thread t owns units
-// (row = t/8 + 32 i, chunk = t % 8), i = 0..3, written at the 128-byte
-// swizzled K-major position (chunk ^ (row & 7)) of its row.
 template <int BITS>
-__device__ __forceinline__ void decode_rows(const uint8_t* pk, uint8_t* dst, int src_off, int dst_off,
-                                            const uint32_t tab[4], const uint16_t* tab6) {
-    constexpr int PKR = pk_row_bytes(BITS);
+__device__ __forceinline__ uint4 decode_unit(Packed8<BITS> u, const uint32_t tab[4], const uint16_t* tab6) {
+    if constexpr (BITS == 4) return decode8_nibbles(u.a, tab);
+    else if constexpr (BITS == 2) return decode8_2bit(u.a, tab);
+    else return decode8_6bit(make_uint2(u.a, u.b), tab6);
+}
+
+// Decode one CTA's 128 x 64 shares of A and W for a K step: thread t owns
+// units (row = t/8 + DEC_ROWS i, chunk = t % 8) of each operand, written
+// at the 128-byte-swizzled K-major position (chunk ^ (row & 7)) of its row.
+// All packed words are read before any decoded word is written, so the
+// shared-memory loads are not held behind the stores.
+template <int BA, int BW>
+__device__ __forceinline__ void decode_stage(const uint8_t* pa, const uint8_t* pb, uint8_t* da, uint8_t* db,
+                                             int srcA, int srcB, int dst_off, const uint32_t tab_a[4],
+                                             const uint32_t tab_w[4], const uint16_t* t6) {
+    constexpr int PKRA = pk_row_bytes(BA), PKRB = pk_row_bytes(BW);
+    Packed8<BA> ua[DEC_UNITS];
+    Packed8<BW> ub[DEC_UNITS];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 v = decode_unit<BITS>(pk + src_off + i * 32 * PKR, tab, tab6);
-        *reinterpret_cast<uint4*>(dst + dst_off + i * 4096) = v;
+    for (int i = 0; i < DEC_UNITS; ++i) ua[i] = load_unit<BA>(pa + srcA + i * DEC_ROWS * PKRA);
+#pragma unroll
+    for (int i = 0; i < DEC_UNITS; ++i) ub[i] = load_unit<BW>(pb + srcB + i * DEC_ROWS * PKRB);
+    uint4 va[DEC_UNITS], vb[DEC_UNITS];
+#pragma unroll
+    for (int i = 0; i < DEC_UNITS; ++i) {
+        va[i] = decode_unit<BA>(ua[i], tab_a, t6);
+        vb[i] = decode_unit<BW>(ub[i], tab_w, t6 + 64);
+    }
+#pragma unroll
+    for (int i = 0; i < DEC_UNITS; ++i) {
+        // DEC_ROWS rows = DEC_ROWS / 8 swizzle atoms of 1024 bytes
+        *reinterpret_cast<uint4*>(da + dst_off + i * DEC_ROWS * 128) = va[i];
+        *reinterpret_cast<uint4*>(db + dst_off + i * DEC_ROWS * 128) = vb[i];
     }
 }
 
@@ -274,6 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     uint64_t* acc_empty = acc_full + 2;         // leader's counts both CTAs' epilogues
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint32_t* sink = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // D_STAGES words the peer's stage signals land in
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank();
@@ -286,8 +336,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mbar_init(&pk_empty[i], NDEC_WARPS);
         }
         for (int i = 0; i < D_STAGES; ++i) {
-            // leader: its own decoder warps plus the peer's relay; peer: its decoder warps
-            mbar_init(&dec_full[i], NDEC_WARPS + (leader ? 1 : 0));
+            // leader: arrivals of its own decoder warps, plus 4 transaction
+            // bytes from each of the peer's decoder warps (st.async)
+            mbar_init(&dec_full[i], NDEC_WARPS);
             mbar_init(&dec_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -337,25 +388,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 if (last_step[i] >= 0) mbar_wait_bounded(&pk_full[i], (last_step[i] / P_STAGES) & 1);
         }
     } else if (warp == 1) {
-        // ------------------------------ relay (peer CTA) --------------------------
-        // The peer's decoder warps arrive on their own CTA's barrier (a cheap
-        // CTA-scope release); one thread forwards each completed stage to the
-        // leader with a single cluster-scope release.
-        if (!leader && lane == 0) {
-            const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
-            int step = 0;
-            bool ok = true;
-            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-                for (int kb = 0; kb < p.KB; ++kb, ++step) {
-                    const int ds = step % D_STAGES;
-                    if (!wait_or_abort<false>(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_remote(dec_full_leader + (uint32_t)(ds * sizeof(uint64_t)));
-                }
-            }
-        }
         // ------------------------------ MMA issuer (leader) -----------------------
         if (leader && lane == 0) {
             int step = 0, acc_it = 0;
@@ -391,6 +423,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int srcB = row * pk_row_bytes(BW) + c * (BW == 6 ? 8 : BW);
         const uint32_t tab_a[4] = {p.tab_a[0], p.tab_a[1], p.tab_a[2], p.tab_a[3]};
         const uint32_t tab_w[4] = {p.tab_w[0], p.tab_w[1], p.tab_w[2], p.tab_w[3]};
+        const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
+        const uint32_t sink_leader = map_to_rank(&sink[0], 0);
         int step = 0;
         bool ok = true;
         for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
@@ -403,13 +437,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 }
                 const uint8_t* pa = pk + ps * PK_STAGE;
                 uint8_t* da = dec + ds * DEC_STAGE;
-                decode_rows<BA>(pa, da, srcA, dst_off, tab_a, t6);
-                decode_rows<BW>(pa + PKA, da + DEC_A, srcB, dst_off, tab_w, t6 + 64);
+                decode_stage<BA, BW>(pa, pa + PKA, da, da + DEC_A, srcA, srcB, dst_off, tab_a, tab_w, t6);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&pk_empty[ps]);
-                    mbar_arrive(&dec_full[ds]);
+                    if (leader) {
+                        if (warp == 2) mbar_arrive_expect_tx(&dec_full[ds], 4 * NDEC_WARPS);  // the peer's share
+                        else mbar_arrive(&dec_full[ds]);
+                    } else {
+                        st_async_complete_tx(sink_leader + 4u * (uint32_t)ds, (uint32_t)step,
+                                             dec_full_leader + 8u * (uint32_t)ds);
+                    }
                 }
             }
         }
@@ -428,29 +467,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const float sm = row_ok ? p.s[row] : 0.f;
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * TN);
 #pragma unroll 1
-            for (int c0 = 0; c0 < TN; c0 += 32) {
-                uint32_t v[32];
-                OQ_TMEM_LD32(taddr + c0, v);
+            for (int c0 = 0; c0 < TN; c0 += 16) {
+                uint32_t v[16];
+                OQ_TMEM_LD16(taddr + c0, v);
                 tmem_wait_ld();
                 const int n = n0 + c0;
                 if (row_ok && n < p.N) {
                     uint16_t* yrow = p.y + (size_t)row * p.N + n;
-                    if (n + 32 <= p.N) {
-                        uint32_t rr[16];
+                    if (n + 16 <= p.N) {
+                        uint32_t rr[8], bb[8], o[8];
                         const uint4* rp = reinterpret_cast<const uint4*>(p.w_r + n);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
+                        for (int i = 0; i < 2; ++i) {
                             const uint4 t4 = __ldg(rp + i);
                             rr[4 * i] = t4.x;
                             rr[4 * i + 1] = t4.y;
                             rr[4 * i + 2] = t4.z;
                             rr[4 * i + 3] = t4.w;
                         }
-                        uint32_t bb[16];
                         if (p.bias) {
                             const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
+                            for (int i = 0; i < 2; ++i) {
                                 const uint4 t4 = __ldg(bp + i);
                                 bb[4 * i] = t4.x;
                                 bb[4 * i + 1] = t4.y;
@@ -458,9 +496,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                                 bb[4 * i + 3] = t4.w;
                             }
                         }
-                        uint32_t o[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
+                        for (int j = 0; j < 8; ++j) {
                             const float r0 = __uint_as_float(rr[j] << 16), r1 = __uint_as_float(rr[j] & 0xffff0000u);
                             float y0 = __uint_as_float(v[2 * j]) * sm * r0;
                             float y1 = __uint_as_float(v[2 * j + 1]) * sm * r1;
@@ -473,18 +510,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         }
                         if ((p.N & 7) == 0) {
                             uint4* yp = reinterpret_cast<uint4*>(yrow);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) yp[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                            yp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                            yp[1] = make_uint4(o[4], o[5], o[6], o[7]);
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
+                            for (int j = 0; j < 8; ++j) {
                                 yrow[2 * j] = (uint16_t)(o[j] & 0xffffu);
                                 yrow[2 * j + 1] = (uint16_t)(o[j] >> 16);
                             }
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {  // unrolled: v stays in registers
+                        for (int j = 0; j < 16; ++j) {  // unrolled: v stays in registers
                             if (n + j < p.N) {
                                 float yv = __uint_as_float(v[j]) * sm * __uint_as_float((uint32_t)p.w_r[n + j] << 16);
                                 if (p.bias) yv += __uint_as_float((uint32_t)p.bias[n + j] << 16);
