@@ -8,15 +8,17 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM; a CTA owns R rows at a time and stages
-//     them in shared memory with 1-D bulk copies (cp.async.bulk), double
-//     buffered on two mbarriers so the next tile streams in while this one
-//     is computed;
+//   - persistent CTAs, one per SM; a CTA owns R rows at a time.  The rows
+//     land in a staging buffer by 1-D bulk copies (cp.async.bulk) on an
+//     mbarrier; one vectorised pass copies them into a work area as x and -x
+//     side by side, which frees the staging buffer at once for the next
+//     tile's copies (they stream in while this tile is computed) and turns
+//     the Rademacher sign into a choice of source (the gather table holds a
+//     byte offset into x or into -x for each coordinate);
 //   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
-//     x[pi(k)] from the staged row (the sign D is folded into the gather
-//     table's top bit), runs the whole Walsh-Hadamard butterfly in registers
-//     (packed f32x2 adds), and adds its block's sum of squares into the row
-//     norm (warp shuffles, then one shared-memory pass);
+//     x[pi(k)] from the work area, runs the whole Walsh-Hadamard butterfly in
+//     registers (packed f32x2 adds), and adds its block's sum of squares into
+//     the row norm (warp shuffles, then one shared-memory pass);
 //   - quantisation needs no search: bin(v) = rint(v G) (one fmaf with a
 //     magic constant) indexes a small table holding, per bin, the count of
 //     thresholds below it and the one threshold inside it, so
@@ -31,34 +33,36 @@
 
 namespace oq {
 
-
 namespace {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 struct SmemLayout {
-    int gtab, lut, stage, red, bar, total;
+    int gtab, lut, xstage, work, wrow, red, bar, total;
 };
 
+// gather table (u16 byte offsets) | lookup table | staging buffer (R rows) |
+// work area (R rows of [x | -x]) | norm partials | mbarrier
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
     L.lut = align_up(p.d * 2, 16);
-    L.stage = align_up(L.lut + p.lut_n * 8, 128);
-    L.red = L.stage + 2 * p.R * p.srow;
+    L.xstage = align_up(L.lut + p.lut_n * 8, 128);
+    L.wrow = 2 * p.row_bytes + 16;
+    L.work = align_up(L.xstage + p.R * p.row_bytes, 128);
+    L.red = L.work + p.R * L.wrow;
     L.bar = align_up(L.red + (p.T / 32) * p.R * 4, 8);
     L.total = L.bar + 16;
     return L;
 }
-
 
 template <typename InT, int H, int BITS, int MODE>
 __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
-    const LutEntry* s_lut = reinterpret_cast<const LutEntry*>(smem + L.lut);
-    uint8_t* s_stage = smem + L.stage;
+    uint8_t* s_x = smem + L.xstage;
+    uint8_t* s_work = smem + L.work;
     float* s_red = reinterpret_cast<float*>(smem + L.red);
     uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
     __shared__ int s_abort;
@@ -69,84 +73,103 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     const int b = tid / R;
     const bool active = b < nb;
     const int lane = tid & 31, warp = tid >> 5, nwarps = p.T >> 5;
+    constexpr int ES = sizeof(InT);
 
+    auto issue = [&](int tile) {
+        const int row0 = tile * R;
+        const int rows = min(R, p.M - row0);
+        mbar_arrive_expect_tx(&s_bar[0], (uint32_t)(rows * p.row_bytes));
+        const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
+        // the tile's rows are contiguous in global memory and in the staging buffer
+        bulk_g2s(s_x, src, (uint32_t)(rows * p.row_bytes), &s_bar[0]);
+    };
+
+    int tile = blockIdx.x;
     if (tid == 0) {
         mbar_init(&s_bar[0], 1);
-        mbar_init(&s_bar[1], 1);
         fence_mbar_init();
         s_abort = 0;
+        if (tile < p.ntiles) issue(tile);  // the first copy overlaps the table set-up
     }
     {
+        // plan entries (pi(k) | sign << 15) -> byte offsets into the [x | -x] row
         const uint4* g = reinterpret_cast<const uint4*>(p.gtab);
-        uint4* s = reinterpret_cast<uint4*>(smem + L.gtab);
-        for (int i = tid; i < p.d / 8; i += blockDim.x) s[i] = g[i];
+        uint4* sg = reinterpret_cast<uint4*>(smem + L.gtab);
+        for (int i = tid; i < p.d / 8; i += blockDim.x) {
+            uint4 v = g[i];
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t lo = w[j] & 0xffffu, hi = w[j] >> 16;
+                const uint32_t olo = (lo & 0x7fffu) * ES + ((lo >> 15) ? (uint32_t)p.row_bytes : 0u);
+                const uint32_t ohi = (hi & 0x7fffu) * ES + ((hi >> 15) ? (uint32_t)p.row_bytes : 0u);
+                w[j] = olo | (ohi << 16);
+            }
+            sg[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
         LutEntry* sl = reinterpret_cast<LutEntry*>(smem + L.lut);
         for (int i = tid; i < p.lut_n; i += blockDim.x) sl[i] = p.lut[i];
     }
     __syncthreads();
 
-    auto issue = [&](int tile, int st) {
-        const int row0 = tile * R;
-        const int rows = min(R, p.M - row0);
-        mbar_arrive_expect_tx(&s_bar[st], (uint32_t)(rows * p.row_bytes));
-        const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
-        uint8_t* dst = s_stage + st * R * p.srow;
-        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &s_bar[st]);
-    };
-
-    int tile = blockIdx.x;
-    if (tid == 0 && tile < p.ntiles) issue(tile, 0);
-    int pending_other = 0;  // tid 0: a copy into the other stage is in flight
-
     const float2 G2 = make_float2(p.G, p.G);
     const float2 M2 = make_float2(kLutMagic, kLutMagic);
-    const int lut_off = p.lut_off;  // -(magic bits) - kmin, as an index offset
+    // shared address of lut[(bits of the magic-biased value) + lut_off], folded into one multiply-add
+    const uint32_t lut_addr0 = smem_u32(smem) + (uint32_t)L.lut + (uint32_t)p.lut_off * 8u;
     constexpr int L2H = H / 2;
+    const int cpr = p.row_bytes / 16;  // 16-byte chunks per row
 
     for (int it = 0; tile < p.ntiles; tile += gridDim.x, ++it) {
-        const int st = it & 1;
-        const int next = tile + gridDim.x;
-        pending_other = 0;
-        if (tid == 0 && next < p.ntiles) {
-            issue(next, st ^ 1);
-            pending_other = 1;
-        }
-        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort = 1;
+        if (!mbar_wait_bounded(&s_bar[0], (uint32_t)(it & 1))) s_abort = 1;
         __syncthreads();
-        if (s_abort) {
-            // give the prefetch into the other stage (bounded) time to land
-            // before this CTA's shared memory goes away
-            if (tid == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
-            break;
+        if (s_abort) break;
+        const int rows = min(R, p.M - tile * R);
+
+        // ---- copy the staged rows to the work area as [x | -x] ------------------
+        {
+            const uint32_t neg = ES == 2 ? 0x80008000u : 0x80000000u;
+            for (int rr = 0; rr < rows; ++rr) {
+                const uint4* src = reinterpret_cast<const uint4*>(s_x + rr * p.row_bytes);
+                uint4* dst = reinterpret_cast<uint4*>(s_work + rr * L.wrow);
+                for (int c = tid; c < cpr; c += blockDim.x) {
+                    const uint4 v = src[c];
+                    dst[c] = v;
+                    dst[cpr + c] = make_uint4(v.x ^ neg, v.y ^ neg, v.z ^ neg, v.w ^ neg);
+                }
+            }
         }
+        __syncthreads();
+        const int next = tile + gridDim.x;
+        if (tid == 0 && next < p.ntiles) issue(next);  // streams in while this tile is computed
 
         const int row = tile * R + r;
-        const bool valid = active && row < p.M;
+        const bool valid = active && r < rows;
 
-        // ---- A1 + A2: gather x[pi(k)] with the sign D folded in --------------
+        // ---- A1 + A2: gather sigma_k x[pi(k)] (the sign picks the -x copy) ----
         float2 v2[L2H];
         if (valid) {
-            const uint8_t* rowp = s_stage + st * R * p.srow + r * p.srow;
+            const uint32_t rowp = smem_u32(s_work) + (uint32_t)(r * L.wrow);
 #pragma unroll
             for (int c = 0; c < H / 8; ++c) {
                 const uint4 ch = reinterpret_cast<const uint4*>(s_gtab)[c * nb + b];
                 const uint32_t w[4] = {ch.x, ch.y, ch.z, ch.w};
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const uint32_t e0 = w[e >> 1] & 0xffffu, e1 = w[e >> 1] >> 16;
+                for (int e = 0; e < 4; ++e) {
                     float f0, f1;
-                    if constexpr (sizeof(InT) == 2) {
-                        const uint32_t r0 = reinterpret_cast<const uint16_t*>(rowp)[e0 & 0x7fffu];
-                        const uint32_t r1 = reinterpret_cast<const uint16_t*>(rowp)[e1 & 0x7fffu];
-                        f0 = __uint_as_float((r0 ^ (e0 & 0x8000u)) << 16);
-                        f1 = __uint_as_float((r1 ^ (e1 & 0x8000u)) << 16);
+                    if constexpr (ES == 2) {
+                        uint32_t r0, r1;
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r0) : "r"(rowp + (w[e] & 0xffffu)));
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r1) : "r"(rowp + (w[e] >> 16)));
+                        f0 = __uint_as_float(r0 * 65536u);
+                        f1 = __uint_as_float(r1 * 65536u);
                     } else {
-                        const uint32_t r0 = reinterpret_cast<const uint32_t*>(rowp)[e0 & 0x7fffu];
-                        const uint32_t r1 = reinterpret_cast<const uint32_t*>(rowp)[e1 & 0x7fffu];
-                        f0 = __uint_as_float(r0 ^ ((e0 & 0x8000u) << 16));
-                        f1 = __uint_as_float(r1 ^ ((e1 & 0x8000u) << 16));
+                        uint32_t r0, r1;
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r0) : "r"(rowp + (w[e] & 0xffffu)));
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r1) : "r"(rowp + (w[e] >> 16)));
+                        f0 = __uint_as_float(r0);
+                        f1 = __uint_as_float(r1);
                     }
-                    v2[c * 4 + (e >> 1)] = make_float2(f0, f1);
+                    v2[c * 4 + e] = make_float2(f0, f1);
                 }
             }
         } else {
@@ -205,38 +228,40 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                 // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
                 constexpr int NB = BITS == 6 ? H : H * BITS / 8;  // packed bytes per h-block
                 constexpr int NW = NB / 4;
+                constexpr int PER = BITS == 6 ? 4 : 32 / BITS;     // codes per 32-bit word
+                constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
                 uint32_t words[NW];
-#pragma unroll
-                for (int i = 0; i < NW; ++i) words[i] = 0u;
                 const bool finite = su <= FLT_MAX;  // false for inf and NaN
                 if (finite) {
                     const float inv = 1.0f / (su + p.eps_h);
                     const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-                    for (int j = 0; j < L2H; ++j) {
-                        const float2 q = f2mul(v2[j], inv2);
-                        const float2 z = f2fma(q, G2, M2);
-                        const LutEntry t0 = s_lut[(int)__float_as_uint(z.x) + lut_off];
-                        const LutEntry t1 = s_lut[(int)__float_as_uint(z.y) + lut_off];
-                        const uint32_t i0 = (uint32_t)(t0.base + (q.x >= t0.T ? 1 : 0));
-                        const uint32_t i1 = (uint32_t)(t1.base + (q.y >= t1.T ? 1 : 0));
-                        const int k = 2 * j;
-                        if constexpr (BITS == 4) {
-                            words[k >> 3] |= (i0 | (i1 << 4)) << (4 * (k & 7));
-                        } else if constexpr (BITS == 2) {
-                            words[k >> 4] |= (i0 | (i1 << 2)) << (2 * (k & 15));
-                        } else {
-                            words[k >> 2] |= (i0 | (i1 << 8)) << (8 * (k & 3));
+                    for (int wi = 0; wi < NW; ++wi) {
+                        // codes of this word, highest position first: acc = acc * 2^bits + code
+                        uint32_t acc_w = 0;
+#pragma unroll
+                        for (int k = PER - 2; k >= 0; k -= 2) {
+                            const float2 q = f2mul(v2[(wi * PER + k) >> 1], inv2);
+                            const float2 z = f2fma(q, G2, M2);
+                            float T0, T1;
+                            int b0, b1;
+                            const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
+                            const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
+                            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
+                            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
+                            const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
+                            const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
+                            acc_w = (acc_w * SH + i1) * SH + i0;
                         }
+                        words[wi] = acc_w;
                     }
                 } else {
                     const uint32_t mid = (uint32_t)(p.L >> 1);
+                    uint32_t wmid = 0;
 #pragma unroll
-                    for (int k = 0; k < H; ++k) {
-                        if constexpr (BITS == 4) words[k >> 3] |= mid << (4 * (k & 7));
-                        else if constexpr (BITS == 2) words[k >> 4] |= mid << (2 * (k & 15));
-                        else words[k >> 2] |= mid << (8 * (k & 3));
-                    }
+                    for (int k = 0; k < PER; ++k) wmid = wmid * SH + mid;
+#pragma unroll
+                    for (int wi = 0; wi < NW; ++wi) words[wi] = wmid;
                 }
                 uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
                 if constexpr (NB % 16 == 0) {
@@ -252,7 +277,12 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                 }
             }
         }
-        __syncthreads();  // s_red and this stage are free for reuse
+        __syncthreads();  // work area and partials free for the next tile
+    }
+    if (s_abort && tid == 0) {
+        // give an in-flight copy (bounded) time to land before shared memory goes away
+        mbar_wait_bounded(&s_bar[0], 0u);
+        mbar_wait_bounded(&s_bar[0], 1u);
     }
 }
 
