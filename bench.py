@@ -52,15 +52,25 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+KERNEL_SOURCES = {"qgemm": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu"}
+
+
 def committed_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if one exists for
-    this kernel and workload (null otherwise)."""
+    this kernel and workload and the kernel source is unchanged since the
+    counters were taken (null otherwise)."""
+    import hashlib
+
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        j = json.load(f)
-    return j.get(kernel, {}).get(workload)
+        j = json.load(f).get(kernel, {})
+    src = os.path.join(ROOT, "rotation_bit_quantization_rpbh_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(src, "rb") as f:
+        if hashlib.md5(f.read()).hexdigest() != j.get("source_md5"):
+            return None
+    return j.get(workload)
 
 
 class ClockSampler:
@@ -124,6 +134,24 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def reduce_max(values, world, device):
+    """Element-wise max over ranks of per-rank device times (the slowest rank
+    sets the job's time); identity on one rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens/s: every rank runs its own batch (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
 def rpbh_bytes(w):
@@ -302,10 +330,7 @@ def run_ours(args):
     ms = float(np.mean(t_step))
     ms_rpbh = float(np.mean(t_rpbh))
     ms_gemm = float(np.mean(t_gemm))
-    if world > 1:
-        tt = torch.tensor([ms, ms_rpbh, ms_gemm], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, ms_rpbh, ms_gemm = [float(v) for v in tt.tolist()]
+    ms, ms_rpbh, ms_gemm = reduce_max([ms, ms_rpbh, ms_gemm], world, dev)
 
     # end to end through the public one-call API with host buffers
     e2e = None
@@ -325,12 +350,8 @@ def run_ours(args):
             y_pin.copy_(y, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": world * w.M / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_ms = reduce_max([e0.elapsed_time(e1) / args.steps], world, dev)[0]
+        e2e = {"value": job_throughput(world, w.M, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_cpu.numel() * x_cpu.element_size()),
                "d2h_bytes_per_step": int(y.numel() * y.element_size()), "ms_per_step": e2e_ms}
 
@@ -341,7 +362,7 @@ def run_ours(args):
     rb = rpbh_bytes(w)
     rpbh_gbs = rb / (ms_rpbh * 1e-3) / 1e9
     out = {
-        "metric": METRIC, "value": world * w.M / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": job_throughput(world, w.M, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "d": w.d, "N": w.N, "h": w.h, "bits_w": w.bits_w,
