@@ -49,8 +49,7 @@ extern "C" {
 typedef enum {
     OQ_OK = 0,
     OQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, mismatched handles */
-    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,4,6}, d % 64 != 0,
-                               d beyond 16384 (bf16) / 8192 (fp32) for the quantising calls */
+    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,4,6}, d % 64 != 0 */
     OQ_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned */
     OQ_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
     OQ_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see oq_device_status) */
@@ -102,8 +101,7 @@ void oq_codebook_free(oq_codebook_t* cb);
 /* sigma_k = (next() >> 63) ? -1 : +1.  (P_pi x)_k = x[pi(k)]; sigma_k     */
 /* multiplies post-permutation coordinate k; H_h is Sylvester-ordered and  */
 /* scaled by 1/sqrt(h).                                                     */
-/*   d % h == 0, h a power of two in [16, 128], d <= 32767.  The quantising */
-/*   calls further need d <= 16384 for bf16 inputs, d <= 8192 for fp32.     */
+/*   d % h == 0, h a power of two in [16, 128], d <= 32767.                */
 /* Uploads the plan's gather table to the current device.                  */
 oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out);
 

@@ -63,7 +63,6 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     }
     const int d = plan->d, h = plan->h, nb = d / h;
     const int esize = dtype == OQ_BF16 ? 2 : 4;
-    if (2 * d * esize > 65536) return OQ_ERR_UNSUPPORTED;  // gather offsets into [x | -x] are 16-bit
     RpbhParams p;
     std::memset(&p, 0, sizeof(p));
     p.x = x;
@@ -71,10 +70,10 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.d = d;
     p.nb = nb;
     p.row_bytes = d * esize;
-    p.srow = 2 * d * esize + 16;
+    p.srow = d * esize + 16;  // +16 B: consecutive rows start 4 banks apart
     int R = 1;
-    // rows per tile: a power of two, at most 256 threads, staging + work area within ~200 KB
-    while (R < 32 && 2 * R * nb <= 256 && (2 * R) * (p.row_bytes + p.srow) <= 200 * 1024) R *= 2;
+    // rows per tile: a power of two, at most 256 threads, two staging buffers within ~160 KB
+    while (R < 32 && 2 * R * nb <= 256 && 2 * (2 * R) * p.srow <= 160 * 1024) R *= 2;
     p.R = R;
     p.T = (nb * R + 31) / 32 * 32;
     if (p.T > 1024) return OQ_ERR_UNSUPPORTED;

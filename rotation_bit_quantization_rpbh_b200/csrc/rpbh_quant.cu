@@ -8,17 +8,15 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM; a CTA owns R rows at a time.  The rows
-//     land in a staging buffer by 1-D bulk copies (cp.async.bulk) on an
-//     mbarrier; one vectorised pass copies them into a work area as x and -x
-//     side by side, which frees the staging buffer at once for the next
-//     tile's copies (they stream in while this tile is computed) and turns
-//     the Rademacher sign into a choice of source (the gather table holds a
-//     byte offset into x or into -x for each coordinate);
+//   - persistent CTAs, one per SM; a CTA owns R rows at a time and stages
+//     them in shared memory with 1-D bulk copies (cp.async.bulk), double
+//     buffered on two mbarriers so the next tile streams in while this one
+//     is computed (the first copy is issued before the table set-up);
 //   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
-//     x[pi(k)] from the work area, runs the whole Walsh-Hadamard butterfly in
-//     registers (packed f32x2 adds), and adds its block's sum of squares into
-//     the row norm (warp shuffles, then one shared-memory pass);
+//     x[pi(k)] from the staged row (the sign D is the gather table entry's
+//     top bit, XORed into the bf16 sign), runs the whole Walsh-Hadamard
+//     butterfly in registers (packed f32x2 adds), and adds its block's sum
+//     of squares into the row norm (warp shuffles, one shared-memory pass);
 //   - quantisation needs no search: bin(v) = rint(v G) (one fmaf with a
 //     magic constant) indexes a small table holding, per bin, the count of
 //     thresholds below it and the one threshold inside it, so
@@ -38,19 +36,17 @@ namespace {
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 struct SmemLayout {
-    int gtab, lut, xstage, work, wrow, red, bar, total;
+    int gtab, lut, stage, red, bar, total;
 };
 
-// gather table (u16 byte offsets) | lookup table | staging buffer (R rows) |
-// work area (R rows of [x | -x]) | norm partials | mbarrier
+// gather table (u16 entries) | lookup table | two staging buffers of R rows |
+// norm partials | two mbarriers
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
     L.lut = align_up(p.d * 2, 16);
-    L.xstage = align_up(L.lut + p.lut_n * 8, 128);
-    L.wrow = 2 * p.row_bytes + 16;
-    L.work = align_up(L.xstage + p.R * p.row_bytes, 128);
-    L.red = L.work + p.R * L.wrow;
+    L.stage = align_up(L.lut + p.lut_n * 8, 128);
+    L.red = L.stage + 2 * p.R * p.srow;
     L.bar = align_up(L.red + (p.T / 32) * p.R * 4, 8);
     L.total = L.bar + 16;
     return L;
@@ -61,8 +57,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
-    uint8_t* s_x = smem + L.xstage;
-    uint8_t* s_work = smem + L.work;
+    uint8_t* s_stage = smem + L.stage;
     float* s_red = reinterpret_cast<float*>(smem + L.red);
     uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
     __shared__ int s_abort;
@@ -75,38 +70,27 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     const int lane = tid & 31, warp = tid >> 5, nwarps = p.T >> 5;
     constexpr int ES = sizeof(InT);
 
-    auto issue = [&](int tile) {
+    auto issue = [&](int tile, int st) {
         const int row0 = tile * R;
         const int rows = min(R, p.M - row0);
-        mbar_arrive_expect_tx(&s_bar[0], (uint32_t)(rows * p.row_bytes));
+        mbar_arrive_expect_tx(&s_bar[st], (uint32_t)(rows * p.row_bytes));
         const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
-        // the tile's rows are contiguous in global memory and in the staging buffer
-        bulk_g2s(s_x, src, (uint32_t)(rows * p.row_bytes), &s_bar[0]);
+        uint8_t* dst = s_stage + st * R * p.srow;
+        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &s_bar[st]);
     };
 
     int tile = blockIdx.x;
     if (tid == 0) {
         mbar_init(&s_bar[0], 1);
+        mbar_init(&s_bar[1], 1);
         fence_mbar_init();
         s_abort = 0;
-        if (tile < p.ntiles) issue(tile);  // the first copy overlaps the table set-up
+        if (tile < p.ntiles) issue(tile, 0);  // the first copy overlaps the table set-up
     }
     {
-        // plan entries (pi(k) | sign << 15) -> byte offsets into the [x | -x] row
         const uint4* g = reinterpret_cast<const uint4*>(p.gtab);
         uint4* sg = reinterpret_cast<uint4*>(smem + L.gtab);
-        for (int i = tid; i < p.d / 8; i += blockDim.x) {
-            uint4 v = g[i];
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t lo = w[j] & 0xffffu, hi = w[j] >> 16;
-                const uint32_t olo = (lo & 0x7fffu) * ES + ((lo >> 15) ? (uint32_t)p.row_bytes : 0u);
-                const uint32_t ohi = (hi & 0x7fffu) * ES + ((hi >> 15) ? (uint32_t)p.row_bytes : 0u);
-                w[j] = olo | (ohi << 16);
-            }
-            sg[i] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        for (int i = tid; i < p.d / 8; i += blockDim.x) sg[i] = g[i];
         LutEntry* sl = reinterpret_cast<LutEntry*>(smem + L.lut);
         for (int i = tid; i < p.lut_n; i += blockDim.x) sl[i] = p.lut[i];
     }
@@ -117,57 +101,53 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     // shared address of lut[(bits of the magic-biased value) + lut_off], folded into one multiply-add
     const uint32_t lut_addr0 = smem_u32(smem) + (uint32_t)L.lut + (uint32_t)p.lut_off * 8u;
     constexpr int L2H = H / 2;
-    const int cpr = p.row_bytes / 16;  // 16-byte chunks per row
+    int pending_other = 0;  // tid 0: a copy into the other stage is in flight
 
     for (int it = 0; tile < p.ntiles; tile += gridDim.x, ++it) {
-        if (!mbar_wait_bounded(&s_bar[0], (uint32_t)(it & 1))) s_abort = 1;
-        __syncthreads();
-        if (s_abort) break;
-        const int rows = min(R, p.M - tile * R);
-
-        // ---- copy the staged rows to the work area as [x | -x] ------------------
-        {
-            const uint32_t neg = ES == 2 ? 0x80008000u : 0x80000000u;
-            for (int rr = 0; rr < rows; ++rr) {
-                const uint4* src = reinterpret_cast<const uint4*>(s_x + rr * p.row_bytes);
-                uint4* dst = reinterpret_cast<uint4*>(s_work + rr * L.wrow);
-                for (int c = tid; c < cpr; c += blockDim.x) {
-                    const uint4 v = src[c];
-                    dst[c] = v;
-                    dst[cpr + c] = make_uint4(v.x ^ neg, v.y ^ neg, v.z ^ neg, v.w ^ neg);
-                }
-            }
-        }
-        __syncthreads();
+        const int st = it & 1;
         const int next = tile + gridDim.x;
-        if (tid == 0 && next < p.ntiles) issue(next);  // streams in while this tile is computed
+        pending_other = 0;
+        if (tid == 0 && next < p.ntiles) {
+            issue(next, st ^ 1);  // streams in while this tile is computed
+            pending_other = 1;
+        }
+        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort = 1;
+        __syncthreads();
+        if (s_abort) {
+            // give the prefetch into the other stage (bounded) time to land
+            // before this CTA's shared memory goes away
+            if (tid == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
+            break;
+        }
 
         const int row = tile * R + r;
-        const bool valid = active && r < rows;
+        const bool valid = active && row < p.M;
 
-        // ---- A1 + A2: gather sigma_k x[pi(k)] (the sign picks the -x copy) ----
+        // ---- A1 + A2: gather sigma_k x[pi(k)] (sign = top bit of the entry) ----
         float2 v2[L2H];
         if (valid) {
-            const uint32_t rowp = smem_u32(s_work) + (uint32_t)(r * L.wrow);
+            const uint32_t rowp = smem_u32(s_stage) + (uint32_t)(st * R * p.srow + r * p.srow);
 #pragma unroll
             for (int c = 0; c < H / 8; ++c) {
                 const uint4 ch = reinterpret_cast<const uint4*>(s_gtab)[c * nb + b];
                 const uint32_t w[4] = {ch.x, ch.y, ch.z, ch.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
+                    const uint32_t e0 = w[e], e1 = w[e] >> 16;  // entry k in the low half, k+1 in the high half
                     float f0, f1;
                     if constexpr (ES == 2) {
                         uint32_t r0, r1;
-                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r0) : "r"(rowp + (w[e] & 0xffffu)));
-                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r1) : "r"(rowp + (w[e] >> 16)));
-                        f0 = __uint_as_float(r0 * 65536u);
-                        f1 = __uint_as_float(r1 * 65536u);
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r0) : "r"(rowp + ((e0 & 0x7fffu) << 1)));
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r1) : "r"(rowp + ((e1 & 0x7fffu) << 1)));
+                        // bf16 -> fp32 with the sign flipped where the entry's top bit is set
+                        f0 = __uint_as_float((r0 ^ (e0 & 0x8000u)) << 16);
+                        f1 = __uint_as_float((r1 ^ (e1 & 0x8000u)) << 16);
                     } else {
                         uint32_t r0, r1;
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r0) : "r"(rowp + (w[e] & 0xffffu)));
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r1) : "r"(rowp + (w[e] >> 16)));
-                        f0 = __uint_as_float(r0);
-                        f1 = __uint_as_float(r1);
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r0) : "r"(rowp + ((e0 & 0x7fffu) << 2)));
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r1) : "r"(rowp + ((e1 & 0x7fffu) << 2)));
+                        f0 = __uint_as_float(r0 ^ ((e0 & 0x8000u) << 16));
+                        f1 = __uint_as_float(r1 ^ ((e1 & 0x8000u) << 16));
                     }
                     v2[c * 4 + e] = make_float2(f0, f1);
                 }
@@ -277,12 +257,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                 }
             }
         }
-        __syncthreads();  // work area and partials free for the next tile
-    }
-    if (s_abort && tid == 0) {
-        // give an in-flight copy (bounded) time to land before shared memory goes away
-        mbar_wait_bounded(&s_bar[0], 0u);
-        mbar_wait_bounded(&s_bar[0], 1u);
+        __syncthreads();  // this stage and the partials are free for reuse
     }
 }
 
