@@ -72,18 +72,20 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.row_bytes = d * esize;
     p.srow = d * esize + 16;  // +16 B: consecutive rows start 4 banks apart
     int R = 1;
-    // rows per tile: a power of two, at most 256 threads, two staging buffers within ~160 KB
-    while (R < 32 && 2 * R * nb <= 256 && 2 * (2 * R) * p.srow <= 160 * 1024) R *= 2;
+    // rows per tile: a power of two, at most 128 threads per warp group,
+    // four staging buffers (two groups x two stages) within ~180 KB
+    while (R < 32 && 2 * R * nb <= 128 && 4 * (2 * R) * p.srow <= 180 * 1024) R *= 2;
     p.R = R;
-    p.T = (nb * R + 31) / 32 * 32;
-    if (p.T > 1024) return OQ_ERR_UNSUPPORTED;
+    p.G = (nb * R + 31) / 32 * 32;
+    p.T = 2 * p.G;
+    if (p.T > 256) return OQ_ERR_UNSUPPORTED;
     p.ntiles = (M + R - 1) / R;
     p.gtab = plan->dev.gtab;
     if (mode != 2) {
         p.lut = dcb->lut;
         p.lut_n = (int)cb->lut.size();
         p.lut_off = -(int)kLutMagicBits - cb->kmin;
-        p.G = cb->G;
+        p.G_lut = cb->G;
         p.L = cb->L;
         p.out_row_bytes = packed_row_bytes(d, cb->bits);
     }

@@ -8,10 +8,13 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM; a CTA owns R rows at a time and stages
-//     them in shared memory with 1-D bulk copies (cp.async.bulk), double
-//     buffered on two mbarriers so the next tile streams in while this one
-//     is computed (the first copy is issued before the table set-up);
+//   - persistent CTAs, one per SM, each split into two warp groups that take
+//     alternate tiles of R rows and run out of phase (own staging buffers,
+//     mbarriers and named barriers), so one group's gathers overlap the
+//     other's butterflies and table lookups; a group stages its rows with
+//     1-D bulk copies (cp.async.bulk), double buffered so its next tile
+//     streams in while this one is computed (the first copies are issued
+//     before the table set-up);
 //   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
 //     x[pi(k)] from the staged row (the sign D is the gather table entry's
 //     top bit, XORed into the bf16 sign), runs the whole Walsh-Hadamard
@@ -39,17 +42,21 @@ struct SmemLayout {
     int gtab, lut, stage, red, bar, total;
 };
 
-// gather table (u16 entries) | lookup table | two staging buffers of R rows |
-// norm partials | two mbarriers
+// gather table (u16 entries) | lookup table | 2 groups x 2 staging buffers of
+// R rows | 2 groups' norm partials | 4 mbarriers
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
     L.lut = align_up(p.d * 2, 16);
     L.stage = align_up(L.lut + p.lut_n * 8, 128);
-    L.red = L.stage + 2 * p.R * p.srow;
-    L.bar = align_up(L.red + (p.T / 32) * p.R * 4, 8);
-    L.total = L.bar + 16;
+    L.red = L.stage + 4 * p.R * p.srow;
+    L.bar = align_up(L.red + 2 * (p.G / 32) * p.R * 4, 8);
+    L.total = L.bar + 32;
     return L;
+}
+
+__device__ __forceinline__ void group_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 template <typename InT, int H, int BITS, int MODE>
@@ -57,35 +64,46 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
-    uint8_t* s_stage = smem + L.stage;
-    float* s_red = reinterpret_cast<float*>(smem + L.red);
-    uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
-    __shared__ int s_abort;
+    __shared__ int s_abort[2];
 
+    // Two warp groups per CTA work through alternate tiles independently (own
+    // staging buffers, mbarriers and named barrier), so one group's gathers
+    // overlap the other's butterflies and table lookups.
     const int tid = threadIdx.x;
-    const int R = p.R, nb = p.nb;
-    const int r = tid & (R - 1);
-    const int b = tid / R;
+    const int G = p.G, R = p.R, nb = p.nb;
+    const int grp = tid >= G ? 1 : 0;
+    const int tg = tid - grp * G;
+    const int r = tg & (R - 1);
+    const int b = tg / R;
     const bool active = b < nb;
-    const int lane = tid & 31, warp = tid >> 5, nwarps = p.T >> 5;
+    const int lane = tg & 31, warp = tg >> 5, nwarps = G >> 5;
     constexpr int ES = sizeof(InT);
+    uint8_t* s_stage = smem + L.stage + grp * 2 * R * p.srow;
+    float* s_red = reinterpret_cast<float*>(smem + L.red) + grp * nwarps * R;
+    uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar) + 2 * grp;
 
-    auto issue = [&](int tile, int st) {
+    auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) {
         const int row0 = tile * R;
         const int rows = min(R, p.M - row0);
-        mbar_arrive_expect_tx(&s_bar[st], (uint32_t)(rows * p.row_bytes));
+        mbar_arrive_expect_tx(&bars[st], (uint32_t)(rows * p.row_bytes));
         const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
-        uint8_t* dst = s_stage + st * R * p.srow;
-        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &s_bar[st]);
+        uint8_t* dst = stage + st * R * p.srow;
+        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &bars[st]);
     };
 
-    int tile = blockIdx.x;
+    // this group's tiles: blockIdx.x + (2k + grp) * gridDim.x
+    const int step = 2 * gridDim.x;
+    int tile = blockIdx.x + grp * gridDim.x;
     if (tid == 0) {
-        mbar_init(&s_bar[0], 1);
-        mbar_init(&s_bar[1], 1);
+        uint64_t* all = reinterpret_cast<uint64_t*>(smem + L.bar);
+        for (int i = 0; i < 4; ++i) mbar_init(&all[i], 1);
         fence_mbar_init();
-        s_abort = 0;
-        if (tile < p.ntiles) issue(tile, 0);  // the first copy overlaps the table set-up
+        s_abort[0] = s_abort[1] = 0;
+        // the first copies overlap the table set-up
+        for (int g = 0; g < 2; ++g) {
+            const int t0 = blockIdx.x + g * gridDim.x;
+            if (t0 < p.ntiles) issue(all + 2 * g, smem + L.stage + g * 2 * R * p.srow, t0, 0);
+        }
     }
     {
         const uint4* g = reinterpret_cast<const uint4*>(p.gtab);
@@ -96,27 +114,27 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     }
     __syncthreads();
 
-    const float2 G2 = make_float2(p.G, p.G);
+    const float2 G2 = make_float2(p.G_lut, p.G_lut);
     const float2 M2 = make_float2(kLutMagic, kLutMagic);
     // shared address of lut[(bits of the magic-biased value) + lut_off], folded into one multiply-add
     const uint32_t lut_addr0 = smem_u32(smem) + (uint32_t)L.lut + (uint32_t)p.lut_off * 8u;
     constexpr int L2H = H / 2;
-    int pending_other = 0;  // tid 0: a copy into the other stage is in flight
+    int pending_other = 0;  // group leader: a copy into the other stage is in flight
 
-    for (int it = 0; tile < p.ntiles; tile += gridDim.x, ++it) {
+    for (int it = 0; tile < p.ntiles; tile += step, ++it) {
         const int st = it & 1;
-        const int next = tile + gridDim.x;
+        const int next = tile + step;
         pending_other = 0;
-        if (tid == 0 && next < p.ntiles) {
-            issue(next, st ^ 1);  // streams in while this tile is computed
+        if (tg == 0 && next < p.ntiles) {
+            issue(s_bar, s_stage, next, st ^ 1);  // streams in while this tile is computed
             pending_other = 1;
         }
-        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort = 1;
-        __syncthreads();
-        if (s_abort) {
+        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort[grp] = 1;
+        group_sync(1 + grp, G);
+        if (s_abort[grp]) {
             // give the prefetch into the other stage (bounded) time to land
             // before this CTA's shared memory goes away
-            if (tid == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
+            if (tg == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
             break;
         }
 
@@ -184,7 +202,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
         for (int o = 16; o >= 1; o >>= 1)
             if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (lane < R) s_red[warp * R + lane] = ss;
-        __syncthreads();
+        group_sync(1 + grp, G);
         float ssum = 0.f;
         for (int w = 0; w < nwarps; ++w) ssum += s_red[w * R + r];
         const float su = __fsqrt_rn(ssum);  // ||H u|| before the 1/sqrt(h) of H_h
@@ -257,7 +275,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                 }
             }
         }
-        __syncthreads();  // this stage and the partials are free for reuse
+        group_sync(1 + grp, G);  // this stage and the partials are free for reuse
     }
 }
 

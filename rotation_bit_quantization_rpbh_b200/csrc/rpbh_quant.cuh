@@ -11,13 +11,13 @@ namespace oq {
 struct RpbhParams {
     const void* x;        // [M, d] rows, bf16 or fp32
     int M, d, nb;         // rows, dimension, h-blocks per row (d / h)
-    int R, T;             // rows per tile (power of two), threads per CTA
+    int R, T, G;          // rows per tile (power of two), threads per CTA, threads per warp group (T = 2G)
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
     int ntiles;
     const uint16_t* gtab;  // device gather table (chunked, see host.cpp)
     const LutEntry* lut;   // device quantiser lookup table
     int lut_n, lut_off;    // entries; index offset = -(magic bits) - kmin
-    float G;               // lookup-table bins per unit of v
+    float G_lut;           // lookup-table bins per unit of v
     int L;                 // levels (2^bits)
     uint8_t* idx_out;      // packed indices
     int out_row_bytes;
