@@ -16,13 +16,17 @@
 //               tiles into a ring (no multicast: each CTA reads its own rows);
 //   warp 1      TMEM: 512 columns = two 128 x 256 fp32 accumulators; in the
 //               leader CTA one thread issues the pair's MMAs;
-//   warps 2-17  decoders: expand packed codes to bf16 centroid values
+//   warps 2-17  decoders, two groups taking alternate K steps: expand
+//               packed codes to bf16 centroid values
 //               (register byte-permute lookups, 64-entry shared table for
 //               6-bit codes) in the 128-byte-swizzled K-major layout, then
 //               signal the leader's "stage full" barrier: the leader's own
 //               warps arrive, the peer's warps complete transaction bytes on
 //               it with st.async (asynchronous, cluster-scope release), so no
-//               decoder thread waits on a cluster-wide release;
+//               decoder thread waits on a cluster-wide release.  Each
+//               group's loop is software-pipelined one step deep on both
+//               sides (codes read a step ahead, stages published a step
+//               behind);
 //   warps 18-21 epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
 //               scale by s_m r_n (+ bias) in fp32, round to bf16, store, and
 //               release the accumulator to the leader.
@@ -48,8 +52,10 @@ constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one C
 constexpr int D_STAGES = 4;                 // decoded ring
 constexpr int P_MAX = 6;                    // packed ring depth (fewer when the packed stage is large)
 constexpr int NDEC_WARPS = 16;
-constexpr int DEC_ROWS = NDEC_WARPS * 4;    // rows one pass of the decoders covers (8 units of 8 codes per row)
-constexpr int DEC_UNITS = HM / DEC_ROWS;   // units per decoder thread and operand per K step
+constexpr int NGROUPS = 2;                        // decoder groups, taking alternate K steps
+constexpr int GROUP_WARPS = NDEC_WARPS / NGROUPS;
+constexpr int DEC_ROWS = GROUP_WARPS * 4;         // rows one pass of a group covers (8 units of 8 codes per row)
+constexpr int DEC_UNITS = HM / DEC_ROWS;          // units per decoder thread and operand per K step
 constexpr int NTHREADS = (2 + NDEC_WARPS + 4) * 32;
 constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 
@@ -198,15 +204,24 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }
 
 // ----------------------------------------------------------------------------
-// Decoding packed indices to bf16 centroid values.
-// The codebooks are symmetric (c_{L-1-j} = -c_j), so a 4-bit index j maps to
-// magnitude m = (j & 7) ^ (j < 8 ? 7 : 0) of the positive half and a sign.
-// One byte-permute picks the 4 high bytes, one the 4 low bytes, a third
-// (with its sign-replicate mode) marks the negative lanes.
+// Decoding packed indices to bf16 centroid values, 8 codes (one 16-byte
+// chunk of a K-major row) at a time.
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ uint4 decode8_nibbles(uint32_t w, const uint32_t tab[4]) {
-    const uint32_t S = (w >> 3) & 0x11111111u;         // bit 3 of each nibble (1: upper half)
-    const uint32_t mw = ~(w ^ (S * 7u)) & 0x77777777u;  // magnitude index per nibble
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 4-bit codes.  The codebook is symmetric (c_{15-j} = -c_j), so index j is
+// centroid magnitude m = j & 7 (j >= 8) or m = ~j & 7 (j < 8), negative for
+// j < 8.  tab holds the high bytes of magnitudes 0..7 (words 0, 1) and their
+// low bytes (words 2, 3); one byte-permute per half-word picks 4 high bytes,
+// one the 4 low bytes, and a third, in its sign-replicate mode, marks the
+// lanes with j < 8.
+__device__ __forceinline__ uint4 decode8_4bit(uint32_t w, const uint32_t tab[4]) {
+    const uint32_t s7 = __umulhi(w & 0x88888888u, 0xE0000000u);  // 7 in each nibble with j >= 8
+    const uint32_t mw = ~(w ^ s7) & 0x77777777u;                   // magnitude per nibble
     uint32_t out[4];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -215,32 +230,42 @@ __device__ __forceinline__ uint4 decode8_nibbles(uint32_t w, const uint32_t tab[
         uint32_t hi = prmt(tab[0], tab[1], sel);
         const uint32_t lo = prmt(tab[2], tab[3], sel);
         const uint32_t neg = prmt(0x7f7f7f7fu, 0x7f7f7f7fu, wh);  // 0x7f where j < 8, 0x00 where j >= 8
-        hi ^= (neg << 7) & 0x80808080u;
+        hi |= (neg << 7) & 0x80808080u;
         out[2 * half] = prmt(lo, hi, 0x5140u);
         out[2 * half + 1] = prmt(lo, hi, 0x7362u);
     }
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// 2-bit codes: spread each 2-bit field into a nibble and offset it by 6, so
-// codes 0..3 land on entries 6..9 of a symmetric 16-entry table whose middle
-// four entries are the 4-level codebook.
-__device__ __forceinline__ uint4 decode8_2bit(uint32_t w16, const uint32_t tab[4]) {
-    uint32_t x = w16 & 0xffffu;
-    x = (x | (x << 8)) & 0x00ff00ffu;
-    x = (x | (x << 4)) & 0x0f0f0f0fu;
-    x = (x | (x << 2)) & 0x33333333u;
-    return decode8_nibbles(x + 0x66666666u, tab);
+// 2-bit codes.  The whole 4-level codebook fits one byte-permute source:
+// tab word 0 = low bytes of c_0..c_3, word 1 = their high bytes, so the
+// selector (j, j + 4, j', j' + 4) yields the bf16 pair (c_j, c_j').  The
+// eight 2-bit fields are first moved one per byte (z0: codes 0-3, z1: codes
+// 4-7); a multiply by 0x11 then duplicates each into a nibble pair.
+__device__ __forceinline__ uint4 decode8_2bit(uint32_t x, const uint32_t tab[4]) {
+    const uint32_t a1 = (x | (x << 12)) & 0x000F000Fu;         // codes 0,1 at bits 0-3; 2,3 at 16-19
+    const uint32_t b1 = ((x >> 8) | (x << 4)) & 0x000F000Fu;   // codes 4,5 at bits 0-3; 6,7 at 16-19
+    const uint32_t z0 = (a1 | (a1 << 6)) & 0x03030303u;        // code i at bits 8i
+    const uint32_t z1 = (b1 | (b1 << 6)) & 0x03030303u;
+    return make_uint4(prmt(tab[0], tab[1], z0 * 0x11u + 0x4040u),
+                      prmt(tab[0], tab[1], mad_hi(z0, 0x110000u, 0x4040u)),  // (z0 >> 16) * 0x11 + 0x4040
+                      prmt(tab[0], tab[1], z1 * 0x11u + 0x4040u),
+                      prmt(tab[0], tab[1], mad_hi(z1, 0x110000u, 0x4040u)));
 }
 
-__device__ __forceinline__ uint4 decode8_6bit(uint2 w, const uint16_t* tab) {
-    const uint32_t a = w.x, b = w.y;
-    const uint32_t e0 = tab[a & 63], e1 = tab[(a >> 8) & 63], e2 = tab[(a >> 16) & 63], e3 = tab[(a >> 24) & 63];
-    const uint32_t e4 = tab[b & 63], e5 = tab[(b >> 8) & 63], e6 = tab[(b >> 16) & 63], e7 = tab[(b >> 24) & 63];
-    return make_uint4(e0 | (e1 << 16), e2 | (e3 << 16), e4 | (e5 << 16), e6 | (e7 << 16));
+// 6-bit codes, one per byte: 64-entry bf16 table in shared memory (128
+// bytes, one bank row: the lookups of a warp never conflict).
+__device__ __forceinline__ uint4 decode8_6bit(uint32_t a, uint32_t b, const uint16_t* tab) {
+    a &= 0x3f3f3f3fu;
+    b &= 0x3f3f3f3fu;
+    const uint32_t e0 = tab[a & 0xffu], e1 = tab[prmt(a, 0u, 0x4441u)], e2 = tab[prmt(a, 0u, 0x4442u)],
+                   e3 = tab[a >> 24];
+    const uint32_t e4 = tab[b & 0xffu], e5 = tab[prmt(b, 0u, 0x4441u)], e6 = tab[prmt(b, 0u, 0x4442u)],
+                   e7 = tab[b >> 24];
+    return make_uint4(e0 + e1 * 65536u, e2 + e3 * 65536u, e4 + e5 * 65536u, e6 + e7 * 65536u);
 }
 
-// Packed codes of one unit (8 indices): 4-bit -> one word, 2-bit -> the low
+// Packed codes of one chunk (8 indices): 4-bit -> one word, 2-bit -> the low
 // half of a word, 6-bit (a byte each) -> two words.
 template <int BITS>
 struct Packed8 {
@@ -266,40 +291,67 @@ __device__ __forceinline__ Packed8<BITS> load_unit(const uint8_t* src) {
 
 template <int BITS>
 __device__ __forceinline__ uint4 decode_unit(Packed8<BITS> u, const uint32_t tab[4], const uint16_t* tab6) {
-    if constexpr (BITS == 4) return decode8_nibbles(u.a, tab);
+    if constexpr (BITS == 4) return decode8_4bit(u.a, tab);
     else if constexpr (BITS == 2) return decode8_2bit(u.a, tab);
-    else return decode8_6bit(make_uint2(u.a, u.b), tab6);
+    else return decode8_6bit(u.a, u.b, tab6);
 }
 
-// Decode one CTA's 128 x 64 shares of A and W for a K step: thread t owns
-// units (row = t/8 + DEC_ROWS i, chunk = t % 8) of each operand, written
-// at the 128-byte-swizzled K-major position (chunk ^ (row & 7)) of its row.
-// All packed words are read before any decoded word is written, so the
-// shared-memory loads are not held behind the stores.
+// One decoder thread's codes of a K step: units (row = t/8 + DEC_ROWS i,
+// chunk = t % 8) of this CTA's 128 x 64 shares of A and W.
 template <int BA, int BW>
-__device__ __forceinline__ void decode_stage(const uint8_t* pa, const uint8_t* pb, uint8_t* da, uint8_t* db,
-                                             int srcA, int srcB, int dst_off, const uint32_t tab_a[4],
-                                             const uint32_t tab_w[4], const uint16_t* t6) {
+struct StageCodes {
+    Packed8<BA> a[DEC_UNITS];
+    Packed8<BW> b[DEC_UNITS];
+};
+
+template <int BA, int BW>
+__device__ __forceinline__ void load_codes(StageCodes<BA, BW>& u, const uint8_t* pa, const uint8_t* pb, int srcA,
+                                           int srcB) {
     constexpr int PKRA = pk_row_bytes(BA), PKRB = pk_row_bytes(BW);
-    Packed8<BA> ua[DEC_UNITS];
-    Packed8<BW> ub[DEC_UNITS];
 #pragma unroll
-    for (int i = 0; i < DEC_UNITS; ++i) ua[i] = load_unit<BA>(pa + srcA + i * DEC_ROWS * PKRA);
+    for (int i = 0; i < DEC_UNITS; ++i) u.a[i] = load_unit<BA>(pa + srcA + i * DEC_ROWS * PKRA);
 #pragma unroll
-    for (int i = 0; i < DEC_UNITS; ++i) ub[i] = load_unit<BW>(pb + srcB + i * DEC_ROWS * PKRB);
-    uint4 va[DEC_UNITS], vb[DEC_UNITS];
+    for (int i = 0; i < DEC_UNITS; ++i) u.b[i] = load_unit<BW>(pb + srcB + i * DEC_ROWS * PKRB);
+}
+
+// Expanded values of one K step, written at the 128-byte-swizzled K-major
+// position (chunk ^ (row & 7)) of each row.
+struct StageValues {
+    uint4 a[DEC_UNITS], b[DEC_UNITS];
+};
+
+template <int BA, int BW>
+__device__ __forceinline__ void decode_codes(StageValues& v, const StageCodes<BA, BW>& u, const uint32_t tab_a[4],
+                                             const uint32_t tab_w[4], const uint16_t* t6) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
-        va[i] = decode_unit<BA>(ua[i], tab_a, t6);
-        vb[i] = decode_unit<BW>(ub[i], tab_w, t6 + 64);
+        v.a[i] = decode_unit<BA>(u.a[i], tab_a, t6);
+        v.b[i] = decode_unit<BW>(u.b[i], tab_w, t6 + 64);
     }
+}
+
+__device__ __forceinline__ void store_values(const StageValues& v, uint8_t* da, uint8_t* db, int dst_off) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
         // DEC_ROWS rows = DEC_ROWS / 8 swizzle atoms of 1024 bytes
-        *reinterpret_cast<uint4*>(da + dst_off + i * DEC_ROWS * 128) = va[i];
-        *reinterpret_cast<uint4*>(db + dst_off + i * DEC_ROWS * 128) = vb[i];
+        *reinterpret_cast<uint4*>(da + dst_off + i * DEC_ROWS * 128) = v.a[i];
+        *reinterpret_cast<uint4*>(db + dst_off + i * DEC_ROWS * 128) = v.b[i];
     }
 }
+
+// Position in a ring of N stages and the parity of its current phase.
+template <int N>
+struct RingPos {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void advance(int by = 1) {  // by <= N
+        idx += by;
+        if (idx >= N) {
+            idx -= N;
+            phase ^= 1u;
+        }
+    }
+};
 
 // ----------------------------------------------------------------------------
 template <int BA, int BW>
@@ -333,12 +385,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < P_STAGES; ++i) {
             mbar_init(&pk_full[i], 1);
-            mbar_init(&pk_empty[i], NDEC_WARPS);
+            mbar_init(&pk_empty[i], GROUP_WARPS);
         }
         for (int i = 0; i < D_STAGES; ++i) {
-            // leader: arrivals of its own decoder warps, plus 4 transaction
-            // bytes from each of the peer's decoder warps (st.async)
-            mbar_init(&dec_full[i], NDEC_WARPS);
+            // leader: arrivals of the group's own warps, plus 4 transaction
+            // bytes from each warp of the peer's group (st.async)
+            mbar_init(&dec_full[i], GROUP_WARPS);
             mbar_init(&dec_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -363,60 +415,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
-            int step = 0;
-            int last_step[P_MAX];
-            for (int i = 0; i < P_MAX; ++i) last_step[i] = -1;
+            RingPos<P_STAGES> ps;
+            int issued = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 const int m0 = (tile % p.num_m) * TM + (int)rank * HM;
                 const int n0 = (tile / p.num_m) * TN + (int)rank * HN;
-                for (int kb = 0; kb < p.KB; ++kb, ++step) {
-                    const int s = step % P_STAGES;
-                    if (!wait_or_abort<false>(&pk_empty[s], ((step / P_STAGES) & 1) ^ 1, abort_flag)) {
+                for (int kb = 0; kb < p.KB; ++kb) {
+                    if (!wait_or_abort<false>(&pk_empty[ps.idx], ps.phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&pk_full[s], PK_STAGE);
-                    uint8_t* dst = pk + s * PK_STAGE;
-                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA), m0, &pk_full[s]);
-                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW), n0, &pk_full[s]);
-                    last_step[s] = step;
+                    mbar_arrive_expect_tx(&pk_full[ps.idx], PK_STAGE);
+                    uint8_t* dst = pk + ps.idx * PK_STAGE;
+                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA), m0, &pk_full[ps.idx]);
+                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW), n0, &pk_full[ps.idx]);
+                    ++issued;
+                    ps.advance();
                 }
             }
             // the loads this thread issued must land before shared memory goes away
-            for (int i = 0; i < P_STAGES; ++i)
-                if (last_step[i] >= 0) mbar_wait_bounded(&pk_full[i], (last_step[i] / P_STAGES) & 1);
+            for (int k = 1; k <= P_STAGES && k <= issued; ++k) {
+                const int st = issued - k;
+                mbar_wait_bounded(&pk_full[st % P_STAGES], (uint32_t)(st / P_STAGES) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer (leader) -----------------------
         if (leader && lane == 0) {
-            int step = 0, acc_it = 0;
+            RingPos<D_STAGES> ds;
+            int acc_it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++acc_it) {
                 const int a = acc_it & 1;
                 if (!wait_or_abort<true>(&acc_empty[a], ((acc_it >> 1) & 1) ^ 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(a * TN);
-                for (int kb = 0; kb < p.KB; ++kb, ++step) {
-                    const int ds = step % D_STAGES;
-                    if (!wait_or_abort<true>(&dec_full[ds], (step / D_STAGES) & 1, abort_flag)) {
+                for (int kb = 0; kb < p.KB; ++kb) {
+                    if (!wait_or_abort<true>(&dec_full[ds.idx], ds.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(dec + ds * DEC_STAGE), b_base = a_base + DEC_A;
+                    const uint32_t a_base = smem_u32(dec + ds.idx * DEC_STAGE), b_base = a_base + DEC_A;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
                         tc_mma_pair(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k), kIdesc,
                                     (kb | k) != 0 ? 1u : 0u);
-                    tc_commit_pair(&dec_empty[ds]);
+                    tc_commit_pair(&dec_empty[ds.idx]);
+                    ds.advance();
                 }
                 if (ok) tc_commit_pair(&acc_full[a]);
             }
         }
     } else if (warp < 2 + NDEC_WARPS) {
         // ------------------------------ decoders ----------------------------------
-        const int t = tid - 64;
+        // Two groups of GROUP_WARPS warps take alternate K steps, so one group
+        // expands codes while the other waits on its barriers.  Within a group
+        // the loop is software-pipelined: the codes of its next step are read
+        // from shared memory before the current step is expanded, and a step
+        // is published (proxy fence + stage signal) only after the group's
+        // following step is expanded, by which time its stores have completed.
+        const int grp = (warp - 2) / GROUP_WARPS;
+        const int t = (warp - 2 - grp * GROUP_WARPS) * 32 + lane;
+        const bool grp_lead = warp == 2 + grp * GROUP_WARPS;
         const int row = t >> 3, c = t & 7;
         const int dst_off = (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4);
         const int srcA = row * pk_row_bytes(BA) + c * (BA == 6 ? 8 : BA);
@@ -425,33 +487,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t tab_w[4] = {p.tab_w[0], p.tab_w[1], p.tab_w[2], p.tab_w[3]};
         const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
         const uint32_t sink_leader = map_to_rank(&sink[0], 0);
-        int step = 0;
-        bool ok = true;
-        for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-            for (int kb = 0; kb < p.KB; ++kb, ++step) {
-                const int ps = step % P_STAGES, ds = step % D_STAGES;
-                if (!wait_or_abort<false>(&pk_full[ps], (step / P_STAGES) & 1, abort_flag) ||
-                    !wait_or_abort<false>(&dec_empty[ds], ((step / D_STAGES) & 1) ^ 1, abort_flag)) {
+        // publish decoded stage `slot` to the leader's MMA issuer
+        auto publish = [&](int slot) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) {
+                    if (grp_lead) mbar_arrive_expect_tx(&dec_full[slot], 4 * GROUP_WARPS);  // the peer's share
+                    else mbar_arrive(&dec_full[slot]);
+                } else {
+                    st_async_complete_tx(sink_leader + 4u * (uint32_t)slot, (uint32_t)slot,
+                                         dec_full_leader + 8u * (uint32_t)slot);
+                }
+            }
+        };
+        const int my_tiles = pair < p.num_tiles ? (p.num_tiles - 1 - pair) / npairs + 1 : 0;
+        const int total = my_tiles * p.KB;
+        RingPos<P_STAGES> ps;
+        RingPos<D_STAGES> ds;
+        ps.idx = grp;
+        ds.idx = grp;
+        int pending = -1;  // decoded slot stored but not yet published
+        StageCodes<BA, BW> cur;
+        bool ok = grp < total && wait_or_abort<false>(&pk_full[ps.idx], 0u, abort_flag);
+        if (ok) load_codes<BA, BW>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+        for (int s = grp; ok && s < total; s += NGROUPS) {
+            StageCodes<BA, BW> nxt;
+            const int ps_cur = ps.idx;
+            ps.advance(NGROUPS);
+            if (s + NGROUPS < total) {
+                if (!wait_or_abort<false>(&pk_full[ps.idx], ps.phase, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* pa = pk + ps * PK_STAGE;
-                uint8_t* da = dec + ds * DEC_STAGE;
-                decode_stage<BA, BW>(pa, pa + PKA, da, da + DEC_A, srcA, srcB, dst_off, tab_a, tab_w, t6);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&pk_empty[ps]);
-                    if (leader) {
-                        if (warp == 2) mbar_arrive_expect_tx(&dec_full[ds], 4 * NDEC_WARPS);  // the peer's share
-                        else mbar_arrive(&dec_full[ds]);
-                    } else {
-                        st_async_complete_tx(sink_leader + 4u * (uint32_t)ds, (uint32_t)step,
-                                             dec_full_leader + 8u * (uint32_t)ds);
-                    }
-                }
+                const uint8_t* pa = pk + ps.idx * PK_STAGE;
+                load_codes<BA, BW>(nxt, pa, pa + PKA, srcA, srcB);
             }
+            StageValues v;
+            decode_codes<BA, BW>(v, cur, tab_a, tab_w, t6);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pk_empty[ps_cur]);  // codes of step s are in registers
+            if (pending >= 0) publish(pending);
+            if (!wait_or_abort<false>(&dec_empty[ds.idx], ds.phase ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            uint8_t* da = dec + ds.idx * DEC_STAGE;
+            store_values(v, da, da + DEC_A, dst_off);
+            pending = ds.idx;
+            ds.advance(NGROUPS);
+            cur = nxt;
         }
+        if (ok && pending >= 0) publish(pending);
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
@@ -575,28 +662,27 @@ bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int b
     return r == CUDA_SUCCESS;
 }
 
-// 4-bit-path tables from a symmetric 16-entry bf16 codebook c16 (c16[8+m] =
-// magnitude m): high bytes of magnitudes 0..7, then low bytes.
-void nibble_tables(const uint16_t* c16, uint32_t tab[4]) {
-    tab[0] = tab[1] = tab[2] = tab[3] = 0;
-    for (int m = 0; m < 8; ++m) {
-        const uint32_t v = c16[8 + m];
-        tab[m / 4] |= ((v >> 8) & 0xffu) << (8 * (m % 4));
-        tab[2 + m / 4] |= (v & 0xffu) << (8 * (m % 4));
-    }
-}
-
+// Byte-permute tables of the register decoders (see decode8_4bit and
+// decode8_2bit); 6-bit codebooks go to the shared-memory table instead.
 void fill_tables(int bits, const uint16_t* cb, uint32_t tab[4], uint16_t* c6) {
-    uint16_t c16[16] = {0};
+    tab[0] = tab[1] = tab[2] = tab[3] = 0;
     std::memset(c6, 0, 64 * sizeof(uint16_t));
     if (bits == 4) {
-        for (int j = 0; j < 16; ++j) c16[j] = cb[j];
+        // magnitude m is centroid 8 + m: high bytes in words 0-1, low bytes in 2-3
+        for (int m = 0; m < 8; ++m) {
+            const uint32_t v = cb[8 + m];
+            tab[m / 4] |= ((v >> 8) & 0xffu) << (8 * (m % 4));
+            tab[2 + m / 4] |= (v & 0xffu) << (8 * (m % 4));
+        }
     } else if (bits == 2) {
-        for (int j = 0; j < 4; ++j) c16[6 + j] = cb[j];
+        // low bytes of c_0..c_3 in word 0, high bytes in word 1
+        for (int j = 0; j < 4; ++j) {
+            tab[0] |= (uint32_t)(cb[j] & 0xffu) << (8 * j);
+            tab[1] |= (uint32_t)((cb[j] >> 8) & 0xffu) << (8 * j);
+        }
     } else {
         for (int j = 0; j < 64; ++j) c6[j] = cb[j];
     }
-    nibble_tables(c16, tab);
 }
 
 template <int BA, int BW>
