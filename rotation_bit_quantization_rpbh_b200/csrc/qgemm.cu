@@ -62,12 +62,14 @@ constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 __host__ __device__ constexpr int pk_row_bytes(int bits) { return bits == 6 ? BK : BK * bits / 8; }
 __host__ __device__ constexpr int pk_stage_bytes(int ba, int bw) { return HM * pk_row_bytes(ba) + HN * pk_row_bytes(bw); }
 __host__ __device__ constexpr int p_stages(int ba, int bw) {
-    return (227 * 1024 - D_STAGES * DEC_STAGE - 2048) / pk_stage_bytes(ba, bw) < P_MAX
-               ? (227 * 1024 - D_STAGES * DEC_STAGE - 2048) / pk_stage_bytes(ba, bw)
+    return (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw) < P_MAX
+               ? (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw)
                : P_MAX;
 }
+// decoded ring | packed ring | 6-bit tables (256 B) | epilogue r and bias of a
+// tile (1 KB) | barriers (256 B) | alignment slack (1 KB)
 __host__ __device__ constexpr int smem_bytes(int ba, int bw) {
-    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 256 + 256 + 1024;
+    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 256 + 1024 + 256 + 1024;
 }
 
 struct QgemmParams {
@@ -157,6 +159,9 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
+
+// named barrier 1 over the four epilogue warps
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -366,7 +371,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     uint8_t* dec = smem;
     uint8_t* pk = smem + D_STAGES * DEC_STAGE;
     uint16_t* t6 = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(t6 + 128);
+    uint16_t* epi_r = t6 + 128;     // r_n of the current tile's 256 columns
+    uint16_t* epi_b = epi_r + TN;   // bias of those columns
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi_b + TN);
     uint64_t* pk_full = bars;
     uint64_t* pk_empty = bars + P_STAGES;
     uint64_t* dec_full = pk_empty + P_STAGES;   // leader's counts both CTAs' decoders
@@ -541,80 +548,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (ok && pending >= 0) publish(pending);
     } else {
         // ------------------------------ epilogue ----------------------------------
+        // Per tile: stage r (and bias) of the tile's 256 columns in shared
+        // memory, then per 32-column chunk read 32 fp32 accumulators of this
+        // thread's row from TMEM, scale by s_m r_n (+ bias), round to bf16 and
+        // store 64 bytes of the row.
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int et = tid - (2 + NDEC_WARPS) * 32;  // 0..127
         const uint32_t acc_empty_leader = map_to_rank(&acc_empty[0], 0);
+        const bool vec_ok = (p.N & 7) == 0;  // rows of y 16-byte aligned
         int acc_it = 0;
         for (int tile = pair; tile < p.num_tiles; tile += npairs, ++acc_it) {
             const int m0 = (tile % p.num_m) * TM + (int)rank * HM, n0 = (tile / p.num_m) * TN;
             const int a = acc_it & 1;
             if (!wait_or_abort<false>(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
             tc_fence_after();
+            epilogue_sync();  // the previous tile's reads of epi_r / epi_b are done
+            for (int j = et; j < TN; j += 128) {
+                const int n = n0 + j;
+                epi_r[j] = n < p.N ? p.w_r[n] : (uint16_t)0;
+                epi_b[j] = (p.bias && n < p.N) ? p.bias[n] : (uint16_t)0;
+            }
+            epilogue_sync();
             const int row = m0 + q * 32 + lane;
             const bool row_ok = row < p.M;
             const float sm = row_ok ? p.s[row] : 0.f;
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * TN);
+            uint16_t* yrow = p.y + (size_t)(row_ok ? row : 0) * p.N;
 #pragma unroll 1
-            for (int c0 = 0; c0 < TN; c0 += 16) {
-                uint32_t v[16];
+            for (int c0 = 0; c0 < TN; c0 += 32) {
+                uint32_t v[32];
                 OQ_TMEM_LD16(taddr + c0, v);
+                OQ_TMEM_LD16(taddr + c0 + 16, (v + 16));
                 tmem_wait_ld();
                 const int n = n0 + c0;
-                if (row_ok && n < p.N) {
-                    uint16_t* yrow = p.y + (size_t)row * p.N + n;
-                    if (n + 16 <= p.N) {
-                        uint32_t rr[8], bb[8], o[8];
-                        const uint4* rp = reinterpret_cast<const uint4*>(p.w_r + n);
+                if (!row_ok || n >= p.N) continue;
+                const uint4* rp = reinterpret_cast<const uint4*>(epi_r + c0);
+                const uint4* bp = reinterpret_cast<const uint4*>(epi_b + c0);
+                uint32_t o[16];
 #pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            const uint4 t4 = __ldg(rp + i);
-                            rr[4 * i] = t4.x;
-                            rr[4 * i + 1] = t4.y;
-                            rr[4 * i + 2] = t4.z;
-                            rr[4 * i + 3] = t4.w;
-                        }
-                        if (p.bias) {
-                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 r4 = rp[i];
+                    const uint32_t rr[4] = {r4.x, r4.y, r4.z, r4.w};
+                    uint32_t bb[4] = {0, 0, 0, 0};
+                    if (p.bias) {
+                        const uint4 b4 = bp[i];
+                        bb[0] = b4.x; bb[1] = b4.y; bb[2] = b4.z; bb[3] = b4.w;
+                    }
 #pragma unroll
-                            for (int i = 0; i < 2; ++i) {
-                                const uint4 t4 = __ldg(bp + i);
-                                bb[4 * i] = t4.x;
-                                bb[4 * i + 1] = t4.y;
-                                bb[4 * i + 2] = t4.z;
-                                bb[4 * i + 3] = t4.w;
-                            }
-                        }
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * i + jj;
+                        const float y0 = __uint_as_float(v[2 * j]) * sm * __uint_as_float(rr[jj] << 16) +
+                                         __uint_as_float(bb[jj] << 16);
+                        const float y1 = __uint_as_float(v[2 * j + 1]) * sm * __uint_as_float(rr[jj] & 0xffff0000u) +
+                                         __uint_as_float(bb[jj] & 0xffff0000u);
+                        o[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
+                               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y1)) << 16);
+                    }
+                }
+                if (vec_ok && n + 32 <= p.N) {
+                    uint4* yp = reinterpret_cast<uint4*>(yrow + n);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float r0 = __uint_as_float(rr[j] << 16), r1 = __uint_as_float(rr[j] & 0xffff0000u);
-                            float y0 = __uint_as_float(v[2 * j]) * sm * r0;
-                            float y1 = __uint_as_float(v[2 * j + 1]) * sm * r1;
-                            if (p.bias) {
-                                y0 += __uint_as_float(bb[j] << 16);
-                                y1 += __uint_as_float(bb[j] & 0xffff0000u);
-                            }
-                            o[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
-                                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y1)) << 16);
-                        }
-                        if ((p.N & 7) == 0) {
-                            uint4* yp = reinterpret_cast<uint4*>(yrow);
-                            yp[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                            yp[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                        } else {
+                    for (int i = 0; i < 4; ++i) yp[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                } else {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                yrow[2 * j] = (uint16_t)(o[j] & 0xffffu);
-                                yrow[2 * j + 1] = (uint16_t)(o[j] >> 16);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {  // unrolled: v stays in registers
-                            if (n + j < p.N) {
-                                float yv = __uint_as_float(v[j]) * sm * __uint_as_float((uint32_t)p.w_r[n + j] << 16);
-                                if (p.bias) yv += __uint_as_float((uint32_t)p.bias[n + j] << 16);
-                                yrow[j] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
-                            }
-                        }
+                    for (int j = 0; j < 16; ++j) {  // unrolled: o stays in registers
+                        if (n + 2 * j < p.N) yrow[n + 2 * j] = (uint16_t)(o[j] & 0xffffu);
+                        if (n + 2 * j + 1 < p.N) yrow[n + 2 * j + 1] = (uint16_t)(o[j] >> 16);
                     }
                 }
             }

@@ -88,6 +88,7 @@ SMALL = [
     (1, 64, 8, 16, 2, 2, "bf16", 14, False),        # a single row, one K step, tiny N
     (260, 1024, 256, 32, 6, 2, "f32", 15, True),    # 6-bit weights, 2-bit activations, h = 32
     (513, 768, 272, 128, 2, 6, "bf16", 16, False),
+    (70, 256, 131, 64, 4, 4, "bf16", 17, True),     # N not a multiple of 8: unaligned output rows
 ]
 
 
