@@ -137,8 +137,11 @@ oq_status oq_quantize_weights(const oq_plan_t* plan, const oq_codebook_t* cb_w, 
 /*   idx_out device, [M, d*bits/8] bytes (bits 6: [M, d]).                  */
 /*   s_out   device, [M] fp32.                                              */
 /* The decision v >= t_j is taken in fp32 (v = x'_k / (s + eps) rounded to */
-/* fp32, t_j the fp32-rounded thresholds).  Rows whose norm is not finite  */
-/* are quantised to the middle cell (index 2^(bits-1)) with s stored as is. */
+/* fp32, t_j the fp32-rounded thresholds).  s is accumulated in fp32 from  */
+/* the inputs (Pi_d is orthogonal, so ||x'|| = ||x||).  Rows whose norm is */
+/* not finite or above FLT_MAX / (2 sqrt(h)) (where the fp32 transform     */
+/* could overflow) are quantised to the middle cell (index 2^(bits-1))     */
+/* with s stored as is.                                                    */
 oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype, int M,
                            uint8_t* idx_out, float* s_out, void* stream);
 

@@ -237,7 +237,7 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
     for (int j = 0; j + 2 < L; ++j) min_gap = std::min(min_gap, (double)cb->t32[j + 1] - (double)cb->t32[j]);
     float G = (float)(1.0 / min_gap);
     if (L == 2) G = 4.0f;
-    const float vmax = 1.0f + 1.0f / 1024.0f;  // |v| <= 1 up to fp32 rounding for finite rows
+    const float vmax = 1.0f + 1.0f / 16.0f;  // |v| <= 1 up to fp32 rounding for the rows the kernel quantises
     for (int tries = 0; tries < 64; ++tries) {
         bool ok = true;
         for (int j = 0; j + 2 < L; ++j)
@@ -259,6 +259,9 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
         }
         e.base = base;
     }
+    // an even entry count: the kernels stage the table with a 16-byte-multiple
+    // bulk copy (the extra entry is never indexed)
+    if (cb->lut.size() % 2) cb->lut.push_back(cb->lut.back());
     return OQ_OK;
 }
 

@@ -15,11 +15,14 @@
 //     1-D bulk copies (cp.async.bulk), double buffered so its next tile
 //     streams in while this one is computed (the first copies are issued
 //     before the table set-up);
+//   - the gather and lookup tables arrive by bulk copy together with each
+//     group's first rows;
 //   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
 //     x[pi(k)] from the staged row (the sign D is the gather table entry's
-//     top bit, XORed into the bf16 sign), runs the whole Walsh-Hadamard
-//     butterfly in registers (packed f32x2 adds), and adds its block's sum
-//     of squares into the row norm (warp shuffles, one shared-memory pass);
+//     top bit, XORed into the bf16 sign) and runs the whole Walsh-Hadamard
+//     butterfly in registers (packed f32x2 adds).  The row norm is the norm
+//     of the gathered inputs (Pi_d is orthogonal, so ||x'|| = ||x||): its
+//     cross-warp reduction is posted before the butterflies and read after;
 //   - quantisation needs no search: bin(v) = rint(v G) (one fmaf with a
 //     magic constant) indexes a small table holding, per bin, the count of
 //     thresholds below it and the one threshold inside it, so
@@ -43,7 +46,7 @@ struct SmemLayout {
 };
 
 // gather table (u16 entries) | lookup table | 2 groups x 2 staging buffers of
-// R rows | 2 groups' norm partials | 4 mbarriers
+// R rows | 2 groups' norm partials | 5 mbarriers (2 per group + tables)
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
@@ -51,7 +54,7 @@ __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     L.stage = align_up(L.lut + p.lut_n * 8, 128);
     L.red = L.stage + 4 * p.R * p.srow;
     L.bar = align_up(L.red + 2 * (p.G / 32) * p.R * 4, 8);
-    L.total = L.bar + 32;
+    L.total = L.bar + 40;
     return L;
 }
 
@@ -80,7 +83,9 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     constexpr int ES = sizeof(InT);
     uint8_t* s_stage = smem + L.stage + grp * 2 * R * p.srow;
     float* s_red = reinterpret_cast<float*>(smem + L.red) + grp * nwarps * R;
-    uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + L.bar) + 2 * grp;
+    uint64_t* all_bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+    uint64_t* s_bar = all_bars + 2 * grp;
+    uint64_t* tab_bar = all_bars + 4;
 
     auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) {
         const int row0 = tile * R;
@@ -95,24 +100,20 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     const int step = 2 * gridDim.x;
     int tile = blockIdx.x + grp * gridDim.x;
     if (tid == 0) {
-        uint64_t* all = reinterpret_cast<uint64_t*>(smem + L.bar);
-        for (int i = 0; i < 4; ++i) mbar_init(&all[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&all_bars[i], 1);
         fence_mbar_init();
         s_abort[0] = s_abort[1] = 0;
-        // the first copies overlap the table set-up
+        // gather and lookup tables, then each group's first rows: all in flight together
+        const uint32_t lut_bytes = (uint32_t)(p.lut_n * 8);
+        mbar_arrive_expect_tx(tab_bar, (uint32_t)(p.d * 2) + lut_bytes);
+        bulk_g2s(smem + L.gtab, p.gtab, (uint32_t)(p.d * 2), tab_bar);
+        if (lut_bytes) bulk_g2s(smem + L.lut, p.lut, lut_bytes, tab_bar);
         for (int g = 0; g < 2; ++g) {
             const int t0 = blockIdx.x + g * gridDim.x;
-            if (t0 < p.ntiles) issue(all + 2 * g, smem + L.stage + g * 2 * R * p.srow, t0, 0);
+            if (t0 < p.ntiles) issue(all_bars + 2 * g, smem + L.stage + g * 2 * R * p.srow, t0, 0);
         }
     }
-    {
-        const uint4* g = reinterpret_cast<const uint4*>(p.gtab);
-        uint4* sg = reinterpret_cast<uint4*>(smem + L.gtab);
-        for (int i = tid; i < p.d / 8; i += blockDim.x) sg[i] = g[i];
-        LutEntry* sl = reinterpret_cast<LutEntry*>(smem + L.lut);
-        for (int i = tid; i < p.lut_n; i += blockDim.x) sl[i] = p.lut[i];
-    }
-    __syncthreads();
+    __syncthreads();  // barriers initialised
 
     const float2 G2 = make_float2(p.G_lut, p.G_lut);
     const float2 M2 = make_float2(kLutMagic, kLutMagic);
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
             issue(s_bar, s_stage, next, st ^ 1);  // streams in while this tile is computed
             pending_other = 1;
         }
+        if (it == 0 && !mbar_wait_bounded(tab_bar, 0u)) s_abort[grp] = 1;
         if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort[grp] = 1;
         group_sync(1 + grp, G);
         if (s_abort[grp]) {
@@ -142,7 +144,11 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
         const bool valid = active && row < p.M;
 
         // ---- A1 + A2: gather sigma_k x[pi(k)] (sign = top bit of the entry) ----
+        // and the sum of squares of the gathered values: ||x'|| = ||x|| since
+        // Pi_d is orthogonal, so the row norm is reduced across the row's
+        // threads while the butterflies run
         float2 v2[L2H];
+        float2 acc = make_float2(0.f, 0.f);
         if (valid) {
             const uint32_t rowp = smem_u32(s_stage) + (uint32_t)(st * R * p.srow + r * p.srow);
 #pragma unroll
@@ -168,12 +174,21 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                         f1 = __uint_as_float(r1 ^ ((e1 & 0x8000u) << 16));
                     }
                     v2[c * 4 + e] = make_float2(f0, f1);
+                    acc = f2fma(v2[c * 4 + e], v2[c * 4 + e], acc);
                 }
             }
         } else {
 #pragma unroll
             for (int j = 0; j < L2H; ++j) v2[j] = make_float2(0.f, 0.f);
         }
+
+        // ---- A4 (first half): this block's sum of squares, summed over the
+        // row's blocks within the warp, one partial per warp and row ----------
+        float ss = acc.x + acc.y;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+            if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane < R) s_red[warp * R + lane] = ss;
 
         // ---- A3: unnormalised Walsh-Hadamard butterflies, Sylvester order ------
 #pragma unroll
@@ -193,22 +208,13 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
             }
         }
 
-        // ---- A4: row norm (sum of squares of the block, then across blocks) ----
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < L2H; ++j) acc = f2fma(v2[j], v2[j], acc);
-        float ss = acc.x + acc.y;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
-            if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane < R) s_red[warp * R + lane] = ss;
+        // ---- A4 (second half): the row norm s = ||x'|| ------------------------
         group_sync(1 + grp, G);
         float ssum = 0.f;
         for (int w = 0; w < nwarps; ++w) ssum += s_red[w * R + r];
-        const float su = __fsqrt_rn(ssum);  // ||H u|| before the 1/sqrt(h) of H_h
+        const float s = __fsqrt_rn(ssum);
 
         if (valid) {
-            const float s = su * p.rsqrt_h;  // ||x'|| with the 1/sqrt(h) of H_h applied
             if (b == 0) {
                 if constexpr (MODE == 0) p.s_out[row] = s;
                 if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
@@ -226,52 +232,60 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
                 // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
                 constexpr int NB = BITS == 6 ? H : H * BITS / 8;  // packed bytes per h-block
                 constexpr int NW = NB / 4;
+                constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
                 constexpr int PER = BITS == 6 ? 4 : 32 / BITS;     // codes per 32-bit word
                 constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
-                uint32_t words[NW];
-                const bool finite = su <= FLT_MAX;  // false for inf and NaN
-                if (finite) {
-                    const float inv = 1.0f / (su + p.eps_h);
+                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
+                auto put = [&](int w0, const uint32_t (&words)[CW]) {
+                    if constexpr (CW == 4)
+                        reinterpret_cast<uint4*>(dst)[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
+                    else if constexpr (CW == 2)
+                        reinterpret_cast<uint2*>(dst)[w0 >> 1] = make_uint2(words[0], words[1]);
+                    else
+                        reinterpret_cast<uint32_t*>(dst)[w0] = words[0];
+                };
+                // s <= s_max keeps every butterfly value below sqrt(h) s (finite),
+                // so |v| <= 1 up to rounding and the table index stays in range;
+                // larger, infinite and NaN norms take the middle cell
+                if (s <= p.s_max) {
+                    // x'/(s+eps) = (H u / sqrt(h)) / (s + eps): one multiplier for the unnormalised butterflies
+                    const float inv = p.rsqrt_h / (s + p.eps);
                     const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-                    for (int wi = 0; wi < NW; ++wi) {
-                        // codes of this word, highest position first: acc = acc * 2^bits + code
-                        uint32_t acc_w = 0;
+                    for (int w0 = 0; w0 < NW; w0 += CW) {
+                        uint32_t words[CW];
 #pragma unroll
-                        for (int k = PER - 2; k >= 0; k -= 2) {
-                            const float2 q = f2mul(v2[(wi * PER + k) >> 1], inv2);
-                            const float2 z = f2fma(q, G2, M2);
-                            float T0, T1;
-                            int b0, b1;
-                            const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
-                            const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
-                            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
-                            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
-                            const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
-                            const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
-                            acc_w = (acc_w * SH + i1) * SH + i0;
+                        for (int wj = 0; wj < CW; ++wj) {
+                            const int wi = w0 + wj;
+                            // codes of this word, highest position first: acc = acc * 2^bits + code
+                            uint32_t acc_w = 0;
+#pragma unroll
+                            for (int k = PER - 2; k >= 0; k -= 2) {
+                                const float2 q = f2mul(v2[(wi * PER + k) >> 1], inv2);
+                                const float2 z = f2fma(q, G2, M2);
+                                float T0, T1;
+                                int b0, b1;
+                                const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
+                                const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
+                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
+                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
+                                const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
+                                const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
+                                acc_w = (acc_w * SH + i1) * SH + i0;
+                            }
+                            words[wj] = acc_w;
                         }
-                        words[wi] = acc_w;
+                        put(w0, words);
                     }
                 } else {
-                    const uint32_t mid = (uint32_t)(p.L >> 1);
                     uint32_t wmid = 0;
 #pragma unroll
-                    for (int k = 0; k < PER; ++k) wmid = wmid * SH + mid;
+                    for (int k = 0; k < PER; ++k) wmid = wmid * SH + (uint32_t)(p.L >> 1);
+                    uint32_t words[CW];
 #pragma unroll
-                    for (int wi = 0; wi < NW; ++wi) words[wi] = wmid;
-                }
-                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
-                if constexpr (NB % 16 == 0) {
+                    for (int wj = 0; wj < CW; ++wj) words[wj] = wmid;
 #pragma unroll
-                    for (int i = 0; i < NW; i += 4)
-                        reinterpret_cast<uint4*>(dst)[i >> 2] = make_uint4(words[i], words[i + 1], words[i + 2], words[i + 3]);
-                } else if constexpr (NB % 8 == 0) {
-#pragma unroll
-                    for (int i = 0; i < NW; i += 2) reinterpret_cast<uint2*>(dst)[i >> 1] = make_uint2(words[i], words[i + 1]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < NW; ++i) reinterpret_cast<uint32_t*>(dst)[i] = words[i];
+                    for (int w0 = 0; w0 < NW; w0 += CW) put(w0, words);
                 }
             }
         }

@@ -26,7 +26,8 @@ struct RpbhParams {
     float* y_out;          // test hook: x' (fp32)
     float* norm_out;       // test hook: ||x'||
     float rsqrt_h;         // 1/sqrt(h)
-    float eps_h;           // eps * sqrt(h) (the split's eps in unnormalised units)
+    float eps;             // the split's eps
+    float s_max;           // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
 };
 
 int rpbh_smem_bytes(const RpbhParams& p);
