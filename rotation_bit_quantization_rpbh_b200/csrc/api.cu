@@ -77,13 +77,16 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     while (R < 32 && 2 * R * nb <= 128 && 4 * (2 * R) * p.srow <= 180 * 1024) R *= 2;
     p.R = R;
     p.G = (nb * R + 31) / 32 * 32;
-    p.T = 2 * p.G;
-    if (p.T > 256) return OQ_ERR_UNSUPPORTED;
+    if (p.G > 128) return OQ_ERR_UNSUPPORTED;
+    p.lut_n = mode != 2 ? (int)cb->lut.size() : 0;
+    // warp groups: as many (up to three) as shared memory holds
+    for (p.NG = kMaxGroups; p.NG > 1; --p.NG)
+        if (rpbh_smem_bytes(p) <= 227 * 1024) break;
+    p.T = p.NG * p.G;
     p.ntiles = (M + R - 1) / R;
     p.gtab = plan->dev.gtab;
     if (mode != 2) {
         p.lut = dcb->lut;
-        p.lut_n = (int)cb->lut.size();
         p.lut_off = -(int)kLutMagicBits - cb->kmin;
         p.G_lut = cb->G;
         p.L = cb->L;

@@ -8,8 +8,8 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM, each split into two warp groups that take
-//     alternate tiles of R rows and run out of phase (own staging buffers,
+//   - persistent CTAs, one per SM, each split into NG (1-3) warp groups that
+//     take interleaved tiles of R rows and run out of phase (own staging buffers,
 //     mbarriers and named barriers), so one group's gathers overlap the
 //     other's butterflies and table lookups; a group stages its rows with
 //     1-D bulk copies (cp.async.bulk), double buffered so its next tile
@@ -45,16 +45,16 @@ struct SmemLayout {
     int gtab, lut, stage, red, bar, total;
 };
 
-// gather table (u16 entries) | lookup table | 2 groups x 2 staging buffers of
-// R rows | 2 groups' norm partials | 5 mbarriers (2 per group + tables)
+// gather table (u16 entries) | lookup table | NG groups x 2 staging buffers
+// of R rows | NG groups' norm partials | mbarriers (2 per group + tables)
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
     L.lut = align_up(p.d * 2, 16);
     L.stage = align_up(L.lut + p.lut_n * 8, 128);
-    L.red = L.stage + 4 * p.R * p.srow;
-    L.bar = align_up(L.red + 2 * (p.G / 32) * p.R * 4, 8);
-    L.total = L.bar + 40;
+    L.red = L.stage + p.NG * 2 * p.R * p.srow;
+    L.bar = align_up(L.red + p.NG * (p.G / 32) * p.R * 4, 8);
+    L.total = L.bar + 8 * (2 * p.NG + 1);
     return L;
 }
 
@@ -63,18 +63,18 @@ __device__ __forceinline__ void group_sync(int id, int count) {
 }
 
 template <typename InT, int H, int BITS, int MODE>
-__global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) {
+__global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
-    __shared__ int s_abort[2];
+    __shared__ int s_abort[kMaxGroups];
 
-    // Two warp groups per CTA work through alternate tiles independently (own
-    // staging buffers, mbarriers and named barrier), so one group's gathers
-    // overlap the other's butterflies and table lookups.
+    // NG warp groups per CTA work through interleaved tiles independently
+    // (own staging buffers, mbarriers and named barrier), so one group's
+    // gathers overlap the others' butterflies and table lookups.
     const int tid = threadIdx.x;
-    const int G = p.G, R = p.R, nb = p.nb;
-    const int grp = tid >= G ? 1 : 0;
+    const int G = p.G, R = p.R, nb = p.nb, NG = p.NG;
+    const int grp = tid / G;
     const int tg = tid - grp * G;
     const int r = tg & (R - 1);
     const int b = tg / R;
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
     float* s_red = reinterpret_cast<float*>(smem + L.red) + grp * nwarps * R;
     uint64_t* all_bars = reinterpret_cast<uint64_t*>(smem + L.bar);
     uint64_t* s_bar = all_bars + 2 * grp;
-    uint64_t* tab_bar = all_bars + 4;
+    uint64_t* tab_bar = all_bars + 2 * NG;
 
     auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) {
         const int row0 = tile * R;
@@ -96,19 +96,19 @@ __global__ void __launch_bounds__(256, 1) rpbh_quant_kernel(const RpbhParams p) 
         for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &bars[st]);
     };
 
-    // this group's tiles: blockIdx.x + (2k + grp) * gridDim.x
-    const int step = 2 * gridDim.x;
+    // this group's tiles: blockIdx.x + (NG k + grp) * gridDim.x
+    const int step = NG * gridDim.x;
     int tile = blockIdx.x + grp * gridDim.x;
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(&all_bars[i], 1);
+        for (int i = 0; i < 2 * NG + 1; ++i) mbar_init(&all_bars[i], 1);
         fence_mbar_init();
-        s_abort[0] = s_abort[1] = 0;
+        for (int g = 0; g < kMaxGroups; ++g) s_abort[g] = 0;
         // gather and lookup tables, then each group's first rows: all in flight together
         const uint32_t lut_bytes = (uint32_t)(p.lut_n * 8);
         mbar_arrive_expect_tx(tab_bar, (uint32_t)(p.d * 2) + lut_bytes);
         bulk_g2s(smem + L.gtab, p.gtab, (uint32_t)(p.d * 2), tab_bar);
         if (lut_bytes) bulk_g2s(smem + L.lut, p.lut, lut_bytes, tab_bar);
-        for (int g = 0; g < 2; ++g) {
+        for (int g = 0; g < NG; ++g) {
             const int t0 = blockIdx.x + g * gridDim.x;
             if (t0 < p.ntiles) issue(all_bars + 2 * g, smem + L.stage + g * 2 * R * p.srow, t0, 0);
         }

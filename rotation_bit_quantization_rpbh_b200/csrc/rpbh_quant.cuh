@@ -11,7 +11,7 @@ namespace oq {
 struct RpbhParams {
     const void* x;        // [M, d] rows, bf16 or fp32
     int M, d, nb;         // rows, dimension, h-blocks per row (d / h)
-    int R, T, G;          // rows per tile (power of two), threads per CTA, threads per warp group (T = 2G)
+    int R, T, G, NG;      // rows per tile (power of two), threads per CTA, threads per warp group, groups (T = NG G)
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
     int ntiles;
     const uint16_t* gtab;  // device gather table (chunked, see host.cpp)
@@ -29,6 +29,8 @@ struct RpbhParams {
     float eps;             // the split's eps
     float s_max;           // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
 };
+
+constexpr int kMaxGroups = 3;  // warp groups per CTA (at most 128 threads each)
 
 int rpbh_smem_bytes(const RpbhParams& p);
 
