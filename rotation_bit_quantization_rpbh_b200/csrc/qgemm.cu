@@ -18,8 +18,8 @@
 //               leader CTA one thread issues the pair's MMAs;
 //   warps 2-17  decoders, two groups taking alternate K steps: expand
 //               packed codes to bf16 centroid values
-//               (register byte-permute lookups, 64-entry shared table for
-//               6-bit codes) in the 128-byte-swizzled K-major layout, then
+//               (register byte-permute lookups, 64-entry static shared
+//               table for 6-bit codes) in the 128-byte-swizzled K-major layout, then
 //               signal the leader's "stage full" barrier: the leader's own
 //               warps arrive, the peer's warps complete transaction bytes on
 //               it with st.async (asynchronous, cluster-scope release), so no
@@ -66,10 +66,10 @@ __host__ __device__ constexpr int p_stages(int ba, int bw) {
                ? (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw)
                : P_MAX;
 }
-// decoded ring | packed ring | 6-bit tables (256 B) | epilogue r and bias of a
-// tile (1 KB) | barriers (256 B) | alignment slack (1 KB)
+// decoded ring | packed ring | epilogue r and bias of a tile (1 KB) |
+// barriers (256 B) | alignment slack (1 KB); the 6-bit tables are static
 __host__ __device__ constexpr int smem_bytes(int ba, int bw) {
-    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 256 + 1024 + 256 + 1024;
+    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 1024 + 256 + 1024;
 }
 
 struct QgemmParams {
@@ -222,20 +222,22 @@ __device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
 // centroid magnitude m = j & 7 (j >= 8) or m = ~j & 7 (j < 8), negative for
 // j < 8.  tab holds the high bytes of magnitudes 0..7 (words 0, 1) and their
 // low bytes (words 2, 3); one byte-permute per half-word picks 4 high bytes,
-// one the 4 low bytes, and a third, in its sign-replicate mode, marks the
-// lanes with j < 8.
+// one the 4 low bytes.  A third permute of w and w << 4 lines up bit 3 of
+// each code (j >= 8) with the top bit of its value's high byte, where one
+// logic op sets the sign of the codes with j < 8.
 __device__ __forceinline__ uint4 decode8_4bit(uint32_t w, const uint32_t tab[4]) {
     const uint32_t s7 = __umulhi(w & 0x88888888u, 0xE0000000u);  // 7 in each nibble with j >= 8
     const uint32_t mw = ~(w ^ s7) & 0x77777777u;                   // magnitude per nibble
+    const uint32_t w4 = w << 4;
     uint32_t out[4];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const uint32_t sel = half ? (mw >> 16) : mw;
-        const uint32_t wh = half ? (w >> 16) : w;
         uint32_t hi = prmt(tab[0], tab[1], sel);
         const uint32_t lo = prmt(tab[2], tab[3], sel);
-        const uint32_t neg = prmt(0x7f7f7f7fu, 0x7f7f7f7fu, wh);  // 0x7f where j < 8, 0x00 where j >= 8
-        hi |= (neg << 7) & 0x80808080u;
+        // byte i: bit 7 = bit 3 of code 4 half + i (even codes from w << 4, odd codes from w)
+        const uint32_t pos = prmt(w, w4, half ? 0x3726u : 0x1504u);
+        hi |= ~pos & 0x80808080u;
         out[2 * half] = prmt(lo, hi, 0x5140u);
         out[2 * half + 1] = prmt(lo, hi, 0x7362u);
     }
@@ -258,15 +260,26 @@ __device__ __forceinline__ uint4 decode8_2bit(uint32_t x, const uint32_t tab[4])
                       prmt(tab[0], tab[1], mad_hi(z1, 0x110000u, 0x4040u)));
 }
 
-// 6-bit codes, one per byte: 64-entry bf16 table in shared memory (128
-// bytes, one bank row: the lookups of a warp never conflict).
-__device__ __forceinline__ uint4 decode8_6bit(uint32_t a, uint32_t b, const uint16_t* tab) {
-    a &= 0x3f3f3f3fu;
-    b &= 0x3f3f3f3fu;
-    const uint32_t e0 = tab[a & 0xffu], e1 = tab[prmt(a, 0u, 0x4441u)], e2 = tab[prmt(a, 0u, 0x4442u)],
-                   e3 = tab[a >> 24];
-    const uint32_t e4 = tab[b & 0xffu], e5 = tab[prmt(b, 0u, 0x4441u)], e6 = tab[prmt(b, 0u, 0x4442u)],
-                   e7 = tab[b >> 24];
+// 6-bit codes, one per byte: 64-entry bf16 tables in static shared memory
+// (A's at entries 0-63, W's at 64-127).  A table's 128 bytes are one bank
+// row, so the lookups of a warp never conflict.  Its address is a link-time
+// constant folded into each load; the codes are extracted as byte offsets
+// (2 x code).
+__shared__ __align__(256) uint16_t g_t6[128];
+
+template <int TAB>
+__device__ __forceinline__ uint32_t t6_at(uint32_t byte_off) {
+    return *reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(g_t6 + 64 * TAB) + byte_off);
+}
+
+template <int TAB>
+__device__ __forceinline__ uint4 decode8_6bit(uint32_t a, uint32_t b) {
+    a = (a << 1) & 0x7e7e7e7eu;  // 2 x code in each byte
+    b = (b << 1) & 0x7e7e7e7eu;
+    const uint32_t e0 = t6_at<TAB>(a & 0xffu), e1 = t6_at<TAB>(prmt(a, 0u, 0x4441u)),
+                   e2 = t6_at<TAB>(prmt(a, 0u, 0x4442u)), e3 = t6_at<TAB>(a >> 24);
+    const uint32_t e4 = t6_at<TAB>(b & 0xffu), e5 = t6_at<TAB>(prmt(b, 0u, 0x4441u)),
+                   e6 = t6_at<TAB>(prmt(b, 0u, 0x4442u)), e7 = t6_at<TAB>(b >> 24);
     return make_uint4(e0 + e1 * 65536u, e2 + e3 * 65536u, e4 + e5 * 65536u, e6 + e7 * 65536u);
 }
 
@@ -294,11 +307,11 @@ __device__ __forceinline__ Packed8<BITS> load_unit(const uint8_t* src) {
     return u;
 }
 
-template <int BITS>
-__device__ __forceinline__ uint4 decode_unit(Packed8<BITS> u, const uint32_t tab[4], const uint16_t* tab6) {
+template <int BITS, int TAB>
+__device__ __forceinline__ uint4 decode_unit(Packed8<BITS> u, const uint32_t tab[4]) {
     if constexpr (BITS == 4) return decode8_4bit(u.a, tab);
     else if constexpr (BITS == 2) return decode8_2bit(u.a, tab);
-    else return decode8_6bit(u.a, u.b, tab6);
+    else return decode8_6bit<TAB>(u.a, u.b);
 }
 
 // One decoder thread's codes of a K step: units (row = t/8 + DEC_ROWS i,
@@ -327,11 +340,11 @@ struct StageValues {
 
 template <int BA, int BW>
 __device__ __forceinline__ void decode_codes(StageValues& v, const StageCodes<BA, BW>& u, const uint32_t tab_a[4],
-                                             const uint32_t tab_w[4], const uint16_t* t6) {
+                                             const uint32_t tab_w[4]) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
-        v.a[i] = decode_unit<BA>(u.a[i], tab_a, t6);
-        v.b[i] = decode_unit<BW>(u.b[i], tab_w, t6 + 64);
+        v.a[i] = decode_unit<BA, 0>(u.a[i], tab_a);
+        v.b[i] = decode_unit<BW, 1>(u.b[i], tab_w);
     }
 }
 
@@ -370,8 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     constexpr int P_STAGES = p_stages(BA, BW);
     uint8_t* dec = smem;
     uint8_t* pk = smem + D_STAGES * DEC_STAGE;
-    uint16_t* t6 = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);
-    uint16_t* epi_r = t6 + 128;     // r_n of the current tile's 256 columns
+    uint16_t* epi_r = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);  // r_n of the tile's 256 columns
     uint16_t* epi_b = epi_r + TN;   // bias of those columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_b + TN);
     uint64_t* pk_full = bars;
@@ -407,8 +419,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (tid < 64) t6[tid] = p.c6a[tid];
-    else if (tid < 128) t6[tid] = p.c6w[tid - 64];
+    if (tid < 64) g_t6[tid] = p.c6a[tid];
+    else if (tid < 128) g_t6[tid] = p.c6w[tid - 64];
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(512u));
@@ -531,7 +543,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 load_codes<BA, BW>(nxt, pa, pa + PKA, srcA, srcB);
             }
             StageValues v;
-            decode_codes<BA, BW>(v, cur, tab_a, tab_w, t6);
+            decode_codes<BA, BW>(v, cur, tab_a, tab_w);
             __syncwarp();
             if (lane == 0) mbar_arrive(&pk_empty[ps_cur]);  // codes of step s are in registers
             if (pending >= 0) publish(pending);
