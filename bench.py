@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ablation", action="store_true",
+                    help="time the rotation ablation (RPBH, Block-RHT, dense Haar) on --workload instead of the layer")
     return ap.parse_args()
 
 
@@ -396,10 +398,84 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+def run_ablation(args):
+    """The page's rotation ablation on one GPU: the fused rotate+quantise
+    kernel with the RPBH plan and with the Block-RHT plan (no permutation),
+    the rotation alone for both (oq_rpbh_apply), and a dense Haar rotation
+    (a cuBLAS bf16 GEMM against a random orthogonal d x d matrix).  Median
+    device time per call over --steps calls, L2 flushed before each."""
+    import numpy as np
+    import torch
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+    from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --ablation needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    w = I.WORKLOADS[args.workload]
+    x = I.make_x(w).to(dev)
+    cb_a = B.codebook(w.d, w.bits_a)
+    plans = {"rpbh": B.rpbh_plan(w.d, w.h, w.plan_seed),
+             "block_rht": B.rotation_plan(w.d, w.h, w.plan_seed, B.OQ_ROT_BLOCK_RHT)}
+    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+    a_idx = torch.empty((w.M, packed), dtype=torch.uint8, device=dev)
+    s = torch.empty(w.M, dtype=torch.float32, device=dev)
+    x_rot = torch.empty((w.M, w.d), dtype=torch.float32, device=dev)
+    # Haar-distributed orthogonal matrix: QR of a Gaussian matrix with the
+    # signs of R's diagonal folded into Q (Mezzadri 2007)
+    g = torch.Generator(device=dev).manual_seed(w.plan_seed)
+    q, r = torch.linalg.qr(torch.randn(w.d, w.d, generator=g, device=dev, dtype=torch.float32))
+    q = q * torch.sign(torch.diagonal(r)).unsqueeze(0)
+    haar_t = q.t().contiguous().to(torch.bfloat16)
+    xb = x.to(torch.bfloat16)
+    y_haar = torch.empty((w.M, w.d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    calls = {
+        "rpbh_quant": lambda: B.quantize_acts(plans["rpbh"], cb_a, x, a_idx, s, stream=stream),
+        "block_rht_quant": lambda: B.quantize_acts(plans["block_rht"], cb_a, x, a_idx, s, stream=stream),
+        "rpbh_rotate": lambda: B.rpbh_apply(plans["rpbh"], x, x_rot, s, stream=stream),
+        "block_rht_rotate": lambda: B.rpbh_apply(plans["block_rht"], x, x_rot, s, stream=stream),
+        "haar_rotate_cublas": lambda: torch.matmul(xb, haar_t, out=y_haar),
+    }
+    ms = {}
+    for name, fn in calls.items():
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+    if B.device_status() != 0:
+        raise SystemExit("a kernel reported a timeout")
+    out = {
+        "metric": "rotation ablation: device ms per call (median)",
+        "workload": w.name, "M": w.M, "d": w.d, "h": w.h, "bits_a": w.bits_a, "steps": args.steps,
+        "ms": ms,
+        "ratios": {
+            "rpbh_over_block_rht_quant": ms["rpbh_quant"] / ms["block_rht_quant"],
+            "rpbh_over_block_rht_rotate": ms["rpbh_rotate"] / ms["block_rht_rotate"],
+            "haar_over_rpbh_rotate": ms["haar_rotate_cublas"] / ms["rpbh_rotate"],
+            "haar_over_rpbh_quant": ms["haar_rotate_cublas"] / ms["rpbh_quant"],
+        },
+        "note": "rotate = oq_rpbh_apply (fp32 x' and norms out); quant = the fused rotate+split+quantise kernel; "
+                "haar = bf16 x @ Q^T with a Haar-random Q, bf16 out (cuBLAS); L2 flushed before every call",
+    }
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.ablation:
+        run_ablation(args)
     else:
         run_ours(args)
 

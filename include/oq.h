@@ -112,6 +112,18 @@ oq_status oq_rpbh_plan_export(const oq_plan_t* plan, int32_t* perm, int8_t* sign
 /* Host-only plan generation (no device tables): same arrays as above. */
 oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign);
 
+/* Rotation variants for the page's rotation ablation [OrbitQuant, section */
+/* 实验 (Experiments), the rotation ablation: Block-RHT, RPBH].            */
+/*   OQ_ROT_RPBH       the plan of oq_rpbh_plan.                           */
+/*   OQ_ROT_BLOCK_RHT  Block-RHT: P_pi = identity; the signs are the first  */
+/*                     d draws of SplitMix64(seed), with the same rule.    */
+/* The variant plan feeds the same calls as an RPBH plan.  Unknown          */
+/* variants return OQ_ERR_INVALID_ARG.                                     */
+#define OQ_ROT_RPBH 0
+#define OQ_ROT_BLOCK_RHT 1
+oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t** out);
+oq_status oq_rotation_plan_host(int d, int h, uint64_t seed, int variant, int32_t* perm, int8_t* sign);
+
 /* (d, h) of a plan.  Host pointers; either may be NULL. */
 oq_status oq_plan_shape(const oq_plan_t* plan, int* d, int* h);
 

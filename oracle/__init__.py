@@ -38,6 +38,7 @@ def lib():
         L.oracle_fd_moments.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double, P, P]
         L.oracle_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_int, P]
         L.oracle_plan.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, P, P]
+        L.oracle_plan_variant.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_int, P, P]
         L.oracle_rpbh.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P]
         L.oracle_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, ctypes.c_int, P,
                                            ctypes.c_double, ctypes.c_int, P, P, P, P]
@@ -94,11 +95,15 @@ def splitmix64(seed, n):
     return out
 
 
-def plan(d, h, seed):
-    """RPBH plan: (perm[d] int32 with (P_pi x)_k = x[perm[k]], sign[d] int8 in {-1,+1})."""
+BLOCK_RHT = 1  # plan variant without the permutation (the page's rotation ablation)
+
+
+def plan(d, h, seed, variant=0):
+    """RPBH plan (variant 0) or Block-RHT plan (variant 1, identity permutation):
+    (perm[d] int32 with (P_pi x)_k = x[perm[k]], sign[d] int8 in {-1,+1})."""
     perm = np.zeros(d, dtype=np.int32)
     sign = np.zeros(d, dtype=np.int8)
-    rc = lib().oracle_plan(d, h, ctypes.c_uint64(seed), _p(perm), _p(sign))
+    rc = lib().oracle_plan_variant(d, h, ctypes.c_uint64(seed), variant, _p(perm), _p(sign))
     if rc != 0:
         raise ValueError("bad plan arguments")
     return perm, sign

@@ -269,16 +269,26 @@ void oracle_splitmix64(uint64_t seed, int n, uint64_t* out) {
     for (int i = 0; i < n; ++i) out[i] = splitmix64_next(&s);
 }
 
+int oracle_plan_variant(int d, int h, uint64_t seed, int variant, int32_t* perm, int8_t* sign);
+
 int oracle_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign) {
-    if (d <= 0 || h <= 0 || d % h != 0) return -1;
+    return oracle_plan_variant(d, h, seed, 0, perm, sign);
+}
+
+/* variant 0: RPBH (above).  variant 1: Block-RHT, the page's ablation
+ * without the permutation (section 实验, rotation ablation): pi is the
+ * identity and the d signs are the generator's first d draws. */
+int oracle_plan_variant(int d, int h, uint64_t seed, int variant, int32_t* perm, int8_t* sign) {
+    if (d <= 0 || h <= 0 || d % h != 0 || (variant != 0 && variant != 1)) return -1;
     uint64_t s = seed;
     for (int i = 0; i < d; ++i) perm[i] = i;
-    for (int i = d - 1; i >= 1; --i) {
-        uint64_t j = splitmix64_next(&s) % (uint64_t)(i + 1);
-        int32_t t = perm[i];
-        perm[i] = perm[j];
-        perm[j] = t;
-    }
+    if (variant == 0)
+        for (int i = d - 1; i >= 1; --i) {
+            uint64_t j = splitmix64_next(&s) % (uint64_t)(i + 1);
+            int32_t t = perm[i];
+            perm[i] = perm[j];
+            perm[j] = t;
+        }
     for (int k = 0; k < d; ++k) sign[k] = (splitmix64_next(&s) >> 63) ? -1 : 1;
     return 0;
 }

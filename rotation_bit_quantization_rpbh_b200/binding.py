@@ -19,13 +19,15 @@ LIB_PATH = os.path.join(_HERE, "liboq.so")
 
 OQ_OK = 0
 OQ_BF16, OQ_F32 = 0, 1
+OQ_ROT_RPBH, OQ_ROT_BLOCK_RHT = 0, 1
 _STATUS = {0: "OQ_OK", 1: "OQ_ERR_INVALID_ARG", 2: "OQ_ERR_UNSUPPORTED", 3: "OQ_ERR_ALIGNMENT", 4: "OQ_ERR_CUDA",
            5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE", 8: "OQ_ERR_TOO_LARGE"}
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 # every symbol include/oq.h declares
 EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf16", "oq_codebook_shape",
-           "oq_codebook_free", "oq_rpbh_plan", "oq_rpbh_plan_export", "oq_rpbh_plan_host", "oq_plan_shape",
+           "oq_codebook_free", "oq_rpbh_plan", "oq_rpbh_plan_export", "oq_rpbh_plan_host", "oq_rotation_plan",
+           "oq_rotation_plan_host", "oq_plan_shape",
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status"]
 
@@ -61,6 +63,8 @@ def lib():
                     "oq_rpbh_plan": ([I, I, U64, P], I),
                     "oq_rpbh_plan_export": ([P, P, P], I),
                     "oq_rpbh_plan_host": ([I, I, U64, P, P], I),
+                    "oq_rotation_plan": ([I, I, U64, I, P], I),
+                    "oq_rotation_plan_host": ([I, I, U64, I, P, P], I),
                     "oq_plan_shape": ([P, P, P], I),
                     "oq_plan_free": ([P], None),
                     "oq_quantize_weights": ([P, P, P, I, I, P, P, P], I),
@@ -143,13 +147,17 @@ class Codebook:
 
 
 class Plan:
-    """RPBH plan (library-owned handle with device tables on the current device)."""
+    """RPBH plan, or a rotation-ablation variant of it (library-owned handle
+    with device tables on the current device)."""
 
-    def __init__(self, d, h, seed):
+    def __init__(self, d, h, seed, variant=OQ_ROT_RPBH):
         hp = ctypes.c_void_p()
-        _check(lib().oq_rpbh_plan(d, h, ctypes.c_uint64(seed), ctypes.byref(hp)), "oq_rpbh_plan")
+        if variant == OQ_ROT_RPBH:
+            _check(lib().oq_rpbh_plan(d, h, ctypes.c_uint64(seed), ctypes.byref(hp)), "oq_rpbh_plan")
+        else:
+            _check(lib().oq_rotation_plan(d, h, ctypes.c_uint64(seed), variant, ctypes.byref(hp)), "oq_rotation_plan")
         self._h = hp
-        self.d, self.h, self.seed = d, h, seed
+        self.d, self.h, self.seed, self.variant = d, h, seed, variant
 
     @property
     def handle(self):
@@ -176,6 +184,20 @@ def codebook(d, bits):
 
 def rpbh_plan(d, h, seed):
     return Plan(d, h, seed)
+
+
+def rotation_plan(d, h, seed, variant):
+    return Plan(d, h, seed, variant)
+
+
+def rotation_plan_host(d, h, seed, variant):
+    import numpy as np
+
+    perm = np.zeros(d, dtype=np.int32)
+    sign = np.zeros(d, dtype=np.int8)
+    _check(lib().oq_rotation_plan_host(d, h, ctypes.c_uint64(seed), variant, perm.ctypes.data_as(ctypes.c_void_p),
+                                       sign.ctypes.data_as(ctypes.c_void_p)), "oq_rotation_plan_host")
+    return perm, sign
 
 
 def rpbh_plan_host(d, h, seed):

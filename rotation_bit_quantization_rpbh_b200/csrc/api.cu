@@ -197,21 +197,31 @@ static oq_status check_plan_args(int d, int h) {
 }
 
 oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign) {
+    return oq_rotation_plan_host(d, h, seed, OQ_ROT_RPBH, perm, sign);
+}
+
+oq_status oq_rotation_plan_host(int d, int h, uint64_t seed, int variant, int32_t* perm, int8_t* sign) {
     oq_status s = check_plan_args(d, h);
     if (s != OQ_OK) return s;
+    if (variant != OQ_ROT_RPBH && variant != OQ_ROT_BLOCK_RHT) return OQ_ERR_INVALID_ARG;
     std::vector<int32_t> pv(d);
     std::vector<int8_t> sv(d);
-    make_plan(d, h, seed, pv.data(), sv.data());
+    make_plan(d, h, seed, pv.data(), sv.data(), variant);
     if (perm) std::memcpy(perm, pv.data(), sizeof(int32_t) * d);
     if (sign) std::memcpy(sign, sv.data(), d);
     return OQ_OK;
 }
 
 oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out) {
+    return oq_rotation_plan(d, h, seed, OQ_ROT_RPBH, out);
+}
+
+oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t** out) {
     if (!out) return OQ_ERR_INVALID_ARG;
     *out = nullptr;
     oq_status s = check_plan_args(d, h);
     if (s != OQ_OK) return s;
+    if (variant != OQ_ROT_RPBH && variant != OQ_ROT_BLOCK_RHT) return OQ_ERR_INVALID_ARG;
     const int dev = current_device();
     if (dev < 0) return OQ_ERR_CUDA;
     oq_plan_t* p = new (std::nothrow) oq_plan_s();
@@ -222,7 +232,7 @@ oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out) {
     p->device = dev;
     p->perm.resize(d);
     p->sign.resize(d);
-    make_plan(d, h, seed, p->perm.data(), p->sign.data());
+    make_plan(d, h, seed, p->perm.data(), p->sign.data(), variant);
     build_gather_table(p, p->gtab_host);
     void* ptr = nullptr;
     if (cudaMalloc(&ptr, sizeof(uint16_t) * d) != cudaSuccess) {

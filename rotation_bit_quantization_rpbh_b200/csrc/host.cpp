@@ -269,7 +269,7 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
 // RPBH plan: SplitMix64 (Steele, Lea & Flood 2014) drives a Fisher-Yates
 // (Durstenfeld) shuffle of the identity, then the Rademacher signs.
 // ---------------------------------------------------------------------------
-void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign) {
+void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int variant) {
     (void)h;
     uint64_t state = seed;
     auto next = [&state]() {
@@ -280,10 +280,13 @@ void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign) {
         return z ^ (z >> 31);
     };
     for (int i = 0; i < d; ++i) perm[i] = i;
-    for (int i = d - 1; i > 0; --i) {
-        const int j = (int)(next() % (uint64_t)(i + 1));
-        std::swap(perm[i], perm[j]);
-    }
+    if (variant == OQ_ROT_RPBH)
+        for (int i = d - 1; i > 0; --i) {
+            const int j = (int)(next() % (uint64_t)(i + 1));
+            std::swap(perm[i], perm[j]);
+        }
+    // Block-RHT (the ablation without P_pi): identity permutation, signs
+    // from the first d draws of the same generator
     for (int k = 0; k < d; ++k) sign[k] = (next() >> 63) ? (int8_t)-1 : (int8_t)1;
 }
 

@@ -63,7 +63,7 @@ namespace oq {
 
 // host-side pieces (host.cpp)
 oq_status build_codebook(int d, int bits, oq_codebook_t* cb);
-void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign);
+void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int variant);
 void build_gather_table(const oq_plan_t* p, std::vector<uint16_t>& out);
 uint16_t bf16_round(double x);
 

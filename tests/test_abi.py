@@ -60,6 +60,28 @@ def test_library_plan_matches_oracle(d, h, seed):
     np.testing.assert_array_equal(s1, s2)
 
 
+@pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (4096, 128, 3)])
+def test_library_block_rht_plan_matches_oracle(d, h, seed):
+    p1, s1 = B.rotation_plan_host(d, h, seed, B.OQ_ROT_BLOCK_RHT)
+    p2, s2 = oracle.plan(d, h, seed, variant=oracle.BLOCK_RHT)
+    np.testing.assert_array_equal(p1, p2)
+    np.testing.assert_array_equal(s1, s2)
+    p3, s3 = B.rotation_plan_host(d, h, seed, B.OQ_ROT_RPBH)  # the RPBH variant is oq_rpbh_plan's plan
+    p4, s4 = B.rpbh_plan_host(d, h, seed)
+    np.testing.assert_array_equal(p3, p4)
+    np.testing.assert_array_equal(s3, s4)
+
+
+def test_unknown_rotation_variant_is_rejected():
+    import ctypes
+
+    L = B.lib()
+    perm = np.zeros(256, dtype=np.int32)
+    sign = np.zeros(256, dtype=np.int8)
+    assert L.oq_rotation_plan_host(256, 64, ctypes.c_uint64(0), 7, perm.ctypes.data_as(ctypes.c_void_p),
+                                   sign.ctypes.data_as(ctypes.c_void_p)) == 1
+
+
 def test_argument_checks_on_host_calls():
     L = B.lib()
     import ctypes

@@ -111,3 +111,23 @@ def test_workload_at_full_size(cuda_device, name):
     full = name == "tiny_w4a4"
     stats = _run_layer(cuda_device, w.M, w.d, w.N, w.h, w.bits_w, w.bits_a, x, W, w.plan_seed, full_check=full)
     print(name, stats)
+
+
+@pytest.mark.parametrize("M,d,h,ba", [(300, 512, 128, 4), (96, 1536, 128, 6)])
+def test_block_rht_variant_matches_oracle(cuda_device, M, d, h, ba):
+    """The rotation ablation's Block-RHT plan (no permutation) through the
+    same kernels: rotation, norms and codes against the oracle's variant."""
+    plan = B.rotation_plan(d, h, 21, B.OQ_ROT_BLOCK_RHT)
+    perm, sign = oracle.plan(d, h, 21, variant=oracle.BLOCK_RHT)
+    pe, se = plan.export()
+    np.testing.assert_array_equal(pe, perm)
+    np.testing.assert_array_equal(se, sign)
+    g = torch.Generator().manual_seed(21)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    cb_a, ocb_a = B.codebook(d, ba), oracle.codebook(d, ba)
+    a_idx, s = B.quantize_acts(plan, cb_a, x.to(cuda_device))
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    rows = np.arange(M)
+    check_rotation(plan, x, rows, h, perm, sign, cuda_device)
+    check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb_a, ocb_a, "acts")

@@ -116,6 +116,20 @@ def test_plan_permutation_is_uniform():
     assert np.all(np.abs(sign_sum) < 5 * math.sqrt(n))
 
 
+def test_block_rht_plan_is_identity_with_the_first_draws_as_signs():
+    """The ablation plan without P_pi: identity permutation; sign k is the top
+    bit of the k-th SplitMix64 output (the generator is pinned above)."""
+    d = 256
+    perm, sign = oracle.plan(d, 64, 1234567, variant=oracle.BLOCK_RHT)
+    np.testing.assert_array_equal(perm, np.arange(d))
+    draws = oracle.splitmix64(1234567, d)
+    np.testing.assert_array_equal(sign, np.where((draws >> np.uint64(63)) == 1, -1, 1))
+    # the RPBH plan of the same seed takes its signs after the d - 1 shuffle draws
+    _, sign_rpbh = oracle.plan(d, 64, 1234567)
+    draws = oracle.splitmix64(1234567, 2 * d - 1)
+    np.testing.assert_array_equal(sign_rpbh, np.where((draws[d - 1:] >> np.uint64(63)) == 1, -1, 1))
+
+
 def test_plan_rejects_ragged_blocks():
     with pytest.raises(ValueError):
         oracle.plan(100, 64, 0)
