@@ -50,7 +50,7 @@ namespace {
 constexpr int TM = 256, TN = 256, BK = 64;  // pair tile and K step
 constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one CTA
 constexpr int D_STAGES = 4;                 // decoded ring
-constexpr int P_MAX = 6;                    // packed ring depth (fewer when the packed stage is large)
+constexpr int P_MAX = 10;                   // packed ring depth (fewer when the packed stage is large)
 constexpr int NDEC_WARPS = 16;
 constexpr int NGROUPS = 2;                        // decoder groups, taking alternate K steps
 constexpr int GROUP_WARPS = NDEC_WARPS / NGROUPS;
@@ -67,9 +67,9 @@ __host__ __device__ constexpr int p_stages(int ba, int bw) {
                : P_MAX;
 }
 // decoded ring | packed ring | epilogue r and bias of a tile (1 KB) |
-// barriers (256 B) | alignment slack (1 KB); the 6-bit tables are static
+// barriers (512 B) | alignment slack (1 KB); the 6-bit tables are static
 __host__ __device__ constexpr int smem_bytes(int ba, int bw) {
-    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 1024 + 256 + 1024;
+    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 1024 + 512 + 1024;
 }
 
 struct QgemmParams {
@@ -527,14 +527,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         ps.idx = grp;
         ds.idx = grp;
         int pending = -1;  // decoded slot stored but not yet published
+        // A packed slot is released as soon as its codes are in registers
+        // (the arrive's release orders the loads before it), so each slot is
+        // held for about one step of the group.
         StageCodes<BA, BW> cur;
         bool ok = grp < total && wait_or_abort<false>(&pk_full[ps.idx], 0u, abort_flag);
-        if (ok) load_codes<BA, BW>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+        if (ok) {
+            load_codes<BA, BW>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pk_empty[ps.idx]);
+        }
         for (int s = grp; ok && s < total; s += NGROUPS) {
             StageCodes<BA, BW> nxt;
-            const int ps_cur = ps.idx;
             ps.advance(NGROUPS);
-            if (s + NGROUPS < total) {
+            const bool more = s + NGROUPS < total;
+            if (more) {
                 if (!wait_or_abort<false>(&pk_full[ps.idx], ps.phase, abort_flag)) {
                     ok = false;
                     break;
@@ -545,7 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             StageValues v;
             decode_codes<BA, BW>(v, cur, tab_a, tab_w);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pk_empty[ps_cur]);  // codes of step s are in registers
+            if (lane == 0 && more) mbar_arrive(&pk_empty[ps.idx]);  // the next step's codes are in registers
             if (pending >= 0) publish(pending);
             if (!wait_or_abort<false>(&dec_empty[ds.idx], ds.phase ^ 1u, abort_flag)) {
                 ok = false;
