@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the fp8 variant of the product (oq_qgemm_fp8: e4m3 centroid values)")
     ap.add_argument("--ablation", action="store_true",
                     help="time the rotation ablation (RPBH, Block-RHT, dense Haar) on --workload instead of the layer")
     return ap.parse_args()
@@ -290,9 +292,11 @@ def run_ours(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
     stream = torch.cuda.current_stream()
 
+    gemm = B.qgemm_fp8 if args.fp8 else B.qgemm
+
     def step():
         B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
-        B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+        gemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -316,7 +320,7 @@ def run_ours(args):
         ev[i][0].record(stream)
         B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
         ev[i][1].record(stream)
-        B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+        gemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -368,7 +372,7 @@ def run_ours(args):
             ev_in[b].record(s_in)
             s_cmp.wait_event(ev_in[b])
             s_cmp.wait_event(ev_out[b])  # the copy-out that last read ys[b] is done
-            B.qlinear(plan, cb_a, cb_w, xs[b], w_idx, w_r, y=ys[b], workspace=wss[b], stream=s_cmp)
+            B.qlinear(plan, cb_a, cb_w, xs[b], w_idx, w_r, y=ys[b], workspace=wss[b], stream=s_cmp, fp8=args.fp8)
             ev_cmp[b].record(s_cmp)
             s_out.wait_event(ev_cmp[b])
             with torch.cuda.stream(s_out):
@@ -385,6 +389,10 @@ def run_ours(args):
                "pipeline": "copy-in, oq_qlinear and copy-out on three streams, two buffers deep"}
 
     peaks = measured_peaks()
+    # the fp8 variant's contraction peak: the measured bf16 peak times the
+    # nominal e4m3 / bf16 dense ratio (4.5 / 2.25 PFLOP/s)
+    mma_peak = peaks["bf16_tflops"] * (2.0 if args.fp8 else 1.0)
+    peak_note = peaks["source"] + (" bf16 (burst) x nominal fp8/bf16 ratio 2" if args.fp8 else " (burst)")
     flops = 2.0 * w.M * w.N * w.d
     gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
     step_tflops = flops / (ms * 1e-3) / 1e12
@@ -393,7 +401,7 @@ def run_ours(args):
     out = {
         "metric": METRIC, "value": job_throughput(world, w.M, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "d": w.d, "N": w.N, "h": w.h, "bits_w": w.bits_w,
                    "bits_a": w.bits_a, "x_dtype": w.x_dtype, "tokens_per_gpu": w.M, "global_batch": world * w.M,
                    "parallelism": f"dp{world} (replicated packed W, no collective)",
@@ -401,9 +409,9 @@ def run_ours(args):
         "tflops": step_tflops,
         "breakdown": {"rpbh_quant_ms": ms_rpbh, "qgemm_ms": ms_gemm, "qgemm_tflops": gemm_tflops,
                       "rpbh_quant_gbs": rpbh_gbs},
-        "roofline": {"bound": "tensor", "kernel": "qgemm", "achieved": gemm_tflops, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops"],
-                     "traffic": committed_traffic("qgemm", w.name), "peak_source": peaks["source"] + " (burst)",
+        "roofline": {"bound": "tensor", "kernel": "qgemm_fp8" if args.fp8 else "qgemm", "achieved": gemm_tflops,
+                     "peak": mma_peak, "unit": "TFLOP/s", "frac": gemm_tflops / mma_peak,
+                     "traffic": None if args.fp8 else committed_traffic("qgemm", w.name), "peak_source": peak_note,
                      "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
         "roofline_rpbh": {"bound": "hbm", "kernel": "rpbh_quant", "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
                           "unit": "GB/s", "frac": rpbh_gbs / peaks["hbm_gbs"],

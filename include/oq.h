@@ -175,6 +175,22 @@ oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, 
                    const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                    void* stream);
 
+/* fp8 variant of oq_qgemm (a low-precision MMA variant the pages do not   */
+/* describe).  The centroids enter the product as e4m3 values of           */
+/* c_j sqrt(d) (rounded once, nearest-even; oq_codebook_fp8), multiplied   */
+/* on tcgen05 kind::f8f6f4 in fp32; the epilogue applies s_m r_n / d (+bias) */
+/* and rounds to bf16 once.  This trades the bf16 centroid values of       */
+/* oq_qgemm (about 2^-9 relative error each) for e4m3 ones (about 2^-4) in */
+/* exchange for throughput.  Same arguments and layouts as oq_qgemm;       */
+/* d % 128 == 0 (OQ_ERR_UNSUPPORTED otherwise).                             */
+oq_status oq_qgemm_fp8(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                       const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                       void* stream);
+
+/* The fp8 variant's centroid values: out[2^bits] host bytes, e4m3 of     */
+/* c_j sqrt(d) (sign, 4 exponent bits with bias 7, 3 mantissa bits).        */
+oq_status oq_codebook_fp8(const oq_codebook_t* cb, uint8_t* out);
+
 /* Bytes of workspace oq_qlinear needs for M rows (packed activation       */
 /* indices plus their norms, 256-byte aligned sections).                   */
 size_t oq_qlinear_workspace(int M, int d, int bits_a);
@@ -187,6 +203,11 @@ size_t oq_qlinear_workspace(int M, int d, int bits_a);
 oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
                      oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
+
+/* oq_qlinear with the fp8 variant of the product (oq_qgemm_fp8).          */
+oq_status oq_qlinear_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
+                         oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
+                         const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* The full layer without any device allocation.  The paper has no        */

@@ -27,7 +27,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20
 # every symbol include/oq.h declares
 EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf16", "oq_codebook_shape",
            "oq_codebook_free", "oq_rpbh_plan", "oq_rpbh_plan_export", "oq_rpbh_plan_host", "oq_rotation_plan",
-           "oq_rotation_plan_host", "oq_plan_shape",
+           "oq_rotation_plan_host", "oq_plan_shape", "oq_qgemm_fp8", "oq_codebook_fp8",
+           "oq_qlinear_fp8",
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status"]
 
@@ -71,6 +72,9 @@ def lib():
                     "oq_quantize_acts": ([P, P, P, I, I, P, P, P], I),
                     "oq_rpbh_apply": ([P, P, I, I, P, P, P], I),
                     "oq_qgemm": ([P, P, I, I, P, P, P, P, P, P, P], I),
+                    "oq_qgemm_fp8": ([P, P, I, I, P, P, P, P, P, P, P], I),
+                    "oq_codebook_fp8": ([P, P], I),
+                    "oq_qlinear_fp8": ([P, P, P, P, I, I, P, P, I, P, P, P, SZ, P], I),
                     "oq_qlinear_workspace": ([I, I, I], SZ),
                     "oq_qlinear": ([P, P, P, P, I, I, P, P, I, P, P, P, SZ, P], I),
                     "oq_qlinear_noalloc": ([P, P, P, P, I, I, P, P, I, P, P, P], I),
@@ -132,6 +136,14 @@ class Codebook:
         _check(lib().oq_codebook_values(self._h, c.ctypes.data_as(ctypes.c_void_p),
                                         t.ctypes.data_as(ctypes.c_void_p)), "oq_codebook_values")
         return c, t[: self.L - 1]
+
+    def e4m3_bytes(self):
+        """The fp8 variant's centroid values: e4m3 bytes of c_j sqrt(d)."""
+        import numpy as np
+
+        b = np.zeros(self.L, dtype=np.uint8)
+        _check(lib().oq_codebook_fp8(self._h, b.ctypes.data_as(ctypes.c_void_p)), "oq_codebook_fp8")
+        return b
 
     def bf16_bits(self):
         import numpy as np
@@ -252,11 +264,22 @@ def qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
     return y
 
 
+def qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
+    """oq_qgemm with e4m3 centroid values on the fp8 tensor cores."""
+    M, N = a_idx.shape[0], w_idx.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_idx.device)
+    _check(lib().oq_qgemm_fp8(cb_a.handle, cb_w.handle, M, N, _ptr(a_idx), _ptr(s), _ptr(w_idx), _ptr(w_r),
+                              _ptr(bias), _ptr(y), _stream(stream)), "oq_qgemm_fp8")
+    return y
+
+
 def qlinear_workspace(M, d, bits_a):
     return int(lib().oq_qlinear_workspace(M, d, bits_a))
 
 
-def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None):
+def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None, fp8=False):
+    """The full layer x -> y (oq_qlinear; oq_qlinear_fp8 with fp8=True)."""
     M, d = x.shape
     N = w_idx.shape[0]
     if y is None:
@@ -264,9 +287,9 @@ def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, 
     need = qlinear_workspace(M, d, cb_a.bits)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    _check(lib().oq_qlinear(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
-                            _ptr(w_r), N, _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
-           "oq_qlinear")
+    fn, name = (lib().oq_qlinear_fp8, "oq_qlinear_fp8") if fp8 else (lib().oq_qlinear, "oq_qlinear")
+    _check(fn(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx), _ptr(w_r), N,
+              _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)), name)
     return y
 
 

@@ -288,12 +288,13 @@ oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, in
                     static_cast<cudaStream_t>(stream));
 }
 
-oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
-                   const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
-                   void* stream) {
+static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                           const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias,
+                           uint16_t* y, void* stream, bool fp8) {
     if (!cb_a || !cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != cb_w->d) return OQ_ERR_INVALID_ARG;
-    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % 64 != 0) return OQ_ERR_UNSUPPORTED;
+    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % (fp8 ? 128 : 64) != 0)
+        return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;  // an empty batch: activation and output buffers may be null
     if (!a_idx || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
     if (!aligned16(a_idx) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
@@ -313,8 +314,29 @@ oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, 
     a.y = y;
     a.ca_bf16 = cb_a->c_bf16.data();
     a.cw_bf16 = cb_w->c_bf16.data();
+    a.fp8 = fp8;
+    a.ca_e4m3 = cb_a->c_e4m3.data();
+    a.cw_e4m3 = cb_w->c_e4m3.data();
     cudaError_t e = launch_qgemm(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
+}
+
+oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                   const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                   void* stream) {
+    return run_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream, false);
+}
+
+oq_status oq_qgemm_fp8(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
+                       const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                       void* stream) {
+    return run_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream, true);
+}
+
+oq_status oq_codebook_fp8(const oq_codebook_t* cb, uint8_t* out) {
+    if (!cb || !out) return OQ_ERR_INVALID_ARG;
+    std::memcpy(out, cb->c_e4m3.data(), cb->c_e4m3.size());
+    return OQ_OK;
 }
 
 size_t oq_qlinear_workspace(int M, int d, int bits_a) {
@@ -324,9 +346,10 @@ size_t oq_qlinear_workspace(int M, int d, int bits_a) {
     return idx_al + ((size_t)M * sizeof(float) + 255) / 256 * 256;
 }
 
-oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
-                     oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
-                     uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
+                             const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
+                             const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream,
+                             bool fp8) {
     if (!plan || !cb_a || !cb_w) return OQ_ERR_INVALID_ARG;
     if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
@@ -341,7 +364,19 @@ oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_
     float* s = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + idx_al);
     oq_status st = oq_quantize_acts(plan, cb_a, x, dtype, M, a_idx, s, stream);
     if (st != OQ_OK) return st;
-    return oq_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream);
+    return run_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream, fp8);
+}
+
+oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
+                     oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
+                     uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+    return run_qlinear(plan, cb_a, cb_w, x, dtype, M, w_idx, w_r, N, bias, y, workspace, ws_bytes, stream, false);
+}
+
+oq_status oq_qlinear_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
+                         oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
+                         const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+    return run_qlinear(plan, cb_a, cb_w, x, dtype, M, w_idx, w_r, N, bias, y, workspace, ws_bytes, stream, true);
 }
 
 // ---------------------------------------------------------------------------

@@ -223,6 +223,8 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
     for (int j = 0; j + 1 < L; ++j) cb->t32[j] = (float)cb->t[j];
     cb->c_bf16.resize(L);
     for (int j = 0; j < L; ++j) cb->c_bf16[j] = bf16_round(cb->c[j]);
+    cb->c_e4m3.resize(L);
+    for (int j = 0; j < L; ++j) cb->c_e4m3[j] = e4m3_round(cb->c[j] * std::sqrt((double)d));
 
     // Lookup table over v in [-vmax, vmax] with at most one fp32 threshold
     // per bin.  The bins are exactly the kernel's: bin(v) = bits of
@@ -263,6 +265,29 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
     // bulk copy (the extra entry is never indexed)
     if (cb->lut.size() % 2) cb->lut.push_back(cb->lut.back());
     return OQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// e4m3 (8 bits: sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+// infinities; largest finite 448; subnormals k * 2^-9): round to nearest,
+// ties to even, once from the exact value; saturates at +-448.
+// ---------------------------------------------------------------------------
+uint8_t e4m3_round(double v) {
+    const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+    const double a = std::fabs(v);
+    if (std::isnan(a)) return sign | 0x7f;
+    int e = 0;
+    std::frexp(a, &e);                        // a in [2^(e-1), 2^e)
+    const int E = std::max(e - 1, -6);        // binade (subnormals share the 2^-6 spacing)
+    const double q = std::ldexp(1.0, E - 3);  // spacing of 3 mantissa bits
+    double r = std::nearbyint(a / q) * q;     // a / q is exact; the default mode rounds ties to even
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return sign;
+    if (r < std::ldexp(1.0, -6)) return sign | (uint8_t)(r / std::ldexp(1.0, -9));
+    std::frexp(r, &e);
+    const int E2 = e - 1;
+    const int mant = (int)((r / std::ldexp(1.0, E2) - 1.0) * 8.0);
+    return sign | (uint8_t)(((E2 + 7) << 3) | mant);
 }
 
 // ---------------------------------------------------------------------------

@@ -38,6 +38,7 @@ struct oq_codebook_s {
     std::vector<double> t;         // L-1 thresholds
     std::vector<float> t32;        // fp32 thresholds (the kernels' decision values)
     std::vector<uint16_t> c_bf16;  // bf16 centroids as the product uses them
+    std::vector<uint8_t> c_e4m3;   // e4m3 bytes of c_j sqrt(d) (the fp8 product variant)
     // quantiser lookup table over v in [-vmax, vmax]:
     //   bin(v) = rint(v * G) (computed as fmaf(v, G, 1.5*2^23) in fp32)
     //   entry index = bin(v) - kmin
@@ -64,6 +65,7 @@ namespace oq {
 // host-side pieces (host.cpp)
 oq_status build_codebook(int d, int bits, oq_codebook_t* cb);
 void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int variant);
+uint8_t e4m3_round(double v);
 void build_gather_table(const oq_plan_t* p, std::vector<uint16_t>& out);
 uint16_t bf16_round(double x);
 

@@ -47,7 +47,7 @@
 namespace oq {
 namespace {
 
-constexpr int TM = 256, TN = 256, BK = 64;  // pair tile and K step
+constexpr int TM = 256, TN = 256;           // pair tile
 constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one CTA
 constexpr int D_STAGES = 4;                 // decoded ring
 constexpr int P_MAX = 10;                   // packed ring depth (fewer when the packed stage is large)
@@ -59,17 +59,24 @@ constexpr int DEC_UNITS = HM / DEC_ROWS;          // units per decoder thread an
 constexpr int NTHREADS = (2 + NDEC_WARPS + 4) * 32;
 constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 
-__host__ __device__ constexpr int pk_row_bytes(int bits) { return bits == 6 ? BK : BK * bits / 8; }
-__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw) { return HM * pk_row_bytes(ba) + HN * pk_row_bytes(bw); }
-__host__ __device__ constexpr int p_stages(int ba, int bw) {
-    return (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw) < P_MAX
-               ? (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw)
+// A K step fills one 128-byte row of each decoded operand: 64 bf16 values,
+// or 128 e4m3 values in the fp8 variant.
+__host__ __device__ constexpr int bk_codes(bool f8) { return f8 ? 128 : 64; }
+__host__ __device__ constexpr int pk_row_bytes(int bits, bool f8) { return bits == 6 ? bk_codes(f8) : bk_codes(f8) * bits / 8; }
+// packed bytes behind one 16-byte decoded chunk (8 bf16 or 16 e4m3 values)
+__host__ __device__ constexpr int unit_bytes(int bits, bool f8) { return (f8 ? 16 : 8) * (bits == 6 ? 8 : bits) / 8; }
+__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw, bool f8) {
+    return HM * pk_row_bytes(ba, f8) + HN * pk_row_bytes(bw, f8);
+}
+__host__ __device__ constexpr int p_stages(int ba, int bw, bool f8) {
+    return (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw, f8) < P_MAX
+               ? (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw, f8)
                : P_MAX;
 }
 // decoded ring | packed ring | epilogue r and bias of a tile (1 KB) |
 // barriers (512 B) | alignment slack (1 KB); the 6-bit tables are static
-__host__ __device__ constexpr int smem_bytes(int ba, int bw) {
-    return D_STAGES * DEC_STAGE + p_stages(ba, bw) * pk_stage_bytes(ba, bw) + 1024 + 512 + 1024;
+__host__ __device__ constexpr int smem_bytes(int ba, int bw, bool f8) {
+    return D_STAGES * DEC_STAGE + p_stages(ba, bw, f8) * pk_stage_bytes(ba, bw, f8) + 1024 + 512 + 1024;
 }
 
 struct QgemmParams {
@@ -80,8 +87,10 @@ struct QgemmParams {
     const uint16_t* w_r;
     const uint16_t* bias;
     uint16_t* y;
-    uint32_t tab_a[4], tab_w[4];  // 4-bit path: magnitude hi bytes (2 words), lo bytes (2 words)
-    uint16_t c6a[64], c6w[64];    // 6-bit path tables
+    float out_scale;              // extra output scale (1/d in the fp8 variant, whose centroids are scaled by sqrt(d))
+    uint32_t tab_a[4], tab_w[4];  // byte-permute tables of the register decoders
+    uint16_t c6a[64], c6w[64];    // 6-bit tables (bf16)
+    uint8_t c6a8[64], c6w8[64];   // 6-bit tables (e4m3)
 };
 
 // ----------------------------------------------------------------------------
@@ -151,13 +160,21 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
         : "memory");
 }
 
+template <bool F8>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
+    if constexpr (F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+            : "memory");
 }
 
 // named barrier 1 over the four epilogue warps
@@ -172,9 +189,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
            ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
-// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major,
-// M = 256 (the CTA pair), N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+// Instruction descriptors, both operands K-major, D = f32, M = 256 (the CTA
+// pair), N = 256: kind::f16 with A = B = bf16 (type 1), or kind::f8f6f4
+// with A = B = e4m3 (type 0).  Each MMA takes 32 bytes of every row (K = 16
+// bf16 or K = 32 e4m3 values).
+constexpr uint32_t kIdescShape = ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | kIdescShape;
+constexpr uint32_t kIdescE4m3 = (1u << 4) | kIdescShape;
 
 #define OQ_TMEM_LD16(taddr, v)                                                                                  \
     asm volatile(                                                                                               \
@@ -283,53 +304,108 @@ __device__ __forceinline__ uint4 decode8_6bit(uint32_t a, uint32_t b) {
     return make_uint4(e0 + e1 * 65536u, e2 + e3 * 65536u, e4 + e5 * 65536u, e6 + e7 * 65536u);
 }
 
-// Packed codes of one chunk (8 indices): 4-bit -> one word, 2-bit -> the low
-// half of a word, 6-bit (a byte each) -> two words.
-template <int BITS>
-struct Packed8 {
-    uint32_t a, b;
+// ---- e4m3 decoders (fp8 variant): 16 codes -> 16 bytes -------------------
+// The e4m3 centroid values are c_j sqrt(d) rounded once (sign-magnitude, so
+// the symmetric codebook's sign is bit 7 of the byte).
+
+// 4-bit: tab words 0-1 hold the magnitudes 0..7; one permute per 4 codes,
+// the sign from the same aligned permute of w and w << 4 as decode8_4bit.
+__device__ __forceinline__ uint2 decode8_4bit_e4m3(uint32_t w, const uint32_t tab[4]) {
+    const uint32_t s7 = __umulhi(w & 0x88888888u, 0xE0000000u);
+    const uint32_t mw = ~(w ^ s7) & 0x77777777u;
+    const uint32_t w4 = w << 4;
+    const uint32_t lo = prmt(tab[0], tab[1], mw) | (~prmt(w, w4, 0x1504u) & 0x80808080u);
+    const uint32_t hi = prmt(tab[0], tab[1], mw >> 16) | (~prmt(w, w4, 0x3726u) & 0x80808080u);
+    return make_uint2(lo, hi);
+}
+
+// 2-bit: tab word 0 holds the four signed values; each byte of codes is
+// spread to four nibbles, which select them.
+__device__ __forceinline__ uint4 decode16_2bit_e4m3(uint32_t x, const uint32_t tab[4]) {
+    const uint32_t v02 = x & 0x00FF00FFu, v13 = (x >> 8) & 0x00FF00FFu;  // bytes 0, 2 and 1, 3
+    uint32_t t02 = (v02 | (v02 << 4)) & 0x0F0F0F0Fu, t13 = (v13 | (v13 << 4)) & 0x0F0F0F0Fu;
+    t02 = (t02 | (t02 << 2)) & 0x33333333u;  // low half: codes 0-3, high half: codes 8-11
+    t13 = (t13 | (t13 << 2)) & 0x33333333u;  // codes 4-7, codes 12-15
+    return make_uint4(prmt(tab[0], 0u, t02), prmt(tab[0], 0u, t13), prmt(tab[0], 0u, t02 >> 16),
+                      prmt(tab[0], 0u, t13 >> 16));
+}
+
+// 6-bit: 64-byte e4m3 tables in static shared memory, one lookup per code.
+__shared__ __align__(128) uint8_t g_t6b[128];
+
+template <int TAB>
+__device__ __forceinline__ uint32_t decode4_6bit_e4m3(uint32_t a) {
+    a &= 0x3f3f3f3fu;
+    const uint8_t* t = g_t6b + 64 * TAB;
+    const uint32_t e0 = t[a & 0xffu], e1 = t[prmt(a, 0u, 0x4441u)], e2 = t[prmt(a, 0u, 0x4442u)], e3 = t[a >> 24];
+    return e0 + e1 * 0x100u + e2 * 0x10000u + e3 * 0x1000000u;
+}
+
+// Packed codes behind one 16-byte decoded chunk: unit_bytes(BITS, F8)
+// bytes, at most four words.
+template <int BITS, bool F8>
+struct PackedU {
+    static constexpr int NB = unit_bytes(BITS, F8);
+    uint32_t w[NB >= 4 ? NB / 4 : 1];
 };
 
-template <int BITS>
-__device__ __forceinline__ Packed8<BITS> load_unit(const uint8_t* src) {
-    Packed8<BITS> u;
-    if constexpr (BITS == 4) {
-        u.a = *reinterpret_cast<const uint32_t*>(src);
-        u.b = 0;
-    } else if constexpr (BITS == 2) {
-        u.a = *reinterpret_cast<const uint16_t*>(src);
-        u.b = 0;
-    } else {
+template <int BITS, bool F8>
+__device__ __forceinline__ PackedU<BITS, F8> load_unit(const uint8_t* src) {
+    PackedU<BITS, F8> u;
+    constexpr int NB = PackedU<BITS, F8>::NB;
+    if constexpr (NB == 2) {
+        u.w[0] = *reinterpret_cast<const uint16_t*>(src);
+    } else if constexpr (NB == 4) {
+        u.w[0] = *reinterpret_cast<const uint32_t*>(src);
+    } else if constexpr (NB == 8) {
         const uint2 t = *reinterpret_cast<const uint2*>(src);
-        u.a = t.x;
-        u.b = t.y;
+        u.w[0] = t.x;
+        u.w[1] = t.y;
+    } else {
+        const uint4 t = *reinterpret_cast<const uint4*>(src);
+        u.w[0] = t.x;
+        u.w[1] = t.y;
+        u.w[2] = t.z;
+        u.w[3] = t.w;
     }
     return u;
 }
 
-template <int BITS, int TAB>
-__device__ __forceinline__ uint4 decode_unit(Packed8<BITS> u, const uint32_t tab[4]) {
-    if constexpr (BITS == 4) return decode8_4bit(u.a, tab);
-    else if constexpr (BITS == 2) return decode8_2bit(u.a, tab);
-    else return decode8_6bit<TAB>(u.a, u.b);
+template <int BITS, int TAB, bool F8>
+__device__ __forceinline__ uint4 decode_unit(const PackedU<BITS, F8>& u, const uint32_t tab[4]) {
+    if constexpr (!F8) {
+        if constexpr (BITS == 4) return decode8_4bit(u.w[0], tab);
+        else if constexpr (BITS == 2) return decode8_2bit(u.w[0], tab);
+        else return decode8_6bit<TAB>(u.w[0], u.w[1]);
+    } else {
+        if constexpr (BITS == 4) {
+            const uint2 lo = decode8_4bit_e4m3(u.w[0], tab), hi = decode8_4bit_e4m3(u.w[1], tab);
+            return make_uint4(lo.x, lo.y, hi.x, hi.y);
+        } else if constexpr (BITS == 2) {
+            return decode16_2bit_e4m3(u.w[0], tab);
+        } else {
+            return make_uint4(decode4_6bit_e4m3<TAB>(u.w[0]), decode4_6bit_e4m3<TAB>(u.w[1]),
+                              decode4_6bit_e4m3<TAB>(u.w[2]), decode4_6bit_e4m3<TAB>(u.w[3]));
+        }
+    }
 }
 
 // One decoder thread's codes of a K step: units (row = t/8 + DEC_ROWS i,
-// chunk = t % 8) of this CTA's 128 x 64 shares of A and W.
-template <int BA, int BW>
+// chunk = t % 8) of this CTA's 128-row shares of A and W.
+template <int BA, int BW, bool F8>
 struct StageCodes {
-    Packed8<BA> a[DEC_UNITS];
-    Packed8<BW> b[DEC_UNITS];
+    PackedU<BA, F8> a[DEC_UNITS];
+    PackedU<BW, F8> b[DEC_UNITS];
 };
 
-template <int BA, int BW>
-__device__ __forceinline__ void load_codes(StageCodes<BA, BW>& u, const uint8_t* pa, const uint8_t* pb, int srcA,
+template <int BA, int BW, bool F8>
+__device__ __forceinline__ void load_codes(StageCodes<BA, BW, F8>& u, const uint8_t* pa, const uint8_t* pb, int srcA,
                                            int srcB) {
-    constexpr int PKRA = pk_row_bytes(BA), PKRB = pk_row_bytes(BW);
+    constexpr int PKRA = pk_row_bytes(BA, F8), PKRB = pk_row_bytes(BW, F8);
 #pragma unroll
-    for (int i = 0; i < DEC_UNITS; ++i) u.a[i] = load_unit<BA>(pa + srcA + i * DEC_ROWS * PKRA);
+    for (int i = 0; i < DEC_UNITS; ++i) u.a[i] = load_unit<BA, F8>(pa + srcA + i * DEC_ROWS * PKRA);
 #pragma unroll
-    for (int i = 0; i < DEC_UNITS; ++i) u.b[i] = load_unit<BW>(pb + srcB + i * DEC_ROWS * PKRB);
+    for (int i = 0; i < DEC_UNITS; ++i) u.b[i] = load_unit<BW, F8>(pb + srcB + i * DEC_ROWS * PKRB);
 }
 
 // Expanded values of one K step, written at the 128-byte-swizzled K-major
@@ -338,13 +414,13 @@ struct StageValues {
     uint4 a[DEC_UNITS], b[DEC_UNITS];
 };
 
-template <int BA, int BW>
-__device__ __forceinline__ void decode_codes(StageValues& v, const StageCodes<BA, BW>& u, const uint32_t tab_a[4],
+template <int BA, int BW, bool F8>
+__device__ __forceinline__ void decode_codes(StageValues& v, const StageCodes<BA, BW, F8>& u, const uint32_t tab_a[4],
                                              const uint32_t tab_w[4]) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
-        v.a[i] = decode_unit<BA, 0>(u.a[i], tab_a);
-        v.b[i] = decode_unit<BW, 1>(u.b[i], tab_w);
+        v.a[i] = decode_unit<BA, 0, F8>(u.a[i], tab_a);
+        v.b[i] = decode_unit<BW, 1, F8>(u.b[i], tab_w);
     }
 }
 
@@ -372,15 +448,15 @@ struct RingPos {
 };
 
 // ----------------------------------------------------------------------------
-template <int BA, int BW>
+template <int BA, int BW, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     qgemm_kernel(const __grid_constant__ QgemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     // the same offset in both CTAs (dynamic shared memory starts at the same address)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int PKA = HM * pk_row_bytes(BA);
-    constexpr int PK_STAGE = pk_stage_bytes(BA, BW);
-    constexpr int P_STAGES = p_stages(BA, BW);
+    constexpr int PKA = HM * pk_row_bytes(BA, F8);
+    constexpr int PK_STAGE = pk_stage_bytes(BA, BW, F8);
+    constexpr int P_STAGES = p_stages(BA, BW, F8);
     uint8_t* dec = smem;
     uint8_t* pk = smem + D_STAGES * DEC_STAGE;
     uint16_t* epi_r = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);  // r_n of the tile's 256 columns
@@ -419,8 +495,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (tid < 64) g_t6[tid] = p.c6a[tid];
-    else if (tid < 128) g_t6[tid] = p.c6w[tid - 64];
+    if constexpr (F8) {
+        if (tid < 64) g_t6b[tid] = p.c6a8[tid];
+        else if (tid < 128) g_t6b[tid] = p.c6w8[tid - 64];
+    } else {
+        if (tid < 64) g_t6[tid] = p.c6a[tid];
+        else if (tid < 128) g_t6[tid] = p.c6w[tid - 64];
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(512u));
@@ -447,8 +528,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     }
                     mbar_arrive_expect_tx(&pk_full[ps.idx], PK_STAGE);
                     uint8_t* dst = pk + ps.idx * PK_STAGE;
-                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA), m0, &pk_full[ps.idx]);
-                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW), n0, &pk_full[ps.idx]);
+                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA, F8), m0, &pk_full[ps.idx]);
+                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW, F8), n0, &pk_full[ps.idx]);
                     ++issued;
                     ps.advance();
                 }
@@ -478,8 +559,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(dec + ds.idx * DEC_STAGE), b_base = a_base + DEC_A;
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_pair(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k), kIdesc,
+                    for (int k = 0; k < 4; ++k)  // 32 bytes of each 128-byte row per MMA
+                        tc_mma_pair<F8>(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k),
+                                        F8 ? kIdescE4m3 : kIdescBf16,
                                     (kb | k) != 0 ? 1u : 0u);
                     tc_commit_pair(&dec_empty[ds.idx]);
                     ds.advance();
@@ -500,8 +582,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const bool grp_lead = warp == 2 + grp * GROUP_WARPS;
         const int row = t >> 3, c = t & 7;
         const int dst_off = (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4);
-        const int srcA = row * pk_row_bytes(BA) + c * (BA == 6 ? 8 : BA);
-        const int srcB = row * pk_row_bytes(BW) + c * (BW == 6 ? 8 : BW);
+        const int srcA = row * pk_row_bytes(BA, F8) + c * unit_bytes(BA, F8);
+        const int srcB = row * pk_row_bytes(BW, F8) + c * unit_bytes(BW, F8);
         const uint32_t tab_a[4] = {p.tab_a[0], p.tab_a[1], p.tab_a[2], p.tab_a[3]};
         const uint32_t tab_w[4] = {p.tab_w[0], p.tab_w[1], p.tab_w[2], p.tab_w[3]};
         const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
@@ -530,15 +612,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // A packed slot is released as soon as its codes are in registers
         // (the arrive's release orders the loads before it), so each slot is
         // held for about one step of the group.
-        StageCodes<BA, BW> cur;
+        StageCodes<BA, BW, F8> cur;
         bool ok = grp < total && wait_or_abort<false>(&pk_full[ps.idx], 0u, abort_flag);
         if (ok) {
-            load_codes<BA, BW>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+            load_codes<BA, BW, F8>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
             __syncwarp();
             if (lane == 0) mbar_arrive(&pk_empty[ps.idx]);
         }
         for (int s = grp; ok && s < total; s += NGROUPS) {
-            StageCodes<BA, BW> nxt;
+            StageCodes<BA, BW, F8> nxt;
             ps.advance(NGROUPS);
             const bool more = s + NGROUPS < total;
             if (more) {
@@ -547,10 +629,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 const uint8_t* pa = pk + ps.idx * PK_STAGE;
-                load_codes<BA, BW>(nxt, pa, pa + PKA, srcA, srcB);
+                load_codes<BA, BW, F8>(nxt, pa, pa + PKA, srcA, srcB);
             }
             StageValues v;
-            decode_codes<BA, BW>(v, cur, tab_a, tab_w);
+            decode_codes<BA, BW, F8>(v, cur, tab_a, tab_w);
             __syncwarp();
             if (lane == 0 && more) mbar_arrive(&pk_empty[ps.idx]);  // the next step's codes are in registers
             if (pending >= 0) publish(pending);
@@ -590,7 +672,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             epilogue_sync();
             const int row = m0 + q * 32 + lane;
             const bool row_ok = row < p.M;
-            const float sm = row_ok ? p.s[row] : 0.f;
+            const float sm = row_ok ? p.s[row] * p.out_scale : 0.f;
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * TN);
             uint16_t* yrow = p.y + (size_t)(row_ok ? row : 0) * p.N;
 #pragma unroll 1
@@ -703,14 +785,46 @@ void fill_tables(int bits, const uint16_t* cb, uint32_t tab[4], uint16_t* c6) {
     }
 }
 
-template <int BA, int BW>
+// e4m3 tables (fp8 variant) from the codebook's e4m3 bytes e[j] (c_j sqrt(d)
+// rounded once): 4-bit: magnitudes of c_8..c_15 in words 0-1; 2-bit: the
+// four signed values in word 0; 6-bit: the 64-byte shared-memory table.
+void fill_tables_e4m3(int bits, const uint8_t* e, uint32_t tab[4], uint8_t* c6) {
+    tab[0] = tab[1] = tab[2] = tab[3] = 0;
+    std::memset(c6, 0, 64);
+    if (bits == 4) {
+        for (int m = 0; m < 8; ++m) tab[m / 4] |= (uint32_t)e[8 + m] << (8 * (m % 4));
+    } else if (bits == 2) {
+        for (int j = 0; j < 4; ++j) tab[0] |= (uint32_t)e[j] << (8 * j);
+    } else {
+        for (int j = 0; j < 64; ++j) c6[j] = e[j];
+    }
+}
+
+template <int BA, int BW, bool F8>
 cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
-    auto k = qgemm_kernel<BA, BW>;
-    const int smem = smem_bytes(BA, BW);
+    auto k = qgemm_kernel<BA, BW, F8>;
+    const int smem = smem_bytes(BA, BW, F8);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k<<<grid, NTHREADS, smem, stream>>>(prm);
     return cudaGetLastError();
+}
+
+template <bool F8>
+cudaError_t launch_bits(const QgemmArgs& a, QgemmParams& prm, int grid, cudaStream_t stream) {
+#define OQ_CASE(X, Y) \
+    if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y, F8>(prm, grid, stream);
+    OQ_CASE(4, 4)
+    OQ_CASE(4, 2)
+    OQ_CASE(6, 4)
+    OQ_CASE(2, 2)
+    OQ_CASE(2, 4)
+    OQ_CASE(4, 6)
+    OQ_CASE(6, 2)
+    OQ_CASE(2, 6)
+    OQ_CASE(6, 6)
+#undef OQ_CASE
+    return cudaErrorInvalidValue;
 }
 
 int qgemm_sm_count() {
@@ -727,35 +841,32 @@ int qgemm_sm_count() {
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     QgemmParams prm;
     std::memset(&prm, 0, sizeof(prm));
-    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a), HM) ||
-        !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w), HN))
+    const bool f8 = a.fp8;
+    if (a.K % bk_codes(f8) != 0) return cudaErrorInvalidValue;
+    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a, f8), HM) ||
+        !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w, f8), HN))
         return cudaErrorInvalidValue;
     prm.M = a.M;
     prm.N = a.N;
-    prm.KB = a.K / BK;
+    prm.KB = a.K / bk_codes(f8);
     prm.num_m = (a.M + TM - 1) / TM;
     prm.num_tiles = prm.num_m * ((a.N + TN - 1) / TN);
     prm.s = a.s;
     prm.w_r = a.w_r;
     prm.bias = a.bias;
     prm.y = a.y;
-    fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
-    fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
+    if (f8) {
+        prm.out_scale = (float)(1.0 / (double)a.K);  // both operands' centroids carry sqrt(d)
+        fill_tables_e4m3(a.bits_a, a.ca_e4m3, prm.tab_a, prm.c6a8);
+        fill_tables_e4m3(a.bits_w, a.cw_e4m3, prm.tab_w, prm.c6w8);
+    } else {
+        prm.out_scale = 1.0f;
+        fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
+        fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
+    }
     const int pairs_max = qgemm_sm_count() / 2;
     const int pairs = prm.num_tiles < pairs_max ? prm.num_tiles : pairs_max;
-#define OQ_CASE(X, Y) \
-    if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y>(prm, 2 * pairs, stream);
-    OQ_CASE(4, 4)
-    OQ_CASE(4, 2)
-    OQ_CASE(6, 4)
-    OQ_CASE(2, 2)
-    OQ_CASE(2, 4)
-    OQ_CASE(4, 6)
-    OQ_CASE(6, 2)
-    OQ_CASE(2, 6)
-    OQ_CASE(6, 6)
-#undef OQ_CASE
-    return cudaErrorInvalidValue;
+    return f8 ? launch_bits<true>(a, prm, 2 * pairs, stream) : launch_bits<false>(a, prm, 2 * pairs, stream);
 }
 
 }  // namespace oq

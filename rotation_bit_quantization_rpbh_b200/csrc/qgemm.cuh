@@ -17,6 +17,9 @@ struct QgemmArgs {
     uint16_t* y;             // [M, N] bf16
     const uint16_t* ca_bf16; // activation centroids (2^bits_a), bf16 bits
     const uint16_t* cw_bf16; // weight centroids (2^bits_w)
+    bool fp8;                // e4m3 variant: centroids c_j sqrt(d) as e4m3, K % 128 == 0
+    const uint8_t* ca_e4m3;  // activation centroids (fp8 variant)
+    const uint8_t* cw_e4m3;  // weight centroids (fp8 variant)
 };
 
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream);

@@ -72,6 +72,20 @@ def test_library_block_rht_plan_matches_oracle(d, h, seed):
     np.testing.assert_array_equal(s3, s4)
 
 
+@pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (4096, 2), (1536, 6), (12288, 4)])
+def test_fp8_centroid_bytes_are_e4m3_of_the_scaled_codebook(d, bits):
+    """oq_codebook_fp8: e4m3 (torch's round-to-nearest-even conversion) of
+    c_j sqrt(d) for the oracle's fp64 centroids."""
+    import math
+
+    import torch
+
+    cb = B.codebook(d, bits)
+    c = oracle.codebook(d, bits)[0]
+    want = torch.tensor(np.asarray(c) * math.sqrt(d), dtype=torch.float64).to(torch.float8_e4m3fn)
+    np.testing.assert_array_equal(cb.e4m3_bytes(), want.view(torch.uint8).numpy())
+
+
 def test_unknown_rotation_variant_is_rejected():
     import ctypes
 

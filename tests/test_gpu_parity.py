@@ -131,3 +131,86 @@ def test_block_rht_variant_matches_oracle(cuda_device, M, d, h, ba):
     rows = np.arange(M)
     check_rotation(plan, x, rows, h, perm, sign, cuda_device)
     check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb_a, ocb_a, "acts")
+
+
+def _e4m3_values(c, d):
+    """e4m3 centroid values of the fp8 variant, from the oracle's fp64 codebook:
+    c_j sqrt(d) rounded once to e4m3 (torch's conversion), scaled back."""
+    q = torch.tensor(np.asarray(c) * math.sqrt(d), dtype=torch.float64).to(torch.float8_e4m3fn)
+    return q.to(torch.float64).numpy() / math.sqrt(d)
+
+
+FP8_CASES = [
+    # M,   d,   N,  h, bw, ba, seed, bias
+    (300, 512, 520, 128, 4, 4, 41, False),
+    (129, 256, 200, 64, 2, 4, 42, True),
+    (77, 384, 264, 128, 4, 6, 43, False),
+    (260, 1024, 256, 32, 6, 2, 44, True),
+    (70, 256, 131, 64, 4, 4, 45, True),
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=[f"M{c[0]}_d{c[1]}_N{c[2]}_W{c[4]}A{c[5]}" for c in FP8_CASES])
+def test_fp8_variant_matches_oracle_on_e4m3_centroids(cuda_device, case):
+    """The fp8 GEMM variant against the oracle's fp64 product on the same
+    indices and norms and the e4m3 centroid values, checked in full."""
+    M, d, N, h, bw, ba, seed, bias = case
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, h, seed)
+    cb_a, cb_w = B.codebook(d, ba), B.codebook(d, bw)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    a_idx, s = B.quantize_acts(plan, cb_a, x.to(cuda_device))
+    bias_t = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16).to(cuda_device) if bias else None
+    y = B.qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=bias_t)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    ca = _e4m3_values(oracle.codebook(d, ba)[0], d)
+    cw = _e4m3_values(oracle.codebook(d, bw)[0], d)
+    ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
+    iw = B.unpack_indices(w_idx, d, bw).cpu().numpy()
+    ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
+                         w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw)
+    if bias:
+        ref = ref + bias_t.cpu().to(torch.float32).numpy().astype(np.float64)[None, :]
+    got = y.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert rel_frob(got, ref) <= GEMM_TOL
+
+
+def test_fp8_variant_needs_d_multiple_of_128(cuda_device):
+    d = 64
+    cb = B.codebook(d, 4)
+    a_idx = torch.zeros((8, d // 2), dtype=torch.uint8, device=cuda_device)
+    s = torch.ones(8, device=cuda_device)
+    w_idx = torch.zeros((16, d // 2), dtype=torch.uint8, device=cuda_device)
+    w_r = torch.ones(16, dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(B.OQError) as e:
+        B.qgemm_fp8(cb, cb, a_idx, s, w_idx, w_r)
+    assert e.value.status == 2  # OQ_ERR_UNSUPPORTED
+
+
+def test_fp8_variant_full_size_flux_qkv_sample(cuda_device):
+    """FLUX-QKV shape in the launch configuration the bench times, checked on
+    sampled rows and columns."""
+    w = I.WORKLOADS["flux_qkv_w4a4"]
+    x = I.make_x(w)
+    W = I.make_w(w)
+    plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
+    cb_a, cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    a_idx, s = B.quantize_acts(plan, cb_a, x.to(cuda_device))
+    y = B.qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(w.M, 128, replace=False))
+    cols = np.sort(rng.choice(w.N, 256, replace=False))
+    ca = _e4m3_values(oracle.codebook(w.d, w.bits_a)[0], w.d)
+    cw = _e4m3_values(oracle.codebook(w.d, w.bits_w)[0], w.d)
+    ia = B.unpack_indices(a_idx, w.d, w.bits_a).cpu().numpy()
+    iw = B.unpack_indices(w_idx, w.d, w.bits_w).cpu().numpy()
+    ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
+                         w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw, rows, cols)
+    got = y.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)]
+    assert rel_frob(got, ref) <= GEMM_TOL
