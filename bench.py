@@ -56,7 +56,7 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-KERNEL_SOURCES = {"qgemm": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu"}
+KERNEL_SOURCES = {"qgemm": "qgemm.cu", "qgemm_fp8": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu"}
 
 
 def committed_traffic(kernel, workload):
@@ -411,7 +411,7 @@ def run_ours(args):
                       "rpbh_quant_gbs": rpbh_gbs},
         "roofline": {"bound": "tensor", "kernel": "qgemm_fp8" if args.fp8 else "qgemm", "achieved": gemm_tflops,
                      "peak": mma_peak, "unit": "TFLOP/s", "frac": gemm_tflops / mma_peak,
-                     "traffic": None if args.fp8 else committed_traffic("qgemm", w.name), "peak_source": peak_note,
+                     "traffic": committed_traffic("qgemm_fp8" if args.fp8 else "qgemm", w.name), "peak_source": peak_note,
                      "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
         "roofline_rpbh": {"bound": "hbm", "kernel": "rpbh_quant", "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
                           "unit": "GB/s", "frac": rpbh_gbs / peaks["hbm_gbs"],
