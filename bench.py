@@ -71,10 +71,22 @@ def committed_traffic(kernel, workload):
     with open(p) as f:
         j = json.load(f).get(kernel, {})
     src = os.path.join(ROOT, "rotation_bit_quantization_rpbh_b200", "csrc", KERNEL_SOURCES[kernel])
-    with open(src, "rb") as f:
-        if hashlib.md5(f.read()).hexdigest() != j.get("source_md5"):
+    with open(src, encoding="utf-8") as f:
+        if hashlib.md5(code_only(f.read()).encode()).hexdigest() != j.get("code_md5"):
             return None
     return j.get(workload)
+
+
+def code_only(src):
+    """C++ source with comments, #include lines and blank lines removed and
+    whitespace runs collapsed: its digest changes with the code, not with
+    its comments."""
+    import re
+
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    lines = [" ".join(ln.split()) for ln in src.splitlines()]
+    return "\n".join(ln for ln in lines if ln and not ln.startswith("#include"))
 
 
 class ClockSampler:

@@ -4,32 +4,39 @@
 // 方法 (Method): W^' = diag(r') Q_bw(W~'), x^' = s Q_ba(x~'), and the layer
 // computes W^' x^' ~ W x with no inverse rotation.  Per output element
 //   y[m, n] = r_n * s_m * sum_k C_w[iw[n, k]] * C_a[ia[m, k]]
-// with the centroids taken as bf16 values, fp32 accumulation, bf16 output.
+// with the centroids taken as bf16 values (the fp8 variant: e4m3 values of
+// C sqrt(d), and an extra 1/d in the epilogue), fp32 accumulation, bf16
+// output.
 //
 // Structure: clusters of two CTAs on an SM pair share one 256 x 256 output
-// tile through tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16 per
-// instruction).  CTA r of the pair owns A rows [128r, 128r + 128) and W rows
+// tile through tcgen05.mma.cta_group::2 (M = 256, N = 256; each instruction
+// takes 32 bytes of every K-major row: K = 16 bf16 or K = 32 e4m3 values).
+// A K step fills one 128-byte row per operand (64 bf16 or 128 e4m3 values).
+// CTA r of the pair owns A rows [128r, 128r + 128) and W rows
 // [128r, 128r + 128) of the tile, so each SM expands 256 rows of codes per
 // K step for a 128 x 256 share of the output (a 1-SM 128 x 256 tile would
 // expand 384).  Per CTA:
 //   warp 0      TMA producer: 2-D tensor loads of this CTA's packed index
-//               tiles into a ring (no multicast: each CTA reads its own rows);
+//               tiles into a ring of up to 10 stages (no multicast: each CTA
+//               reads its own rows);
 //   warp 1      TMEM: 512 columns = two 128 x 256 fp32 accumulators; in the
 //               leader CTA one thread issues the pair's MMAs;
 //   warps 2-17  decoders, two groups taking alternate K steps: expand
-//               packed codes to bf16 centroid values
-//               (register byte-permute lookups, 64-entry static shared
-//               table for 6-bit codes) in the 128-byte-swizzled K-major layout, then
-//               signal the leader's "stage full" barrier: the leader's own
-//               warps arrive, the peer's warps complete transaction bytes on
-//               it with st.async (asynchronous, cluster-scope release), so no
-//               decoder thread waits on a cluster-wide release.  Each
-//               group's loop is software-pipelined one step deep on both
-//               sides (codes read a step ahead, stages published a step
-//               behind);
-//   warps 18-21 epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
-//               scale by s_m r_n (+ bias) in fp32, round to bf16, store, and
-//               release the accumulator to the leader.
+//               packed codes to centroid values (register byte-permute
+//               lookups; 64-entry static shared tables for 6-bit codes)
+//               into a 4-stage ring in the 128-byte-swizzled K-major
+//               layout, then signal the leader's "stage full" barrier: the
+//               leader's own warps arrive, the peer's warps complete
+//               transaction bytes on it with st.async (asynchronous,
+//               cluster-scope release), so no decoder thread waits on a
+//               cluster-wide release.  Each group's loop is
+//               software-pipelined one step deep on both sides (codes read
+//               a step ahead, stages published a step behind), and a packed
+//               stage is released as soon as its codes are in registers;
+//   warps 18-21 epilogue: stage the tile's r (and bias) in shared memory,
+//               tcgen05.ld this CTA's 128 accumulator rows 32 columns at a
+//               time, scale by s_m r_n (+ bias) in fp32, round to bf16,
+//               store, and release the accumulator to the leader.
 // The leader's MMA completions are multicast (tcgen05.commit) to the
 // barriers of both CTAs.  Every mbarrier wait is bounded: on a timeout the
 // kernel raises the device error flag, drains its own TMA loads, leaves the

@@ -11,10 +11,9 @@
 //   - persistent CTAs, one per SM, each split into NG (1-3) warp groups that
 //     take interleaved tiles of R rows and run out of phase (own staging buffers,
 //     mbarriers and named barriers), so one group's gathers overlap the
-//     other's butterflies and table lookups; a group stages its rows with
+//     others' butterflies and table lookups; a group stages its rows with
 //     1-D bulk copies (cp.async.bulk), double buffered so its next tile
-//     streams in while this one is computed (the first copies are issued
-//     before the table set-up);
+//     streams in while this one is computed;
 //   - the gather and lookup tables arrive by bulk copy together with each
 //     group's first rows;
 //   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
@@ -27,8 +26,10 @@
 //     magic constant) indexes a small table holding, per bin, the count of
 //     thresholds below it and the one threshold inside it, so
 //     index = base + (v >= T) -- exactly #{ j : t_j <= v } in fp32;
-//   - indices are packed LSB-first and written with 16-byte stores.
-#include <cfloat>
+//   - rows whose norm is not finite or exceeds FLT_MAX / (2 sqrt(h)) (where
+//     the fp32 butterfly could overflow) take the middle cell;
+//   - indices are packed LSB-first and written 16 bytes at a time as they
+//     are produced.
 #include <cuda_bf16.h>
 
 #include "device_util.cuh"
