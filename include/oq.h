@@ -32,7 +32,10 @@
  *   - Layouts are row-major.  Packed indices are K-major rows, LSB-first:
  *     bits = 4: two indices per byte (index k in bits 4*(k%2) of byte k/2);
  *     bits = 2: four per byte (bits 2*(k%4) of byte k/4);
- *     bits = 6: one index per byte (low 6 bits).
+ *     bits = 6: one index per byte (low 6 bits);
+ *     bits = 3: a bit stream, index k in bits 3k..3k+2 of the row (eight
+ *               indices per three bytes); needs h >= 32 and d % 128 == 0,
+ *               and runs through the fp8 product variant only.
  *     Index j means centroid c_j of C_d sorted ascending (0 = most negative).
  *   - eps = 1e-12 on both the weight and the activation side.
  */

@@ -315,10 +315,17 @@ def device_status(clear=True, stream=None):
 
 def unpack_indices(packed, d, bits):
     """Unpack LSB-first packed indices [rows, bytes] to one index per byte
-    [rows, d] (a layout conversion for tests and callers, on any device)."""
+    [rows, d] (a layout conversion for tests and callers, on any device).
+    3-bit codes are a bit stream, 8 codes per 3 bytes."""
     p = packed.to(torch.int32)
     if bits == 6:
         return (p & 63).to(torch.uint8)
+    if bits == 3:
+        rows = p.shape[0]
+        b = p.reshape(rows, -1, 3)
+        g = b[..., 0] | (b[..., 1] << 8) | (b[..., 2] << 16)  # 24 bits = 8 codes
+        shifts = torch.arange(8, device=p.device, dtype=torch.int32) * 3
+        return ((g.unsqueeze(-1) >> shifts) & 7).reshape(rows, -1)[:, :d].to(torch.uint8)
     per = 8 // bits
     shifts = torch.arange(per, device=p.device, dtype=torch.int32) * bits
     v = (p.unsqueeze(-1) >> shifts) & ((1 << bits) - 1)

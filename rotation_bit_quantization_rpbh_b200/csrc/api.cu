@@ -29,7 +29,7 @@ int device_sms() {
     return count[dev] > 0 ? count[dev] : 148;
 }
 
-bool quant_bits_ok(int bits) { return bits == 2 || bits == 4 || bits == 6; }
+bool quant_bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 6; }
 
 int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }
 
@@ -47,6 +47,7 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
         if (cb->d != plan->d) return OQ_ERR_INVALID_ARG;
         if (!quant_bits_ok(cb->bits)) return OQ_ERR_UNSUPPORTED;
         if (packed_row_bytes(plan->d, cb->bits) % 4 != 0) return OQ_ERR_UNSUPPORTED;
+        if (cb->bits == 3 && (plan->h < 32 || plan->d % 128 != 0)) return OQ_ERR_UNSUPPORTED;  // 16-byte rows
         if (!aligned16(idx_out)) return OQ_ERR_ALIGNMENT;
     }
     if (mode == 0 && (!s_out || !aligned16(s_out))) return s_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
@@ -294,6 +295,10 @@ static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
     if (!cb_a || !cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != cb_w->d) return OQ_ERR_INVALID_ARG;
     if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % (fp8 ? 128 : 64) != 0)
+        return OQ_ERR_UNSUPPORTED;
+    // 3-bit rows hold 24 bytes per 64 codes, too narrow for the bf16 kernel's TMA step
+    if (!fp8 && (cb_a->bits == 3 || cb_w->bits == 3)) return OQ_ERR_UNSUPPORTED;
+    if (fp8 && (cb_a->bits == 3 || cb_w->bits == 3) && !((cb_a->bits == 3 || cb_a->bits == 4) && (cb_w->bits == 3 || cb_w->bits == 4)))
         return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;  // an empty batch: activation and output buffers may be null
     if (!a_idx || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;

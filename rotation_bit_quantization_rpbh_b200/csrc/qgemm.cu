@@ -22,8 +22,9 @@
 //   warp 1      TMEM: 512 columns = two 128 x 256 fp32 accumulators; in the
 //               leader CTA one thread issues the pair's MMAs;
 //   warps 2-17  decoders, two groups taking alternate K steps: expand
-//               packed codes to centroid values (register byte-permute
-//               lookups; 64-entry static shared tables for 6-bit codes)
+//               packed 2/3/4/6-bit codes to centroid values (register
+//               byte-permute lookups; 64-entry static shared tables for 6-bit
+//               codes; 3-bit codes in the fp8 variant only)
 //               into a 4-stage ring in the 128-byte-swizzled K-major
 //               layout, then signal the leader's "stage full" barrier: the
 //               leader's own warps arrive, the peer's warps complete
@@ -337,6 +338,23 @@ __device__ __forceinline__ uint4 decode16_2bit_e4m3(uint32_t x, const uint32_t t
                       prmt(tab[0], 0u, t13 >> 16));
 }
 
+// 3-bit (codes LSB-first, 8 per 3 bytes): the 24 bits of 8 codes are spread
+// to 8 nibbles in three shift-and-mask steps (halves, pairs, singles), which
+// select from the 8 signed e4m3 values in tab words 0-1.
+__device__ __forceinline__ uint32_t spread3to4(uint32_t x) {
+    uint32_t y = (x & 0xFFFu) | ((x << 4) & 0x0FFF0000u);  // codes 0-3 at bits 0.., 4-7 at 16..
+    y = (y & 0x003F003Fu) | ((y << 2) & 0x3F003F00u);      // pairs at bytes
+    y = (y & 0x07070707u) | ((y << 1) & 0x70707070u);      // one code per nibble
+    return y;
+}
+
+__device__ __forceinline__ uint4 decode16_3bit_e4m3(uint32_t lo, uint32_t hi, const uint32_t tab[4]) {
+    const uint32_t y0 = spread3to4(lo & 0xFFFFFFu);               // codes 0-7
+    const uint32_t y1 = spread3to4((lo >> 24) | (hi << 8));      // codes 8-15
+    return make_uint4(prmt(tab[0], tab[1], y0), prmt(tab[0], tab[1], y0 >> 16), prmt(tab[0], tab[1], y1),
+                      prmt(tab[0], tab[1], y1 >> 16));
+}
+
 // 6-bit: 64-byte e4m3 tables in static shared memory, one lookup per code.
 __shared__ __align__(128) uint8_t g_t6b[128];
 
@@ -353,7 +371,7 @@ __device__ __forceinline__ uint32_t decode4_6bit_e4m3(uint32_t a) {
 template <int BITS, bool F8>
 struct PackedU {
     static constexpr int NB = unit_bytes(BITS, F8);
-    uint32_t w[NB >= 4 ? NB / 4 : 1];
+    uint32_t w[NB >= 4 ? (NB + 3) / 4 : 1];
 };
 
 template <int BITS, bool F8>
@@ -362,6 +380,10 @@ __device__ __forceinline__ PackedU<BITS, F8> load_unit(const uint8_t* src) {
     constexpr int NB = PackedU<BITS, F8>::NB;
     if constexpr (NB == 2) {
         u.w[0] = *reinterpret_cast<const uint16_t*>(src);
+    } else if constexpr (NB == 6) {  // 16 3-bit codes at a 2-byte-aligned offset
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
+        u.w[0] = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+        u.w[1] = h[2];
     } else if constexpr (NB == 4) {
         u.w[0] = *reinterpret_cast<const uint32_t*>(src);
     } else if constexpr (NB == 8) {
@@ -380,6 +402,7 @@ __device__ __forceinline__ PackedU<BITS, F8> load_unit(const uint8_t* src) {
 
 template <int BITS, int TAB, bool F8>
 __device__ __forceinline__ uint4 decode_unit(const PackedU<BITS, F8>& u, const uint32_t tab[4]) {
+    static_assert(BITS != 3 || F8, "3-bit codes run in the fp8 variant only");
     if constexpr (!F8) {
         if constexpr (BITS == 4) return decode8_4bit(u.w[0], tab);
         else if constexpr (BITS == 2) return decode8_2bit(u.w[0], tab);
@@ -390,6 +413,8 @@ __device__ __forceinline__ uint4 decode_unit(const PackedU<BITS, F8>& u, const u
             return make_uint4(lo.x, lo.y, hi.x, hi.y);
         } else if constexpr (BITS == 2) {
             return decode16_2bit_e4m3(u.w[0], tab);
+        } else if constexpr (BITS == 3) {
+            return decode16_3bit_e4m3(u.w[0], u.w[1], tab);
         } else {
             return make_uint4(decode4_6bit_e4m3<TAB>(u.w[0]), decode4_6bit_e4m3<TAB>(u.w[1]),
                               decode4_6bit_e4m3<TAB>(u.w[2]), decode4_6bit_e4m3<TAB>(u.w[3]));
@@ -802,6 +827,8 @@ void fill_tables_e4m3(int bits, const uint8_t* e, uint32_t tab[4], uint8_t* c6) 
         for (int m = 0; m < 8; ++m) tab[m / 4] |= (uint32_t)e[8 + m] << (8 * (m % 4));
     } else if (bits == 2) {
         for (int j = 0; j < 4; ++j) tab[0] |= (uint32_t)e[j] << (8 * j);
+    } else if (bits == 3) {
+        for (int j = 0; j < 8; ++j) tab[j / 4] |= (uint32_t)e[j] << (8 * (j % 4));
     } else {
         for (int j = 0; j < 64; ++j) c6[j] = e[j];
     }
@@ -819,6 +846,11 @@ cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
 
 template <bool F8>
 cudaError_t launch_bits(const QgemmArgs& a, QgemmParams& prm, int grid, cudaStream_t stream) {
+    if constexpr (F8) {  // 3-bit codes: the fp8 variant only
+        if (a.bits_a == 3 && a.bits_w == 3) return launch_qgemm_t<3, 3, true>(prm, grid, stream);
+        if (a.bits_a == 3 && a.bits_w == 4) return launch_qgemm_t<3, 4, true>(prm, grid, stream);
+        if (a.bits_a == 4 && a.bits_w == 3) return launch_qgemm_t<4, 3, true>(prm, grid, stream);
+    }
 #define OQ_CASE(X, Y) \
     if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y, F8>(prm, grid, stream);
     OQ_CASE(4, 4)

@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
                 constexpr int NB = BITS == 6 ? H : H * BITS / 8;  // packed bytes per h-block
                 constexpr int NW = NB / 4;
                 constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
-                constexpr int PER = BITS == 6 ? 4 : 32 / BITS;     // codes per 32-bit word
+                constexpr int PER = BITS == 6 ? 4 : (BITS == 3 ? 8 : 32 / BITS);  // codes per word (3-bit: per 24-bit group)
                 constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
                 uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
                 auto put = [&](int w0, const uint32_t (&words)[CW]) {
@@ -248,7 +248,46 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
                 // s <= s_max keeps every butterfly value below sqrt(h) s (finite),
                 // so |v| <= 1 up to rounding and the table index stays in range;
                 // larger, infinite and NaN norms take the middle cell
-                if (s <= p.s_max) {
+                if (BITS == 3 && s <= p.s_max) {
+                    // 3-bit: codes 8g..8g+7 form a 24-bit group (LSB first); four
+                    // groups fill three words
+                    const float inv = p.rsqrt_h / (s + p.eps);
+                    const float2 inv2 = make_float2(inv, inv);
+                    uint32_t words[NW];
+#pragma unroll
+                    for (int g4 = 0; g4 < H / 32; ++g4) {
+                        uint32_t grp[4];
+#pragma unroll
+                        for (int gi = 0; gi < 4; ++gi) {
+                            uint32_t acc_w = 0;
+#pragma unroll
+                            for (int k = 6; k >= 0; k -= 2) {
+                                const float2 q = f2mul(v2[(32 * g4 + 8 * gi + k) >> 1], inv2);
+                                const float2 z = f2fma(q, G2, M2);
+                                float T0, T1;
+                                int b0, b1;
+                                const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
+                                const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
+                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
+                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
+                                const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
+                                const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
+                                acc_w = (acc_w * 8u + i1) * 8u + i0;
+                            }
+                            grp[gi] = acc_w;
+                        }
+                        words[3 * g4] = grp[0] | (grp[1] << 24);
+                        words[3 * g4 + 1] = (grp[1] >> 8) | (grp[2] << 16);
+                        words[3 * g4 + 2] = (grp[2] >> 16) | (grp[3] << 8);
+                    }
+#pragma unroll
+                    for (int w0 = 0; w0 < NW; w0 += CW) {
+                        uint32_t ws[CW];
+#pragma unroll
+                        for (int wj = 0; wj < CW; ++wj) ws[wj] = words[w0 + wj];
+                        put(w0, ws);
+                    }
+                } else if (BITS != 3 && s <= p.s_max) {
                     // x'/(s+eps) = (H u / sqrt(h)) / (s + eps): one multiplier for the unnormalised butterflies
                     const float inv = p.rsqrt_h / (s + p.eps);
                     const float2 inv2 = make_float2(inv, inv);
@@ -277,6 +316,17 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
                             words[wj] = acc_w;
                         }
                         put(w0, words);
+                    }
+                } else if (BITS == 3) {
+                    // middle code 4 everywhere: the 3-bit stream repeats every 3 words
+                    constexpr uint32_t g = 04444'4444u;  // eight 3-bit fours (octal)
+                    const uint32_t pat[3] = {g | (g << 24), (g >> 8) | (g << 16), (g >> 16) | (g << 8)};
+#pragma unroll
+                    for (int w0 = 0; w0 < NW; w0 += CW) {
+                        uint32_t ws[CW];
+#pragma unroll
+                        for (int wj = 0; wj < CW; ++wj) ws[wj] = pat[(w0 + wj) % 3];
+                        put(w0, ws);
                     }
                 } else {
                     uint32_t wmid = 0;
@@ -308,6 +358,9 @@ template <typename InT, int H, int MODE>
 cudaError_t launch_bits(const RpbhParams& p, int bits, int grid, cudaStream_t stream) {
     switch (bits) {
         case 2: return launch_rpbh_t<InT, H, 2, MODE>(p, grid, stream);
+        case 3:
+            if constexpr (H >= 32) return launch_rpbh_t<InT, H, 3, MODE>(p, grid, stream);
+            return cudaErrorInvalidValue;
         case 4: return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
         case 6: return launch_rpbh_t<InT, H, 6, MODE>(p, grid, stream);
     }

@@ -36,7 +36,7 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (12288, 4), (4096, 2), (4096, 4), (1536, 4), (1536, 6),
-                                    (64, 2), (64, 4), (64, 6), (512, 2), (8, 2)])
+                                    (64, 2), (64, 4), (64, 6), (512, 2), (8, 2), (3072, 3), (128, 3)])
 def test_library_codebook_matches_oracle(d, bits):
     """Two independent solvers (library: Newton on the Lloyd-Max conditions
     with incomplete-beta cell masses; oracle: Lloyd iteration with
@@ -72,7 +72,7 @@ def test_library_block_rht_plan_matches_oracle(d, h, seed):
     np.testing.assert_array_equal(s3, s4)
 
 
-@pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (4096, 2), (1536, 6), (12288, 4)])
+@pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (4096, 2), (1536, 6), (12288, 4), (3072, 3)])
 def test_fp8_centroid_bytes_are_e4m3_of_the_scaled_codebook(d, bits):
     """oq_codebook_fp8: e4m3 (torch's round-to-nearest-even conversion) of
     c_j sqrt(d) for the oracle's fp64 centroids."""
@@ -120,7 +120,9 @@ def test_workspace_size():
     assert ws >= 4096 * 1536 + 4096 * 4 and ws % 256 == 0
     assert B.qlinear_workspace(32760, 1536, 6) >= 32760 * 1536 + 32760 * 4
     assert B.qlinear_workspace(0, 1536, 4) == 0
-    assert B.qlinear_workspace(10, 1536, 3) == 0
+    ws3 = B.qlinear_workspace(10, 1536, 3)  # 3-bit: 8 codes per 3 bytes
+    assert ws3 >= 10 * 1536 * 3 // 8 + 10 * 4 and ws3 % 256 == 0
+    assert B.qlinear_workspace(10, 1536, 5) == 0
 
 
 def test_unpack_layout():

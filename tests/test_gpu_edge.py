@@ -73,9 +73,9 @@ def test_mismatched_handles_are_rejected(layer, cuda_device):
     with pytest.raises(B.OQError) as e:
         B.quantize_acts(plan, other, x)
     assert e.value.status == 1
-    cb3 = B.codebook(d, 3)
+    cb5 = B.codebook(d, 5)  # a codebook width the quantiser does not pack
     with pytest.raises(B.OQError) as e:
-        B.quantize_acts(plan, cb3, x)
+        B.quantize_acts(plan, cb5, x)
     assert e.value.status == 2
 
 

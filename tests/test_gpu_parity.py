@@ -214,3 +214,62 @@ def test_fp8_variant_full_size_flux_qkv_sample(cuda_device):
                          w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw, rows, cols)
     got = y.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)]
     assert rel_frob(got, ref) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("M,d,h,seed", [(300, 512, 128, 51), (97, 384, 64, 52), (64, 256, 32, 53)])
+def test_three_bit_codes_match_oracle(cuda_device, M, d, h, seed):
+    """3-bit codes (8 per 3 bytes, LSB first) for activations and weights."""
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, h, seed)
+    perm, sign = oracle.plan(d, h, seed)
+    cb, ocb = B.codebook(d, 3), oracle.codebook(d, 3)
+    a_idx, s = B.quantize_acts(plan, cb, x.to(cuda_device))
+    w_idx, r = B.quantize_weights(plan, cb, x.to(cuda_device))
+    torch.cuda.synchronize()
+    assert a_idx.shape == (M, d * 3 // 8)
+    rows = np.arange(M)
+    check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb, ocb, "acts")
+    check_quantized_rows(w_idx, r, x, rows, h, perm, sign, cb, ocb, "weights")
+
+
+@pytest.mark.parametrize("bw,ba", [(3, 3), (4, 3), (3, 4)])
+def test_three_bit_fp8_product_matches_oracle(cuda_device, bw, ba):
+    """W3A3 (the pages' ablation setting) and the mixed 3/4-bit pairs through
+    the fp8 variant, against the oracle on the e4m3 centroid values."""
+    M, d, N, h, seed = 260, 768, 264, 128, 54 + bw + ba
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, h, seed)
+    cb_a, cb_w = B.codebook(d, ba), B.codebook(d, bw)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    xg = x.to(cuda_device)
+    a_idx, s = B.quantize_acts(plan, cb_a, xg)
+    y = B.qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r)
+    y2 = B.qlinear(plan, cb_a, cb_w, xg, w_idx, w_r, fp8=True)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert torch.equal(y, y2)
+    ca = _e4m3_values(oracle.codebook(d, ba)[0], d)
+    cw = _e4m3_values(oracle.codebook(d, bw)[0], d)
+    ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
+    iw = B.unpack_indices(w_idx, d, bw).cpu().numpy()
+    ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
+                         w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw)
+    assert rel_frob(y.float().cpu().numpy().astype(np.float64), ref) <= GEMM_TOL
+
+
+def test_three_bit_limits_are_reported(cuda_device):
+    d = 256
+    cb = B.codebook(d, 3)
+    x = torch.randn(8, d, device=cuda_device).to(torch.bfloat16)
+    with pytest.raises(B.OQError) as e:  # h = 16 would give 6-byte blocks
+        B.quantize_acts(B.rpbh_plan(d, 16, 1), cb, x)
+    assert e.value.status == 2
+    a_idx, s = B.quantize_acts(B.rpbh_plan(d, 64, 1), cb, x)
+    w_idx = torch.zeros((16, d * 3 // 8), dtype=torch.uint8, device=cuda_device)
+    w_r = torch.ones(16, dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(B.OQError) as e:  # the bf16 kernel's 64-code step is 24 bytes of 3-bit codes
+        B.qgemm(cb, cb, a_idx, s, w_idx, w_r)
+    assert e.value.status == 2
