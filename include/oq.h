@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     OQ_OK = 0,
     OQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, mismatched handles */
-    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,4,6}, d % 64 != 0 */
+    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,3,4,6}, d % 64 != 0 */
     OQ_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned */
     OQ_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
     OQ_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see oq_device_status) */
@@ -246,6 +246,25 @@ oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
 /* error flag that kernels set when a bounded wait runs out.  Synchronises */
 /* `stream`.  *out receives OQ_OK or OQ_ERR_TIMEOUT.                        */
 oq_status oq_device_status(int clear, int* out, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Test hooks: failures made on the host, so that error handling is tested */
+/* without faulting a GPU.  Not for production use.                        */
+/*                                                                          */
+/* oq_debug_fail_allocations(n): the next n device allocations the library */
+/*   makes for its own tables (a plan's gather table, a codebook's lookup   */
+/*   table on first use on a device) report failure, so the call returns    */
+/*   OQ_ERR_OOM and leaves no partial state; n <= 0 cancels.                */
+/* oq_debug_starve(mask): the next launch of each kernel named in `mask`    */
+/*   issues none of its input copies, so its bounded waits run out (about   */
+/*   one second), it records OQ_ERR_TIMEOUT for oq_device_status() and      */
+/*   returns without faulting; the context stays usable.  The output of     */
+/*   that launch is undefined.  The call itself still returns OQ_OK.        */
+/*   Each call replaces the pending set; mask 0 cancels.                    */
+#define OQ_STARVE_RPBH 1 /* the rotate-and-quantise kernel (acts and weights) */
+#define OQ_STARVE_GEMM 2 /* the codebook-decode GEMM (bf16 and fp8)           */
+void oq_debug_fail_allocations(int n);
+void oq_debug_starve(int mask);
 
 #ifdef __cplusplus
 }

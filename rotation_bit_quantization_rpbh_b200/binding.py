@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liboq.so")
 OQ_OK = 0
 OQ_BF16, OQ_F32 = 0, 1
 OQ_ROT_RPBH, OQ_ROT_BLOCK_RHT = 0, 1
+OQ_STARVE_RPBH, OQ_STARVE_GEMM = 1, 2
 _STATUS = {0: "OQ_OK", 1: "OQ_ERR_INVALID_ARG", 2: "OQ_ERR_UNSUPPORTED", 3: "OQ_ERR_ALIGNMENT", 4: "OQ_ERR_CUDA",
            5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE", 8: "OQ_ERR_TOO_LARGE"}
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -30,7 +31,8 @@ EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf
            "oq_rotation_plan_host", "oq_plan_shape", "oq_qgemm_fp8", "oq_codebook_fp8",
            "oq_qlinear_fp8",
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
-           "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status"]
+           "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status",
+           "oq_debug_fail_allocations", "oq_debug_starve"]
 
 
 class OQError(RuntimeError):
@@ -79,6 +81,8 @@ def lib():
                     "oq_qlinear": ([P, P, P, P, I, I, P, P, I, P, P, P, SZ, P], I),
                     "oq_qlinear_noalloc": ([P, P, P, P, I, I, P, P, I, P, P, P], I),
                     "oq_device_status": ([I, P, P], I),
+                    "oq_debug_fail_allocations": ([I], None),
+                    "oq_debug_starve": ([I], None),
                 }
                 for name, (args, res) in sig.items():
                     f = getattr(L, name)
@@ -311,6 +315,20 @@ def device_status(clear=True, stream=None):
     out = ctypes.c_int(0)
     _check(lib().oq_device_status(int(clear), ctypes.byref(out), _stream(stream)), "oq_device_status")
     return out.value
+
+
+def debug_fail_allocations(n):
+    """Test hook: the library's next ``n`` own device allocations fail
+    (the calls making them return OQ_ERR_OOM); ``n <= 0`` cancels."""
+    lib().oq_debug_fail_allocations(int(n))
+
+
+def debug_starve(mask):
+    """Test hook: the next launch of each kernel in ``mask``
+    (OQ_STARVE_RPBH | OQ_STARVE_GEMM) issues no input copies, so its bounded
+    waits run out and ``device_status()`` reports OQ_ERR_TIMEOUT.  Replaces
+    the pending set; 0 cancels."""
+    lib().oq_debug_starve(int(mask))
 
 
 def unpack_indices(packed, d, bits):

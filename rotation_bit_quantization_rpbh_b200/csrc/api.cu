@@ -2,6 +2,7 @@
 // management, lazy per-device uploads and kernel dispatch.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 #include <new>
 
@@ -28,6 +29,22 @@ int device_sms() {
     if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
     return count[dev] > 0 ? count[dev] : 148;
 }
+
+// Test hooks (failure detection without a GPU fault): pending allocation
+// failures and the kernels whose next launch issues no input copies.
+static std::atomic<int> g_fail_allocs{0};
+static std::atomic<int> g_starve_mask{0};
+
+static bool device_alloc(void** ptr, size_t bytes) {
+    int n = g_fail_allocs.load();
+    while (n > 0 && !g_fail_allocs.compare_exchange_weak(n, n - 1)) {
+    }
+    if (n > 0) return false;
+    return cudaMalloc(ptr, bytes) == cudaSuccess;
+}
+
+// true (once) if the next launch of `kernel` is to be starved
+bool take_starve(int kernel) { return (g_starve_mask.fetch_and(~kernel) & kernel) != 0; }
 
 bool quant_bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 6; }
 
@@ -100,6 +117,7 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.norm_out = norm_out;
     p.rsqrt_h = (float)(1.0 / std::sqrt((double)h));
     p.eps = (float)kEps;
+    p.starve = take_starve(OQ_STARVE_RPBH) ? 1 : 0;
     p.s_max = (float)(3.4028234663852886e38 / (2.0 * std::sqrt((double)h)));
     if (rpbh_smem_bytes(p) > 227 * 1024) return OQ_ERR_UNSUPPORTED;
     const int grid = p.ntiles < device_sms() ? p.ntiles : device_sms();
@@ -117,7 +135,7 @@ oq_status codebook_device(oq_codebook_t* cb, const DeviceCodebook** out) {
     if (!dc.lut) {
         void* ptr = nullptr;
         const size_t bytes = cb->lut.size() * sizeof(LutEntry);
-        if (cudaMalloc(&ptr, bytes) != cudaSuccess) return OQ_ERR_OOM;
+        if (!device_alloc(&ptr, bytes)) return OQ_ERR_OOM;
         if (cudaMemcpy(ptr, cb->lut.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
             cudaFree(ptr);
             return OQ_ERR_CUDA;
@@ -236,7 +254,7 @@ oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t**
     make_plan(d, h, seed, p->perm.data(), p->sign.data(), variant);
     build_gather_table(p, p->gtab_host);
     void* ptr = nullptr;
-    if (cudaMalloc(&ptr, sizeof(uint16_t) * d) != cudaSuccess) {
+    if (!device_alloc(&ptr, sizeof(uint16_t) * d)) {
         delete p;
         return OQ_ERR_OOM;
     }
@@ -322,6 +340,7 @@ static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
     a.fp8 = fp8;
     a.ca_e4m3 = cb_a->c_e4m3.data();
     a.cw_e4m3 = cb_w->c_e4m3.data();
+    a.starve = take_starve(OQ_STARVE_GEMM);
     cudaError_t e = launch_qgemm(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
 }
@@ -432,6 +451,10 @@ oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     return oq_qlinear(plan, cb_a, cb_w, x, dtype, M, w_idx, w_r, N, bias, y, scratch, OQ_NOALLOC_SCRATCH_BYTES,
                       stream);
 }
+
+void oq_debug_fail_allocations(int n) { g_fail_allocs.store(n > 0 ? n : 0); }
+
+void oq_debug_starve(int mask) { g_starve_mask.store(mask & (OQ_STARVE_RPBH | OQ_STARVE_GEMM)); }
 
 oq_status oq_device_status(int clear, int* out, void* stream) {
     if (!out) return OQ_ERR_INVALID_ARG;

@@ -96,6 +96,7 @@ struct QgemmParams {
     const uint16_t* bias;
     uint16_t* y;
     float out_scale;              // extra output scale (1/d in the fp8 variant, whose centroids are scaled by sqrt(d))
+    int starve;                   // test hook: the producer issues no loads
     uint32_t tab_a[4], tab_w[4];  // byte-permute tables of the register decoders
     uint16_t c6a[64], c6w[64];    // 6-bit tables (bf16)
     uint8_t c6a8[64], c6w8[64];   // 6-bit tables (e4m3)
@@ -549,7 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
             RingPos<P_STAGES> ps;
             int issued = 0;
-            bool ok = true;
+            bool ok = !p.starve;  // a starved launch loads nothing: every consumer's wait runs out
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 const int m0 = (tile % p.num_m) * TM + (int)rank * HM;
                 const int n0 = (tile / p.num_m) * TN + (int)rank * HN;
@@ -894,6 +895,7 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     prm.w_r = a.w_r;
     prm.bias = a.bias;
     prm.y = a.y;
+    prm.starve = a.starve ? 1 : 0;
     if (f8) {
         prm.out_scale = (float)(1.0 / (double)a.K);  // both operands' centroids carry sqrt(d)
         fill_tables_e4m3(a.bits_a, a.ca_e4m3, prm.tab_a, prm.c6a8);

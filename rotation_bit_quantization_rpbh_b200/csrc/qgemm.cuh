@@ -20,6 +20,7 @@ struct QgemmArgs {
     bool fp8;                // e4m3 variant: centroids c_j sqrt(d) as e4m3, K % 128 == 0
     const uint8_t* ca_e4m3;  // activation centroids (fp8 variant)
     const uint8_t* cw_e4m3;  // weight centroids (fp8 variant)
+    bool starve = false;     // test hook: the producer issues no loads (the waits run out)
 };
 
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream);

@@ -88,13 +88,17 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
     uint64_t* s_bar = all_bars + 2 * grp;
     uint64_t* tab_bar = all_bars + 2 * NG;
 
-    auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) {
+    // returns whether a copy was issued; a starved launch (test hook) issues
+    // none, so the stage waits below run out and report a timeout
+    auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) -> int {
+        if (p.starve) return 0;
         const int row0 = tile * R;
         const int rows = min(R, p.M - row0);
         mbar_arrive_expect_tx(&bars[st], (uint32_t)(rows * p.row_bytes));
         const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
         uint8_t* dst = stage + st * R * p.srow;
         for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &bars[st]);
+        return 1;
     };
 
     // this group's tiles: blockIdx.x + (NG k + grp) * gridDim.x
@@ -128,8 +132,7 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
         const int next = tile + step;
         pending_other = 0;
         if (tg == 0 && next < p.ntiles) {
-            issue(s_bar, s_stage, next, st ^ 1);  // streams in while this tile is computed
-            pending_other = 1;
+            pending_other = issue(s_bar, s_stage, next, st ^ 1);  // streams in while this tile is computed
         }
         if (it == 0 && !mbar_wait_bounded(tab_bar, 0u)) s_abort[grp] = 1;
         if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort[grp] = 1;

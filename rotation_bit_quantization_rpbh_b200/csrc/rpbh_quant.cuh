@@ -28,6 +28,7 @@ struct RpbhParams {
     float rsqrt_h;         // 1/sqrt(h)
     float eps;             // the split's eps
     float s_max;           // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
+    int starve;            // test hook: issue no row copies (the waits run out)
 };
 
 constexpr int kMaxGroups = 3;  // warp groups per CTA (at most 128 threads each)

@@ -115,6 +115,27 @@ def test_argument_checks_on_host_calls():
     assert L.oq_rpbh_plan_host(256, 64, 0, P, S) == 0
 
 
+def test_debug_hooks_leave_host_calls_alone():
+    """The failure hooks only touch device allocations and kernel launches:
+    host-side plans and codebooks are built while failures are pending."""
+    import ctypes
+
+    L = B.lib()
+    B.debug_fail_allocations(3)
+    B.debug_starve(B.OQ_STARVE_RPBH | B.OQ_STARVE_GEMM)
+    try:
+        perm = np.zeros(256, dtype=np.int32)
+        sign = np.zeros(256, dtype=np.int8)
+        assert L.oq_rpbh_plan_host(256, 64, 3, perm.ctypes.data_as(ctypes.c_void_p),
+                                   sign.ctypes.data_as(ctypes.c_void_p)) == 0
+        assert sorted(perm.tolist()) == list(range(256))
+        cb = B.codebook(256, 4)
+        assert cb.bits == 4
+    finally:
+        B.debug_fail_allocations(0)
+        B.debug_starve(0)
+
+
 def test_workspace_size():
     ws = B.qlinear_workspace(4096, 3072, 4)
     assert ws >= 4096 * 1536 + 4096 * 4 and ws % 256 == 0
