@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline sample")
     ap.add_argument("--fp8", action="store_true",
                     help="time the fp8 variant of the product (oq_qgemm_fp8: e4m3 centroid values)")
+    ap.add_argument("--schedule", default="auto", choices=["auto", "codes", "values"],
+                    help="layer schedule timed: activation codes decoded in the GEMM, or centroid values written by "
+                         "the quantiser and streamed into the GEMM; auto = the one oq_qlinear takes")
     ap.add_argument("--ablation", action="store_true",
                     help="time the rotation ablation (RPBH, Block-RHT, dense Haar) on --workload instead of the layer")
     return ap.parse_args()
@@ -56,7 +59,9 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-KERNEL_SOURCES = {"qgemm": "qgemm.cu", "qgemm_fp8": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu"}
+KERNEL_SOURCES = {"qgemm": "qgemm.cu", "qgemm_fp8": "qgemm.cu", "qgemm_values": "qgemm.cu",
+                  "qgemm_values_fp8": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu", "rpbh_quant_values": "rpbh_quant.cu",
+                  "rpbh_quant_values_fp8": "rpbh_quant.cu"}
 
 
 def committed_traffic(kernel, workload):
@@ -170,10 +175,16 @@ def job_throughput(world, tokens_per_rank, ms_per_step):
     return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
-def rpbh_bytes(w):
+def rpbh_bytes(w, schedule="codes", fp8=False):
+    """Algorithmic bytes of one quantiser launch: x read, then the packed
+    codes (codes schedule) or the centroid values (values schedule: 2 bytes
+    each, 1 in e4m3) written, plus s."""
     esize = 4 if w.x_dtype == "f32" else 2
-    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
-    return w.M * (w.d * esize + packed + 4)
+    if schedule == "values":
+        out = w.d * (1 if fp8 else 2)
+    else:
+        out = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+    return w.M * (w.d * esize + out + 4)
 
 
 def cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, max_rows):
@@ -295,20 +306,40 @@ def run_ours(args):
     cb_a, cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
     x = x_cpu.to(dev)
     w_idx, w_r = B.quantize_weights(plan, cb_w, W_cpu.to(dev))  # offline pass, untimed
-    ws = torch.empty(B.qlinear_workspace(w.M, w.d, w.bits_a), dtype=torch.uint8, device=dev)
-    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
-    a_idx = ws[: w.M * packed].view(w.M, packed)
-    s_off = (w.M * packed + 255) // 256 * 256
+    schedule = "values" if args.schedule == "auto" else args.schedule  # the one oq_qlinear takes
+    ws = torch.empty(max(B.qlinear_workspace(w.M, w.d, w.bits_a), B.qlinear_workspace_values(w.M, w.d)),
+                     dtype=torch.uint8, device=dev)
+    if schedule == "values":
+        vb = 1 if args.fp8 else 2
+        a_in = ws[: w.M * w.d * vb].view(w.M, w.d * vb)
+        if not args.fp8:
+            a_in = a_in.view(torch.bfloat16)
+        s_off = (w.M * w.d * vb + 255) // 256 * 256
+    else:
+        packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+        a_in = ws[: w.M * packed].view(w.M, packed)
+        s_off = (w.M * packed + 255) // 256 * 256
     s = ws[s_off: s_off + 4 * w.M].view(torch.float32)
     y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
     stream = torch.cuda.current_stream()
 
-    gemm = B.qgemm_fp8 if args.fp8 else B.qgemm
+    if schedule == "values":
+        def quant():
+            B.quantize_acts_values(plan, cb_a, x, a_in, s, stream=stream, fp8=args.fp8)
+
+        def gemm():
+            B.qgemm_values(cb_w, a_in, s, w_idx, w_r, y=y, stream=stream, fp8=args.fp8)
+    else:
+        def quant():
+            B.quantize_acts(plan, cb_a, x, a_in, s, stream=stream)
+
+        def gemm():
+            (B.qgemm_fp8 if args.fp8 else B.qgemm)(cb_a, cb_w, a_in, s, w_idx, w_r, y=y, stream=stream)
 
     def step():
-        B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
-        gemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+        quant()
+        gemm()
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -330,9 +361,9 @@ def run_ours(args):
     for i in range(args.steps):
         flush.zero_()  # cold L2 for every step (outside the events)
         ev[i][0].record(stream)
-        B.quantize_acts(plan, cb_a, x, a_idx, s, stream=stream)
+        quant()
         ev[i][1].record(stream)
-        gemm(cb_a, cb_w, a_idx, s, w_idx, w_r, y=y, stream=stream)
+        gemm()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -360,7 +391,11 @@ def run_ours(args):
         nbuf = 2
         xs = [torch.empty_like(x) for _ in range(nbuf)]
         ys = [torch.empty_like(y) for _ in range(nbuf)]
-        wss = [torch.empty_like(ws) for _ in range(nbuf)]
+        # oq_qlinear takes its preferred schedule when the workspace holds it;
+        # a codes-sized workspace makes it take the codes schedule
+        e2e_schedule = schedule
+        ws_e2e = ws.numel() if e2e_schedule == "values" else B.qlinear_workspace(w.M, w.d, w.bits_a)
+        wss = [torch.empty(ws_e2e, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
         y_pins = [torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
         s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(nbuf)]
@@ -398,7 +433,8 @@ def run_ours(args):
         e2e = {"value": job_throughput(world, w.M, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_cpu.numel() * x_cpu.element_size()),
                "d2h_bytes_per_step": int(y.numel() * y.element_size()), "ms_per_step": e2e_ms,
-               "pipeline": "copy-in, oq_qlinear and copy-out on three streams, two buffers deep"}
+               "pipeline": "copy-in, oq_qlinear and copy-out on three streams, two buffers deep",
+               "schedule": e2e_schedule}
 
     peaks = measured_peaks()
     # the fp8 variant's contraction peak: the measured bf16 peak times the
@@ -408,27 +444,30 @@ def run_ours(args):
     flops = 2.0 * w.M * w.N * w.d
     gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
     step_tflops = flops / (ms * 1e-3) / 1e12
-    rb = rpbh_bytes(w)
+    rb = rpbh_bytes(w, schedule, args.fp8)
     rpbh_gbs = rb / (ms_rpbh * 1e-3) / 1e9
+    gemm_key = ("qgemm_values" if schedule == "values" else "qgemm") + ("_fp8" if args.fp8 else "")
+    rpbh_key = "rpbh_quant" + (("_values_fp8" if args.fp8 else "_values") if schedule == "values" else "")
     out = {
         "metric": METRIC, "value": job_throughput(world, w.M, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "d": w.d, "N": w.N, "h": w.h, "bits_w": w.bits_w,
                    "bits_a": w.bits_a, "x_dtype": w.x_dtype, "tokens_per_gpu": w.M, "global_batch": world * w.M,
-                   "parallelism": f"dp{world} (replicated packed W, no collective)",
+                   "parallelism": f"dp{world} (replicated packed W, no collective)", "schedule": schedule,
                    "l2": "flushed (256 MB write) before every timed step, outside the events"},
         "tflops": step_tflops,
         "breakdown": {"rpbh_quant_ms": ms_rpbh, "qgemm_ms": ms_gemm, "qgemm_tflops": gemm_tflops,
                       "rpbh_quant_gbs": rpbh_gbs},
-        "roofline": {"bound": "tensor", "kernel": "qgemm_fp8" if args.fp8 else "qgemm", "achieved": gemm_tflops,
+        "roofline": {"bound": "tensor", "kernel": gemm_key, "achieved": gemm_tflops,
                      "peak": mma_peak, "unit": "TFLOP/s", "frac": gemm_tflops / mma_peak,
-                     "traffic": committed_traffic("qgemm_fp8" if args.fp8 else "qgemm", w.name), "peak_source": peak_note,
+                     "traffic": committed_traffic(gemm_key, w.name), "peak_source": peak_note,
                      "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
-        "roofline_rpbh": {"bound": "hbm", "kernel": "rpbh_quant", "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
+        "roofline_rpbh": {"bound": "hbm", "kernel": rpbh_key, "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
                           "unit": "GB/s", "frac": rpbh_gbs / peaks["hbm_gbs"],
-                          "traffic": committed_traffic("rpbh_quant", w.name),
-                          "algorithmic": f"M*(d*in_bytes + packed + 4) = {rb} B per launch"},
+                          "traffic": committed_traffic(rpbh_key, w.name),
+                          "algorithmic": f"M*(d*in_bytes + {'values' if schedule == 'values' else 'packed'} + 4) = "
+                                         f"{rb} B per launch"},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "e2e": e2e,

@@ -160,6 +160,19 @@ oq_status oq_quantize_weights(const oq_plan_t* plan, const oq_codebook_t* cb_w, 
 oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype, int M,
                            uint8_t* idx_out, float* s_out, void* stream);
 
+/* The online pass with the centroid values written instead of the codes:  */
+/* val_out[m, k] = C_a[idx[m, k]] with idx as oq_quantize_acts decides it  */
+/* (same decision, same middle-cell rule), and the same s_out.            */
+/*   val_out device, [M, d] bf16 bit patterns (the bf16 centroid values    */
+/*           the product uses), row-major.                                 */
+/* The _fp8 form writes the e4m3 bytes of c sqrt(d) that oq_qgemm_fp8      */
+/* decodes to (oq_codebook_fp8); it needs d % 128 == 0.  Any bits in       */
+/* {2, 3, 4, 6}.  Used by the values schedule of oq_qlinear.               */
+oq_status oq_quantize_acts_values(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
+                                  int M, uint16_t* val_out, float* s_out, void* stream);
+oq_status oq_quantize_acts_values_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
+                                      int M, uint8_t* val_out, float* s_out, void* stream);
+
 /* Test hook: steps A1-A4 only (permute, sign, block WHT, norm).           */
 /*   x_rot   device, [M, d] fp32: x' = Pi_d x.   norm_out device, [M] fp32. */
 oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, int M, float* x_rot, float* norm_out,
@@ -190,19 +203,42 @@ oq_status oq_qgemm_fp8(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int
                        const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                        void* stream);
 
+/* oq_qgemm with A given as centroid values instead of codes:             */
+/*   y[m, n] = r_n * s_m * sum_k  C_w[iw[n, k]] * a_val[m, k]  (+ bias_n)    */
+/*   a_val   device, [M, d] bf16 (oq_quantize_acts_values), row-major.     */
+/* With a_val = C_a[ia] this gives oq_qgemm's result bit for bit: the       */
+/* tensor cores see the same values in the same order; only W is decoded   */
+/* in the kernel, and A's values arrive by TMA.  d % 64 == 0, bits_w in     */
+/* {2, 4, 6}.  The _fp8 form takes e4m3 bytes of c sqrt(d)                  */
+/* (oq_quantize_acts_values_fp8) and matches oq_qgemm_fp8 bit for bit;     */
+/* d % 128 == 0, bits_w in {2, 3, 4, 6}.                                    */
+oq_status oq_qgemm_values(const oq_codebook_t* cb_w, int M, int N, const uint16_t* a_val, const float* s,
+                          const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y, void* stream);
+oq_status oq_qgemm_values_fp8(const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_val, const float* s,
+                              const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                              void* stream);
+
 /* The fp8 variant's centroid values: out[2^bits] host bytes, e4m3 of     */
 /* c_j sqrt(d) (sign, 4 exponent bits with bias 7, 3 mantissa bits).        */
 oq_status oq_codebook_fp8(const oq_codebook_t* cb, uint8_t* out);
 
-/* Bytes of workspace oq_qlinear needs for M rows (packed activation       */
-/* indices plus their norms, 256-byte aligned sections).                   */
+/* Bytes of workspace oq_qlinear needs for M rows in its codes schedule   */
+/* (packed activation indices plus their norms, 256-byte aligned sections) */
+/* and in its values schedule (bf16 activation values plus norms; enough  */
+/* for the fp8 form too).                                                  */
 size_t oq_qlinear_workspace(int M, int d, int bits_a);
+size_t oq_qlinear_workspace_values(int M, int d);
 
-/* Full layer x -> y: oq_quantize_acts into `workspace`, then oq_qgemm.     */
+/* Full layer x -> y.  Two schedules with the same result bit for bit:    */
+/*   values: oq_quantize_acts_values into `workspace`, then               */
+/*     oq_qgemm_values; taken when ws_bytes >=                             */
+/*     oq_qlinear_workspace_values(M, d) (fp8: M*d bytes plus the norms,  */
+/*     256-byte aligned sections, suffice).  The faster one on B200.      */
+/*   codes: oq_quantize_acts into `workspace`, then oq_qgemm; otherwise,  */
+/*     with ws_bytes >= oq_qlinear_workspace(M, d, bits_a).                */
 /*   x device [M, d] of dtype; w_idx / w_r from oq_quantize_weights with the */
-/*   same plan; workspace device, >= oq_qlinear_workspace(M, d, bits_a)     */
-/*   bytes, 256-byte aligned (OQ_ERR_OOM if too small).  Other arguments as */
-/*   in oq_qgemm.                                                           */
+/*   same plan; workspace device, 256-byte aligned (OQ_ERR_OOM if smaller   */
+/*   than both sizes).  Other arguments as in oq_qgemm.                     */
 oq_status oq_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, const void* x,
                      oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N, const uint16_t* bias,
                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
@@ -223,7 +259,9 @@ oq_status oq_qlinear_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const
 /*   Same arguments and results as oq_qlinear, minus the workspace: the   */
 /*   packed activation codes and their norms go to a scratch array that   */
 /*   the library reserves statically on every device that loads it        */
-/*   (OQ_NOALLOC_SCRATCH_BYTES, 64 MiB, held until the process exits).    */
+/*   (OQ_NOALLOC_SCRATCH_BYTES, 128 MiB, held until the process exits),   */
+/*   in the values schedule when its workspace fits there, else in the    */
+/*   codes schedule.                                                       */
 /*   Requests needing more than that (oq_qlinear_workspace(M, d, bits_a)  */
 /*   > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE before any work. */
 /*   Nothing is allocated here: the plan and both codebooks must already  */
@@ -236,7 +274,7 @@ oq_status oq_qlinear_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const
 /*   contents; every call overwrites the part it reads, so nothing needs  */
 /*   clearing.  Calls whose kernels overlap on the GPU (other streams,    */
 /*   other host threads) race on the array: order them on one stream.    */
-#define OQ_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+#define OQ_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
 oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
                              const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
                              const uint16_t* bias, uint16_t* y, void* stream);

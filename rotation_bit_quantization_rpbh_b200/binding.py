@@ -23,7 +23,7 @@ OQ_ROT_RPBH, OQ_ROT_BLOCK_RHT = 0, 1
 OQ_STARVE_RPBH, OQ_STARVE_GEMM = 1, 2
 _STATUS = {0: "OQ_OK", 1: "OQ_ERR_INVALID_ARG", 2: "OQ_ERR_UNSUPPORTED", 3: "OQ_ERR_ALIGNMENT", 4: "OQ_ERR_CUDA",
            5: "OQ_ERR_TIMEOUT", 6: "OQ_ERR_OOM", 7: "OQ_ERR_NO_CONVERGENCE", 8: "OQ_ERR_TOO_LARGE"}
-NOALLOC_SCRATCH_BYTES = 64 << 20
+NOALLOC_SCRATCH_BYTES = 128 << 20
 
 # every symbol include/oq.h declares
 EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf16", "oq_codebook_shape",
@@ -32,7 +32,8 @@ EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf
            "oq_qlinear_fp8",
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status",
-           "oq_debug_fail_allocations", "oq_debug_starve"]
+           "oq_debug_fail_allocations", "oq_debug_starve", "oq_quantize_acts_values",
+           "oq_quantize_acts_values_fp8", "oq_qgemm_values", "oq_qgemm_values_fp8", "oq_qlinear_workspace_values"]
 
 
 class OQError(RuntimeError):
@@ -83,6 +84,11 @@ def lib():
                     "oq_device_status": ([I, P, P], I),
                     "oq_debug_fail_allocations": ([I], None),
                     "oq_debug_starve": ([I], None),
+                    "oq_quantize_acts_values": ([P, P, P, I, I, P, P, P], I),
+                    "oq_quantize_acts_values_fp8": ([P, P, P, I, I, P, P, P], I),
+                    "oq_qgemm_values": ([P, I, I, P, P, P, P, P, P, P], I),
+                    "oq_qgemm_values_fp8": ([P, I, I, P, P, P, P, P, P, P], I),
+                    "oq_qlinear_workspace_values": ([I, I], SZ),
                 }
                 for name, (args, res) in sig.items():
                     f = getattr(L, name)
@@ -248,6 +254,21 @@ def quantize_acts(plan, cb_a, x, idx_out=None, s_out=None, stream=None):
     return idx_out, s_out
 
 
+def quantize_acts_values(plan, cb_a, x, val_out=None, s_out=None, stream=None, fp8=False):
+    """The online pass writing the centroid values C_a[idx] (a bf16 tensor
+    [M, d]) instead of the codes; ``fp8=True`` writes the e4m3 bytes of
+    c sqrt(d) (uint8)."""
+    M, d = x.shape
+    if val_out is None:
+        val_out = torch.empty((M, d), dtype=torch.uint8 if fp8 else torch.bfloat16, device=x.device)
+    if s_out is None:
+        s_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    fn, name = ((lib().oq_quantize_acts_values_fp8, "oq_quantize_acts_values_fp8") if fp8
+                else (lib().oq_quantize_acts_values, "oq_quantize_acts_values"))
+    _check(fn(plan.handle, cb_a.handle, _ptr(x), _dtype_code(x), M, _ptr(val_out), _ptr(s_out), _stream(stream)), name)
+    return val_out, s_out
+
+
 def rpbh_apply(plan, x, x_rot=None, norm_out=None, stream=None):
     M, d = x.shape
     if x_rot is None:
@@ -278,17 +299,42 @@ def qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
     return y
 
 
+def qgemm_values(cb_w, a_val, s, w_idx, w_r, bias=None, y=None, stream=None, fp8=False):
+    """The product with A given as centroid values (bf16 [M, d], or uint8
+    e4m3 bytes with ``fp8=True``): only W is decoded in the kernel."""
+    M, N = a_val.shape[0], w_idx.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_val.device)
+    fn, name = (lib().oq_qgemm_values_fp8, "oq_qgemm_values_fp8") if fp8 else (lib().oq_qgemm_values,
+                                                                                "oq_qgemm_values")
+    _check(fn(cb_w.handle, M, N, _ptr(a_val), _ptr(s), _ptr(w_idx), _ptr(w_r), _ptr(bias), _ptr(y), _stream(stream)),
+           name)
+    return y
+
+
 def qlinear_workspace(M, d, bits_a):
     return int(lib().oq_qlinear_workspace(M, d, bits_a))
 
 
-def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None, fp8=False):
-    """The full layer x -> y (oq_qlinear; oq_qlinear_fp8 with fp8=True)."""
+def qlinear_workspace_values(M, d):
+    return int(lib().oq_qlinear_workspace_values(M, d))
+
+
+def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None, fp8=False,
+            schedule="auto"):
+    """The full layer x -> y (oq_qlinear; oq_qlinear_fp8 with fp8=True).
+    ``schedule`` sizes the workspace allocated here: "auto" (room for the
+    values schedule, which the library then takes) or "codes"."""
     M, d = x.shape
     N = w_idx.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    need = qlinear_workspace(M, d, cb_a.bits)
+    if schedule not in ("auto", "codes"):
+        raise ValueError(f"unknown schedule {schedule!r}")
+    if schedule == "auto":
+        need = max(qlinear_workspace_values(M, d), qlinear_workspace(M, d, cb_a.bits))
+    else:
+        need = qlinear_workspace(M, d, cb_a.bits)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     fn, name = (lib().oq_qlinear_fp8, "oq_qlinear_fp8") if fp8 else (lib().oq_qlinear, "oq_qlinear")

@@ -50,7 +50,9 @@ bool quant_bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bit
 
 int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }
 
-// Launch the fused rotate/quantise kernel in one of its three modes.
+// Launch the fused rotate/quantise kernel in one of its modes: 0 activation
+// codes, 1 weight codes, 2 rotation only, 3 / 4 activation values (bf16 /
+// e4m3 of c sqrt(d)) written to idx_out.
 oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_dtype dtype, int M, int mode,
                    uint8_t* idx_out, float* s_out, uint16_t* r_out, float* y_out, float* norm_out, cudaStream_t st) {
     if (!plan || M < 0) return OQ_ERR_INVALID_ARG;
@@ -63,11 +65,12 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
         if (!idx_out) return OQ_ERR_INVALID_ARG;
         if (cb->d != plan->d) return OQ_ERR_INVALID_ARG;
         if (!quant_bits_ok(cb->bits)) return OQ_ERR_UNSUPPORTED;
-        if (packed_row_bytes(plan->d, cb->bits) % 4 != 0) return OQ_ERR_UNSUPPORTED;
-        if (cb->bits == 3 && (plan->h < 32 || plan->d % 128 != 0)) return OQ_ERR_UNSUPPORTED;  // 16-byte rows
+        if (mode < 2 && packed_row_bytes(plan->d, cb->bits) % 4 != 0) return OQ_ERR_UNSUPPORTED;
+        if (mode < 2 && cb->bits == 3 && (plan->h < 32 || plan->d % 128 != 0))
+            return OQ_ERR_UNSUPPORTED;  // 16-byte rows
         if (!aligned16(idx_out)) return OQ_ERR_ALIGNMENT;
     }
-    if (mode == 0 && (!s_out || !aligned16(s_out))) return s_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
+    if ((mode == 0 || mode >= 3) && (!s_out || !aligned16(s_out))) return s_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
     if (mode == 1 && (!r_out || !aligned16(r_out))) return r_out ? OQ_ERR_ALIGNMENT : OQ_ERR_INVALID_ARG;
     if (mode == 2 && (!y_out || !norm_out)) return OQ_ERR_INVALID_ARG;
     if (mode == 2 && (!aligned16(y_out) || !aligned16(norm_out))) return OQ_ERR_ALIGNMENT;
@@ -104,11 +107,12 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.ntiles = (M + R - 1) / R;
     p.gtab = plan->dev.gtab;
     if (mode != 2) {
-        p.lut = dcb->lut;
+        p.lut = mode == 3 ? dcb->lut_vb : (mode == 4 ? dcb->lut_v8 : dcb->lut);
         p.lut_off = -(int)kLutMagicBits - cb->kmin;
         p.G_lut = cb->G;
         p.L = cb->L;
-        p.out_row_bytes = packed_row_bytes(d, cb->bits);
+        p.out_row_bytes = mode == 3 ? 2 * d : (mode == 4 ? d : packed_row_bytes(d, cb->bits));
+        p.mid_val = mode == 3 ? cb->c_bf16[cb->L / 2] : (mode == 4 ? cb->c_e4m3[cb->L / 2] : 0u);
     }
     p.idx_out = idx_out;
     p.s_out = s_out;
@@ -133,14 +137,28 @@ oq_status codebook_device(oq_codebook_t* cb, const DeviceCodebook** out) {
     std::lock_guard<std::mutex> lk(cb->mu);
     DeviceCodebook& dc = cb->dev[dev];
     if (!dc.lut) {
+        // three tables of the same bins: code counts, then the bf16 and the
+        // e4m3 centroid values of the two cells each bin can give (the one
+        // below its threshold in the low half, the one above in the high)
+        const size_t n = cb->lut.size();
+        std::vector<LutEntry> all(3 * n);
+        for (size_t i = 0; i < n; ++i) {
+            const LutEntry& e = cb->lut[i];
+            const int lo = e.base, hi = e.base + 1 < cb->L ? e.base + 1 : e.base;
+            all[i] = e;
+            all[n + i] = {e.T, (int32_t)((uint32_t)cb->c_bf16[lo] | ((uint32_t)cb->c_bf16[hi] << 16))};
+            all[2 * n + i] = {e.T, (int32_t)((uint32_t)cb->c_e4m3[lo] | ((uint32_t)cb->c_e4m3[hi] << 8))};
+        }
         void* ptr = nullptr;
-        const size_t bytes = cb->lut.size() * sizeof(LutEntry);
+        const size_t bytes = all.size() * sizeof(LutEntry);
         if (!device_alloc(&ptr, bytes)) return OQ_ERR_OOM;
-        if (cudaMemcpy(ptr, cb->lut.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+        if (cudaMemcpy(ptr, all.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
             cudaFree(ptr);
             return OQ_ERR_CUDA;
         }
         dc.lut = static_cast<LutEntry*>(ptr);
+        dc.lut_vb = dc.lut + n;
+        dc.lut_v8 = dc.lut + 2 * n;
     }
     *out = &dc;
     return OQ_OK;
@@ -301,6 +319,19 @@ oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, con
                     static_cast<cudaStream_t>(stream));
 }
 
+oq_status oq_quantize_acts_values(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
+                                  int M, uint16_t* val_out, float* s_out, void* stream) {
+    return run_rpbh(plan, const_cast<oq_codebook_t*>(cb_a), x, dtype, M, 3, reinterpret_cast<uint8_t*>(val_out), s_out,
+                    nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_quantize_acts_values_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
+                                      int M, uint8_t* val_out, float* s_out, void* stream) {
+    if (cb_a && cb_a->d % 128 != 0) return OQ_ERR_UNSUPPORTED;  // the fp8 product's K step
+    return run_rpbh(plan, const_cast<oq_codebook_t*>(cb_a), x, dtype, M, 4, val_out, s_out, nullptr, nullptr, nullptr,
+                    static_cast<cudaStream_t>(stream));
+}
+
 oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, int M, float* x_rot, float* norm_out,
                         void* stream) {
     return run_rpbh(plan, nullptr, x, dtype, M, 2, nullptr, nullptr, nullptr, x_rot, norm_out,
@@ -345,6 +376,52 @@ static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
     return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
 }
 
+// The product with A given as centroid values (bf16, or e4m3 of c sqrt(d)).
+static oq_status run_qgemm_values(const oq_codebook_t* cb_w, int M, int N, const void* a_val, const float* s,
+                                  const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                                  void* stream, bool fp8) {
+    if (!cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
+    if (!quant_bits_ok(cb_w->bits) || cb_w->d % (fp8 ? 128 : 64) != 0) return OQ_ERR_UNSUPPORTED;
+    if (!fp8 && cb_w->bits == 3) return OQ_ERR_UNSUPPORTED;
+    if (M == 0) return OQ_OK;
+    if (!a_val || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
+    if (!aligned16(a_val) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
+        (bias && !aligned16(bias)))
+        return OQ_ERR_ALIGNMENT;
+    QgemmArgs a;
+    a.M = M;
+    a.N = N;
+    a.K = cb_w->d;
+    a.bits_a = 0;
+    a.bits_w = cb_w->bits;
+    a.a_idx = nullptr;
+    a.a_val = a_val;
+    a.w_idx = w_idx;
+    a.s = s;
+    a.w_r = w_r;
+    a.bias = bias;
+    a.y = y;
+    a.ca_bf16 = nullptr;
+    a.cw_bf16 = cb_w->c_bf16.data();
+    a.fp8 = fp8;
+    a.ca_e4m3 = nullptr;
+    a.cw_e4m3 = cb_w->c_e4m3.data();
+    a.starve = take_starve(OQ_STARVE_GEMM);
+    cudaError_t e = launch_qgemm(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
+}
+
+oq_status oq_qgemm_values(const oq_codebook_t* cb_w, int M, int N, const uint16_t* a_val, const float* s,
+                          const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y, void* stream) {
+    return run_qgemm_values(cb_w, M, N, a_val, s, w_idx, w_r, bias, y, stream, false);
+}
+
+oq_status oq_qgemm_values_fp8(const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_val, const float* s,
+                              const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
+                              void* stream) {
+    return run_qgemm_values(cb_w, M, N, a_val, s, w_idx, w_r, bias, y, stream, true);
+}
+
 oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
                    const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                    void* stream) {
@@ -370,6 +447,11 @@ size_t oq_qlinear_workspace(int M, int d, int bits_a) {
     return idx_al + ((size_t)M * sizeof(float) + 255) / 256 * 256;
 }
 
+size_t oq_qlinear_workspace_values(int M, int d) {
+    if (M <= 0 || d <= 0) return 0;
+    return ((size_t)M * (size_t)d * 2 + 255) / 256 * 256 + ((size_t)M * sizeof(float) + 255) / 256 * 256;
+}
+
 static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
                              const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
                              const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream,
@@ -381,6 +463,22 @@ static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     if (M == 0) return OQ_OK;
     if (!workspace) return OQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return OQ_ERR_ALIGNMENT;
+    // The values schedule (the quantiser writes c_index itself; the product
+    // loads A's values by TMA and decodes only W) trades A's in-kernel decode
+    // for four (bf16) or two (e4m3) times the bytes of A to stream per tile;
+    // with a deep A ring and N-fastest tiles it is the faster one on B200 at
+    // every shape measured, so it is taken whenever the workspace holds it.
+    const size_t val_al = ((size_t)M * plan->d * (fp8 ? 1 : 2) + 255) / 256 * 256;
+    if (ws_bytes >= val_al + ((size_t)M * sizeof(float) + 255) / 256 * 256) {
+        if (fp8 && plan->d % 128 != 0) return OQ_ERR_UNSUPPORTED;
+        float* s = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + val_al);
+        oq_status st = fp8 ? oq_quantize_acts_values_fp8(plan, cb_a, x, dtype, M, static_cast<uint8_t*>(workspace), s,
+                                                         stream)
+                           : oq_quantize_acts_values(plan, cb_a, x, dtype, M, static_cast<uint16_t*>(workspace), s,
+                                                     stream);
+        if (st != OQ_OK) return st;
+        return run_qgemm_values(cb_w, M, N, workspace, s, w_idx, w_r, bias, y, stream, fp8);
+    }
     const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
     if (ws_bytes < need) return OQ_ERR_OOM;
     uint8_t* a_idx = static_cast<uint8_t*>(workspace);
@@ -440,7 +538,7 @@ oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
     if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
-    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
+    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);  // the codes schedule; values when they fit
     if (need > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE;
     if (current_device() != plan->device) return OQ_ERR_INVALID_ARG;
     // the activation codebook's tables must already be here (its upload would allocate)

@@ -23,7 +23,9 @@ struct LutEntry {
 };
 
 struct DeviceCodebook {
-    LutEntry* lut = nullptr;  // device copy of the lookup table
+    LutEntry* lut = nullptr;     // device copy of the lookup table
+    LutEntry* lut_vb = nullptr;  // the same bins with bf16 centroid values (see codebook_device)
+    LutEntry* lut_v8 = nullptr;  // the same bins with e4m3 values of c sqrt(d)
 };
 
 struct DevicePlan {

@@ -38,6 +38,17 @@
 //               tcgen05.ld this CTA's 128 accumulator rows 32 columns at a
 //               time, scale by s_m r_n (+ bias) in fp32, round to bf16,
 //               store, and release the accumulator to the leader.
+// A-values variant (AV): A arrives as centroid values [M, K] (bf16, or e4m3
+// in the fp8 variant) written by the quantiser.  The producer also loads
+// each K step's 128 x 128-byte A box by TMA with 128-byte swizzle, straight
+// into the layout the MMA reads, into a ring of its own (as deep as shared
+// memory allows next to 4 packed W stages: these loads are latency-bound);
+// the decoders expand W only, and each group's lead waits for this CTA's A
+// box of the step before publishing it, so the leader's "stage full"
+// covers A in both CTAs.  Tiles run N-fastest, so the few A tiles in use
+// stay in L2 while the packed W cycles.  The MMAs see the same values in
+// the same order as in the codes variant: the result is identical bit for
+// bit.
 // The leader's MMA completions are multicast (tcgen05.commit) to the
 // barriers of both CTAs.  Every mbarrier wait is bounded: on a timeout the
 // kernel raises the device error flag, drains its own TMA loads, leaves the
@@ -57,7 +68,12 @@ namespace {
 
 constexpr int TM = 256, TN = 256;           // pair tile
 constexpr int HM = 128, HN = 128;           // rows of A and of W owned by one CTA
-constexpr int D_STAGES = 4;                 // decoded ring
+// Ring depths.  Decoded ring: 4 stages.  With A given as values (loaded by
+// TMA, see qgemm_kernel) the A ring is as deep as shared memory allows next
+// to 4 packed W stages, up to AV_MAX: its loads are latency-bound.
+constexpr int AV_MAX = 12;
+constexpr int PK_MIN_AV = 4;
+__host__ __device__ constexpr int d_stages(bool av) { return av ? 4 : 4; }
 constexpr int P_MAX = 10;                   // packed ring depth (fewer when the packed stage is large)
 constexpr int NDEC_WARPS = 16;
 constexpr int NGROUPS = 2;                        // decoder groups, taking alternate K steps
@@ -73,24 +89,39 @@ __host__ __device__ constexpr int bk_codes(bool f8) { return f8 ? 128 : 64; }
 __host__ __device__ constexpr int pk_row_bytes(int bits, bool f8) { return bits == 6 ? bk_codes(f8) : bk_codes(f8) * bits / 8; }
 // packed bytes behind one 16-byte decoded chunk (8 bf16 or 16 e4m3 values)
 __host__ __device__ constexpr int unit_bytes(int bits, bool f8) { return (f8 ? 16 : 8) * (bits == 6 ? 8 : bits) / 8; }
-__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw, bool f8) {
-    return HM * pk_row_bytes(ba, f8) + HN * pk_row_bytes(bw, f8);
+// With A given as values (av) the decoded ring holds W only and the packed
+// ring W's codes only; A's values have a ring of their own.
+__host__ __device__ constexpr int dec_stage_bytes(bool av) { return av ? DEC_B : DEC_STAGE; }
+__host__ __device__ constexpr int pk_stage_bytes(int ba, int bw, bool f8, bool av) {
+    return (av ? 0 : HM * pk_row_bytes(ba, f8)) + HN * pk_row_bytes(bw, f8);
 }
-__host__ __device__ constexpr int p_stages(int ba, int bw, bool f8) {
-    return (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw, f8) < P_MAX
-               ? (227 * 1024 - D_STAGES * DEC_STAGE - 3072) / pk_stage_bytes(ba, bw, f8)
+__host__ __device__ constexpr int av_stages(int bw, bool f8, bool av) {
+    return !av ? 0
+               : ((227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) / DEC_A <
+                          AV_MAX
+                      ? (227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) / DEC_A
+                      : AV_MAX);
+}
+__host__ __device__ constexpr int rings_bytes(int bw, bool f8, bool av) {
+    return d_stages(av) * dec_stage_bytes(av) + av_stages(bw, f8, av) * DEC_A;
+}
+__host__ __device__ constexpr int p_stages(int ba, int bw, bool f8, bool av) {
+    return (227 * 1024 - rings_bytes(bw, f8, av) - 3072) / pk_stage_bytes(ba, bw, f8, av) < P_MAX
+               ? (227 * 1024 - rings_bytes(bw, f8, av) - 3072) / pk_stage_bytes(ba, bw, f8, av)
                : P_MAX;
 }
-// decoded ring | packed ring | epilogue r and bias of a tile (1 KB) |
-// barriers (512 B) | alignment slack (1 KB); the 6-bit tables are static
-__host__ __device__ constexpr int smem_bytes(int ba, int bw, bool f8) {
-    return D_STAGES * DEC_STAGE + p_stages(ba, bw, f8) * pk_stage_bytes(ba, bw, f8) + 1024 + 512 + 1024;
+// decoded ring | A-values ring (av) | packed ring | epilogue r and bias of a
+// tile (1 KB) | barriers (512 B) | alignment slack (1 KB); the 6-bit tables
+// are static
+__host__ __device__ constexpr int smem_bytes(int ba, int bw, bool f8, bool av) {
+    return rings_bytes(bw, f8, av) + p_stages(ba, bw, f8, av) * pk_stage_bytes(ba, bw, f8, av) + 1024 + 512 + 1024;
 }
 
 struct QgemmParams {
     CUtensorMap tmA;
     CUtensorMap tmB;
-    int M, N, KB, num_m, num_tiles;
+    int M, N, KB, num_m, num_n, num_tiles;
+    int n_fastest;                // tile order: N tiles fastest (A's values stay in L2 while W's codes cycle)
     const float* s;
     const uint16_t* w_r;
     const uint16_t* bias;
@@ -431,12 +462,14 @@ struct StageCodes {
     PackedU<BW, F8> b[DEC_UNITS];
 };
 
-template <int BA, int BW, bool F8>
+// (AV: A arrives as values, so only W's codes are loaded and expanded)
+template <int BA, int BW, bool F8, bool AV>
 __device__ __forceinline__ void load_codes(StageCodes<BA, BW, F8>& u, const uint8_t* pa, const uint8_t* pb, int srcA,
                                            int srcB) {
     constexpr int PKRA = pk_row_bytes(BA, F8), PKRB = pk_row_bytes(BW, F8);
+    constexpr int NUA = AV ? 0 : DEC_UNITS;
 #pragma unroll
-    for (int i = 0; i < DEC_UNITS; ++i) u.a[i] = load_unit<BA, F8>(pa + srcA + i * DEC_ROWS * PKRA);
+    for (int i = 0; i < NUA; ++i) u.a[i] = load_unit<BA, F8>(pa + srcA + i * DEC_ROWS * PKRA);
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) u.b[i] = load_unit<BW, F8>(pb + srcB + i * DEC_ROWS * PKRB);
 }
@@ -447,22 +480,34 @@ struct StageValues {
     uint4 a[DEC_UNITS], b[DEC_UNITS];
 };
 
-template <int BA, int BW, bool F8>
+template <int BA, int BW, bool F8, bool AV>
 __device__ __forceinline__ void decode_codes(StageValues& v, const StageCodes<BA, BW, F8>& u, const uint32_t tab_a[4],
                                              const uint32_t tab_w[4]) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
-        v.a[i] = decode_unit<BA, 0, F8>(u.a[i], tab_a);
+        if constexpr (!AV) v.a[i] = decode_unit<BA, 0, F8>(u.a[i], tab_a);
         v.b[i] = decode_unit<BW, 1, F8>(u.b[i], tab_w);
     }
 }
 
+template <bool AV>
 __device__ __forceinline__ void store_values(const StageValues& v, uint8_t* da, uint8_t* db, int dst_off) {
 #pragma unroll
     for (int i = 0; i < DEC_UNITS; ++i) {
         // DEC_ROWS rows = DEC_ROWS / 8 swizzle atoms of 1024 bytes
-        *reinterpret_cast<uint4*>(da + dst_off + i * DEC_ROWS * 128) = v.a[i];
+        if constexpr (!AV) *reinterpret_cast<uint4*>(da + dst_off + i * DEC_ROWS * 128) = v.a[i];
         *reinterpret_cast<uint4*>(db + dst_off + i * DEC_ROWS * 128) = v.b[i];
+    }
+}
+
+// Tile coordinates (M tile, N tile) of linear tile index `tile`.
+__device__ __forceinline__ void tile_mn(const QgemmParams& p, int tile, int& mt, int& nt) {
+    if (p.n_fastest) {
+        nt = tile % p.num_n;
+        mt = tile / p.num_n;
+    } else {
+        mt = tile % p.num_m;
+        nt = tile / p.num_m;
     }
 }
 
@@ -481,17 +526,24 @@ struct RingPos {
 };
 
 // ----------------------------------------------------------------------------
-template <int BA, int BW, bool F8>
+template <int BA, int BW, bool F8, bool AV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     qgemm_kernel(const __grid_constant__ QgemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     // the same offset in both CTAs (dynamic shared memory starts at the same address)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int PKA = HM * pk_row_bytes(BA, F8);
-    constexpr int PK_STAGE = pk_stage_bytes(BA, BW, F8);
-    constexpr int P_STAGES = p_stages(BA, BW, F8);
+    constexpr int PKA = AV ? 0 : HM * pk_row_bytes(BA, F8);  // A's share of a packed stage
+    constexpr int PK_STAGE = pk_stage_bytes(BA, BW, F8, AV);
+    constexpr int P_STAGES = p_stages(BA, BW, F8, AV);
+    constexpr int D_STAGES = d_stages(AV);
+    constexpr int AV_STAGES = AV ? av_stages(BW, F8, AV) : 1;
+    static_assert(P_STAGES >= NGROUPS && D_STAGES >= NGROUPS && (!AV || AV_STAGES >= NGROUPS),
+                  "each decoder group starts on a stage of its own");
+    constexpr int DSTAGE = dec_stage_bytes(AV);  // decoded stage: A then W, or W alone (AV)
+    constexpr int DOFF_B = AV ? 0 : DEC_A;       // offset of W's values in a decoded stage
     uint8_t* dec = smem;
-    uint8_t* pk = smem + D_STAGES * DEC_STAGE;
+    uint8_t* av = smem + D_STAGES * DSTAGE;      // A-values ring (AV): 1024-byte aligned stages for the swizzled TMA
+    uint8_t* pk = smem + rings_bytes(BW, F8, AV);
     uint16_t* epi_r = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);  // r_n of the tile's 256 columns
     uint16_t* epi_b = epi_r + TN;   // bias of those columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_b + TN);
@@ -501,7 +553,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     uint64_t* dec_empty = dec_full + D_STAGES;  // arrived by the leader's multicast commit
     uint64_t* acc_full = dec_empty + D_STAGES;  // arrived by the leader's multicast commit
     uint64_t* acc_empty = acc_full + 2;         // leader's counts both CTAs' epilogues
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    uint64_t* av_full = acc_empty + 2;          // AV: this CTA's A values landed (TMA transaction bytes)
+    uint64_t* av_empty = av_full + AV_STAGES;   // AV: arrived by the leader's multicast commit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(av_empty + AV_STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     uint32_t* sink = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // D_STAGES words the peer's stage signals land in
 
@@ -524,6 +578,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 2 * 4);
+        }
+        if constexpr (AV) {
+            for (int i = 0; i < AV_STAGES; ++i) {
+                mbar_init(&av_full[i], 1);
+                mbar_init(&av_empty[i], 1);
+            }
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -549,11 +609,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             RingPos<P_STAGES> ps;
-            int issued = 0;
+            RingPos<AV_STAGES> as;
+            int issued = 0, issued_av = 0;
             bool ok = !p.starve;  // a starved launch loads nothing: every consumer's wait runs out
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-                const int m0 = (tile % p.num_m) * TM + (int)rank * HM;
-                const int n0 = (tile / p.num_m) * TN + (int)rank * HN;
+                int mt, nt;
+                tile_mn(p, tile, mt, nt);
+                const int m0 = mt * TM + (int)rank * HM;
+                const int n0 = nt * TN + (int)rank * HN;
                 for (int kb = 0; kb < p.KB; ++kb) {
                     if (!wait_or_abort<false>(&pk_empty[ps.idx], ps.phase ^ 1u, abort_flag)) {
                         ok = false;
@@ -561,10 +624,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     }
                     mbar_arrive_expect_tx(&pk_full[ps.idx], PK_STAGE);
                     uint8_t* dst = pk + ps.idx * PK_STAGE;
-                    tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA, F8), m0, &pk_full[ps.idx]);
+                    if constexpr (!AV) tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA, F8), m0, &pk_full[ps.idx]);
                     tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW, F8), n0, &pk_full[ps.idx]);
                     ++issued;
                     ps.advance();
+                    if constexpr (AV) {
+                        // A's values for this K step: one 128-byte row per A row,
+                        // landed by the TMA in the swizzled layout the MMA reads
+                        if (!wait_or_abort<false>(&av_empty[as.idx], as.phase ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&av_full[as.idx], DEC_A);
+                        tma_load_2d(av + as.idx * DEC_A, &p.tmA, kb * 128, m0, &av_full[as.idx]);
+                        ++issued_av;
+                        as.advance();
+                    }
                 }
             }
             // the loads this thread issued must land before shared memory goes away
@@ -572,11 +647,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 const int st = issued - k;
                 mbar_wait_bounded(&pk_full[st % P_STAGES], (uint32_t)(st / P_STAGES) & 1u);
             }
+            for (int k = 1; k <= AV_STAGES && k <= issued_av; ++k) {
+                const int st = issued_av - k;
+                mbar_wait_bounded(&av_full[st % AV_STAGES], (uint32_t)(st / AV_STAGES) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer (leader) -----------------------
         if (leader && lane == 0) {
             RingPos<D_STAGES> ds;
+            RingPos<AV_STAGES> as;
             int acc_it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++acc_it) {
@@ -590,13 +670,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(dec + ds.idx * DEC_STAGE), b_base = a_base + DEC_A;
+                    // (AV: the stage's "full" signal also covers A's values in both CTAs,
+                    // since each CTA's decoders publish only after their A load landed)
+                    const uint32_t a_base = AV ? smem_u32(av + as.idx * DEC_A) : smem_u32(dec + ds.idx * DSTAGE);
+                    const uint32_t b_base = smem_u32(dec + ds.idx * DSTAGE) + DOFF_B;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)  // 32 bytes of each 128-byte row per MMA
                         tc_mma_pair<F8>(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k),
                                         F8 ? kIdescE4m3 : kIdescBf16,
                                     (kb | k) != 0 ? 1u : 0u);
                     tc_commit_pair(&dec_empty[ds.idx]);
+                    if constexpr (AV) {
+                        tc_commit_pair(&av_empty[as.idx]);
+                        as.advance();
+                    }
                     ds.advance();
                 }
                 if (ok) tc_commit_pair(&acc_full[a]);
@@ -621,10 +708,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t tab_w[4] = {p.tab_w[0], p.tab_w[1], p.tab_w[2], p.tab_w[3]};
         const uint32_t dec_full_leader = map_to_rank(&dec_full[0], 0);
         const uint32_t sink_leader = map_to_rank(&sink[0], 0);
-        // publish decoded stage `slot` to the leader's MMA issuer
-        auto publish = [&](int slot) {
+        // publish decoded stage `slot` to the leader's MMA issuer; with A
+        // given as values the group's lead first waits (bounded) for this
+        // CTA's A load of the same step, so the leader's "full" signal covers
+        // it.  Returns false if that wait gave up.
+        auto publish = [&](int slot, int aslot, uint32_t aphase) -> bool {
             fence_proxy_async_smem();
             __syncwarp();
+            int landed = 1;
+            if constexpr (AV) {
+                if (lane == 0 && grp_lead) landed = wait_or_abort<true>(&av_full[aslot], aphase, abort_flag) ? 1 : 0;
+                landed = __shfl_sync(0xffffffffu, landed, 0);
+                if (!landed) return false;
+            }
             if (lane == 0) {
                 if (leader) {
                     if (grp_lead) mbar_arrive_expect_tx(&dec_full[slot], 4 * GROUP_WARPS);  // the peer's share
@@ -634,21 +730,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                                          dec_full_leader + 8u * (uint32_t)slot);
                 }
             }
+            return true;
         };
         const int my_tiles = pair < p.num_tiles ? (p.num_tiles - 1 - pair) / npairs + 1 : 0;
         const int total = my_tiles * p.KB;
         RingPos<P_STAGES> ps;
         RingPos<D_STAGES> ds;
+        RingPos<AV_STAGES> as;  // A-values slot of the step (AV)
         ps.idx = grp;
         ds.idx = grp;
+        as.idx = grp;
         int pending = -1;  // decoded slot stored but not yet published
+        int pend_as = 0;   // and its A-values slot and phase
+        uint32_t pend_ap = 0;
         // A packed slot is released as soon as its codes are in registers
         // (the arrive's release orders the loads before it), so each slot is
         // held for about one step of the group.
         StageCodes<BA, BW, F8> cur;
         bool ok = grp < total && wait_or_abort<false>(&pk_full[ps.idx], 0u, abort_flag);
         if (ok) {
-            load_codes<BA, BW, F8>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+            load_codes<BA, BW, F8, AV>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
             __syncwarp();
             if (lane == 0) mbar_arrive(&pk_empty[ps.idx]);
         }
@@ -662,24 +763,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 const uint8_t* pa = pk + ps.idx * PK_STAGE;
-                load_codes<BA, BW, F8>(nxt, pa, pa + PKA, srcA, srcB);
+                load_codes<BA, BW, F8, AV>(nxt, pa, pa + PKA, srcA, srcB);
             }
             StageValues v;
-            decode_codes<BA, BW, F8>(v, cur, tab_a, tab_w);
+            decode_codes<BA, BW, F8, AV>(v, cur, tab_a, tab_w);
             __syncwarp();
             if (lane == 0 && more) mbar_arrive(&pk_empty[ps.idx]);  // the next step's codes are in registers
-            if (pending >= 0) publish(pending);
+            if (pending >= 0 && !publish(pending, pend_as, pend_ap)) {
+                ok = false;
+                break;
+            }
             if (!wait_or_abort<false>(&dec_empty[ds.idx], ds.phase ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
-            uint8_t* da = dec + ds.idx * DEC_STAGE;
-            store_values(v, da, da + DEC_A, dst_off);
+            uint8_t* da = dec + ds.idx * DSTAGE;
+            store_values<AV>(v, da, da + DOFF_B, dst_off);
             pending = ds.idx;
+            pend_as = as.idx;
+            pend_ap = as.phase;
             ds.advance(NGROUPS);
+            if constexpr (AV) as.advance(NGROUPS);
             cur = nxt;
         }
-        if (ok && pending >= 0) publish(pending);
+        if (ok && pending >= 0) publish(pending, pend_as, pend_ap);
     } else {
         // ------------------------------ epilogue ----------------------------------
         // Per tile: stage r (and bias) of the tile's 256 columns in shared
@@ -692,7 +799,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const bool vec_ok = (p.N & 7) == 0;  // rows of y 16-byte aligned
         int acc_it = 0;
         for (int tile = pair; tile < p.num_tiles; tile += npairs, ++acc_it) {
-            const int m0 = (tile % p.num_m) * TM + (int)rank * HM, n0 = (tile / p.num_m) * TN;
+            int mt, nt;
+            tile_mn(p, tile, mt, nt);
+            const int m0 = mt * TM + (int)rank * HM, n0 = nt * TN;
             const int a = acc_it & 1;
             if (!wait_or_abort<false>(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
             tc_fence_after();
@@ -782,7 +891,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows) {
+bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows,
+               bool swizzle128 = false) {
     auto fn = get_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
@@ -790,7 +900,8 @@ bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int b
     cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -835,10 +946,10 @@ void fill_tables_e4m3(int bits, const uint8_t* e, uint32_t tab[4], uint8_t* c6) 
     }
 }
 
-template <int BA, int BW, bool F8>
+template <int BA, int BW, bool F8, bool AV = false>
 cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
-    auto k = qgemm_kernel<BA, BW, F8>;
-    const int smem = smem_bytes(BA, BW, F8);
+    auto k = qgemm_kernel<BA, BW, F8, AV>;
+    const int smem = smem_bytes(BA, BW, F8, AV);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k<<<grid, NTHREADS, smem, stream>>>(prm);
@@ -847,6 +958,14 @@ cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
 
 template <bool F8>
 cudaError_t launch_bits(const QgemmArgs& a, QgemmParams& prm, int grid, cudaStream_t stream) {
+    if (a.a_val) {  // A given as values: only W's width selects the kernel
+        if (a.bits_w == 4) return launch_qgemm_t<0, 4, F8, true>(prm, grid, stream);
+        if (a.bits_w == 2) return launch_qgemm_t<0, 2, F8, true>(prm, grid, stream);
+        if (a.bits_w == 6) return launch_qgemm_t<0, 6, F8, true>(prm, grid, stream);
+        if constexpr (F8)
+            if (a.bits_w == 3) return launch_qgemm_t<0, 3, true, true>(prm, grid, stream);
+        return cudaErrorInvalidValue;
+    }
     if constexpr (F8) {  // 3-bit codes: the fp8 variant only
         if (a.bits_a == 3 && a.bits_w == 3) return launch_qgemm_t<3, 3, true>(prm, grid, stream);
         if (a.bits_a == 3 && a.bits_w == 4) return launch_qgemm_t<3, 4, true>(prm, grid, stream);
@@ -883,14 +1002,24 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     std::memset(&prm, 0, sizeof(prm));
     const bool f8 = a.fp8;
     if (a.K % bk_codes(f8) != 0) return cudaErrorInvalidValue;
-    if (!make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8, pk_row_bytes(a.bits_a, f8), HM) ||
+    // A: packed codes, or (a_val) values whose 128-byte K step rows the TMA
+    // lands directly in the MMA's 128-byte-swizzled layout
+    const bool tm_ok = a.a_val ? make_tmap(&prm.tmA, a.a_val, a.M, a.K * (f8 ? 1 : 2), 128, HM, true)
+                               : make_tmap(&prm.tmA, a.a_idx, a.M, a.bits_a == 6 ? a.K : a.K * a.bits_a / 8,
+                                           pk_row_bytes(a.bits_a, f8), HM);
+    if (!tm_ok ||
         !make_tmap(&prm.tmB, a.w_idx, a.N, a.bits_w == 6 ? a.K : a.K * a.bits_w / 8, pk_row_bytes(a.bits_w, f8), HN))
         return cudaErrorInvalidValue;
     prm.M = a.M;
     prm.N = a.N;
     prm.KB = a.K / bk_codes(f8);
     prm.num_m = (a.M + TM - 1) / TM;
-    prm.num_tiles = prm.num_m * ((a.N + TN - 1) / TN);
+    prm.num_n = (a.N + TN - 1) / TN;
+    prm.num_tiles = prm.num_m * prm.num_n;
+    // A's values are 2 (e4m3: 1) bytes per element, more than L2 holds at the
+    // larger shapes: N-fastest order keeps the few A tiles in use resident
+    // while the (small) packed W cycles.  Packed A is small: M-fastest.
+    prm.n_fastest = a.a_val ? 1 : 0;
     prm.s = a.s;
     prm.w_r = a.w_r;
     prm.bias = a.bias;
@@ -898,11 +1027,11 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     prm.starve = a.starve ? 1 : 0;
     if (f8) {
         prm.out_scale = (float)(1.0 / (double)a.K);  // both operands' centroids carry sqrt(d)
-        fill_tables_e4m3(a.bits_a, a.ca_e4m3, prm.tab_a, prm.c6a8);
+        if (!a.a_val) fill_tables_e4m3(a.bits_a, a.ca_e4m3, prm.tab_a, prm.c6a8);
         fill_tables_e4m3(a.bits_w, a.cw_e4m3, prm.tab_w, prm.c6w8);
     } else {
         prm.out_scale = 1.0f;
-        fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
+        if (!a.a_val) fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
         fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
     }
     const int pairs_max = qgemm_sm_count() / 2;

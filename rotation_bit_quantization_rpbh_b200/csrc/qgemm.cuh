@@ -20,6 +20,7 @@ struct QgemmArgs {
     bool fp8;                // e4m3 variant: centroids c_j sqrt(d) as e4m3, K % 128 == 0
     const uint8_t* ca_e4m3;  // activation centroids (fp8 variant)
     const uint8_t* cw_e4m3;  // weight centroids (fp8 variant)
+    const void* a_val = nullptr;  // instead of a_idx: A as centroid values [M, K] (bf16, or e4m3 in the fp8 variant)
     bool starve = false;     // test hook: the producer issues no loads (the waits run out)
 };
 

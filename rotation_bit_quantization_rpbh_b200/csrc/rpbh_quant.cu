@@ -29,7 +29,11 @@
 //   - rows whose norm is not finite or exceeds FLT_MAX / (2 sqrt(h)) (where
 //     the fp32 butterfly could overflow) take the middle cell;
 //   - indices are packed LSB-first and written 16 bytes at a time as they
-//     are produced.
+//     are produced;
+//   - in the value modes the table entry holds, instead of the count, the
+//     centroid values of the bin's two possible cells (bf16 or e4m3 of
+//     c sqrt(d)), so the same compare selects C[index] itself, written as
+//     bf16 pairs or e4m3 quads, 16 bytes at a time.
 #include <cuda_bf16.h>
 
 #include "device_util.cuh"
@@ -57,6 +61,12 @@ __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     L.bar = align_up(L.red + p.NG * (p.G / 32) * p.R * 4, 8);
     L.total = L.bar + 8 * (2 * p.NG + 1);
     return L;
+}
+
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
 __device__ __forceinline__ void group_sync(int id, int count) {
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
 
         if (valid) {
             if (b == 0) {
-                if constexpr (MODE == 0) p.s_out[row] = s;
+                if constexpr (MODE == 0 || MODE >= 3) p.s_out[row] = s;
                 if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
                 if constexpr (MODE == 2) p.norm_out[row] = s;
             }
@@ -231,6 +241,56 @@ __global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) 
                 for (int j = 0; j < L2H; j += 2) {
                     const float2 a = f2mul(v2[j], sc), c = f2mul(v2[j + 1], sc);
                     yo[j >> 1] = make_float4(a.x, a.y, c.x, c.y);
+                }
+            } else if constexpr (MODE >= 3) {
+                // ---- A5 with the centroid values written instead of the codes:
+                // the table entry holds the values of both cells its bin can
+                // give (the cell below the bin's threshold and the one above),
+                // so one compare selects c_index directly ----------------------
+                constexpr int VB = MODE == 3 ? 2 : 1;  // bytes per value: bf16, or e4m3
+                uint4* dst = reinterpret_cast<uint4*>(p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * H * VB);
+                if (s <= p.s_max) {
+                    const float inv = p.rsqrt_h / (s + p.eps);
+                    const float2 inv2 = make_float2(inv, inv);
+                    // table word of element pair j and the selector bits of its two values
+                    auto pick = [&](int j, uint32_t& val0, uint32_t& val1, uint32_t& ge0, uint32_t& ge1) {
+                        const float2 q = f2mul(v2[j], inv2);
+                        const float2 z = f2fma(q, G2, M2);
+                        float T0, T1;
+                        const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
+                        const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
+                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(val0) : "r"(a0));
+                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(val1) : "r"(a1));
+                        ge0 = q.x >= T0 ? 1u : 0u;
+                        ge1 = q.y >= T1 ? 1u : 0u;
+                    };
+#pragma unroll
+                    for (int w0 = 0; w0 < H * VB / 4; w0 += 4) {
+                        uint32_t words[4];
+#pragma unroll
+                        for (int wj = 0; wj < 4; ++wj) {
+                            if constexpr (VB == 2) {
+                                // bf16 pair: (lo or hi half of entry 0, lo or hi half of entry 1)
+                                uint32_t val0, val1, ge0, ge1;
+                                pick(w0 + wj, val0, val1, ge0, ge1);
+                                words[wj] = prmt_b32(val0, val1, 0x5410u + ge0 * 0x22u + ge1 * 0x2200u);
+                            } else {
+                                // four e4m3 bytes: byte 0 or 1 of each entry's value word
+                                uint32_t val0, val1, val2, val3, ge0, ge1, ge2, ge3;
+                                pick(2 * (w0 + wj), val0, val1, ge0, ge1);
+                                pick(2 * (w0 + wj) + 1, val2, val3, ge2, ge3);
+                                const uint32_t lo = prmt_b32(val0, val1, 0x40u + ge0 + ge1 * 0x10u);
+                                const uint32_t hi = prmt_b32(val2, val3, 0x40u + ge2 + ge3 * 0x10u);
+                                words[wj] = prmt_b32(lo, hi, 0x5410u);
+                            }
+                        }
+                        dst[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
+                    }
+                } else {
+                    // the middle cell's value everywhere (see the codes branch)
+                    const uint32_t wm = VB == 2 ? p.mid_val * 0x10001u : p.mid_val * 0x01010101u;
+#pragma unroll
+                    for (int w0 = 0; w0 < H * VB / 4; w0 += 4) dst[w0 >> 2] = make_uint4(wm, wm, wm, wm);
                 }
             } else {
                 // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
@@ -359,15 +419,20 @@ cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
 
 template <typename InT, int H, int MODE>
 cudaError_t launch_bits(const RpbhParams& p, int bits, int grid, cudaStream_t stream) {
-    switch (bits) {
-        case 2: return launch_rpbh_t<InT, H, 2, MODE>(p, grid, stream);
-        case 3:
-            if constexpr (H >= 32) return launch_rpbh_t<InT, H, 3, MODE>(p, grid, stream);
-            return cudaErrorInvalidValue;
-        case 4: return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
-        case 6: return launch_rpbh_t<InT, H, 6, MODE>(p, grid, stream);
+    // the rotation alone and the value outputs do not depend on the code width
+    if constexpr (MODE >= 2) {
+        return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
+    } else {
+        switch (bits) {
+            case 2: return launch_rpbh_t<InT, H, 2, MODE>(p, grid, stream);
+            case 3:
+                if constexpr (H >= 32) return launch_rpbh_t<InT, H, 3, MODE>(p, grid, stream);
+                return cudaErrorInvalidValue;
+            case 4: return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
+            case 6: return launch_rpbh_t<InT, H, 6, MODE>(p, grid, stream);
+        }
+        return cudaErrorInvalidValue;
     }
-    return cudaErrorInvalidValue;
 }
 
 template <typename InT, int MODE>
@@ -390,10 +455,14 @@ cudaError_t launch_rpbh_quant(const RpbhParams& p, bool in_bf16, int h, int bits
     if (in_bf16) {
         if (mode == 0) return launch_h<__nv_bfloat16, 0>(p, h, bits, grid, stream);
         if (mode == 1) return launch_h<__nv_bfloat16, 1>(p, h, bits, grid, stream);
+        if (mode == 3) return launch_h<__nv_bfloat16, 3>(p, h, bits, grid, stream);
+        if (mode == 4) return launch_h<__nv_bfloat16, 4>(p, h, bits, grid, stream);
         return launch_h<__nv_bfloat16, 2>(p, h, 4, grid, stream);
     }
     if (mode == 0) return launch_h<float, 0>(p, h, bits, grid, stream);
     if (mode == 1) return launch_h<float, 1>(p, h, bits, grid, stream);
+    if (mode == 3) return launch_h<float, 3>(p, h, bits, grid, stream);
+    if (mode == 4) return launch_h<float, 4>(p, h, bits, grid, stream);
     return launch_h<float, 2>(p, h, 4, grid, stream);
 }
 

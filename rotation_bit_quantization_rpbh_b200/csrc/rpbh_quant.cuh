@@ -29,13 +29,15 @@ struct RpbhParams {
     float eps;             // the split's eps
     float s_max;           // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
     int starve;            // test hook: issue no row copies (the waits run out)
+    uint32_t mid_val;      // value outputs: the middle cell's value (bf16 bits or e4m3 byte)
 };
 
 constexpr int kMaxGroups = 3;  // warp groups per CTA (at most 128 threads each)
 
 int rpbh_smem_bytes(const RpbhParams& p);
 
-// mode 0: activations (s fp32), 1: weights (r bf16), 2: rotation only (x', norm)
+// mode 0: activations (s fp32), 1: weights (r bf16), 2: rotation only (x', norm),
+// 3 / 4: activations as centroid values, bf16 / e4m3 of c sqrt(d) (s fp32)
 cudaError_t launch_rpbh_quant(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
                               cudaStream_t stream);
 

@@ -93,10 +93,16 @@ def test_starved_weight_quantizer_times_out_and_context_survives(layer):
     assert B.device_status() == 0
 
 
-@pytest.mark.parametrize("fp8", [False, True])
-def test_starved_gemm_times_out_and_context_survives(layer, fp8):
+@pytest.mark.parametrize("fp8,values", [(False, False), (True, False), (False, True), (True, True)])
+def test_starved_gemm_times_out_and_context_survives(layer, fp8, values):
     L = layer
-    run = B.qgemm_fp8 if fp8 else B.qgemm
+    if values:
+        v, _ = B.quantize_acts_values(L["plan"], L["cb4"], L["x"], fp8=fp8)
+
+        def run(cb_a, cb_w, idx, s, w_idx, w_r):
+            return B.qgemm_values(cb_w, v, s, w_idx, w_r, fp8=fp8)
+    else:
+        run = B.qgemm_fp8 if fp8 else B.qgemm
     ref = run(L["cb4"], L["cb2"], L["idx"], L["s"], L["w_idx"], L["w_r"])
     torch.cuda.synchronize()
     assert B.device_status() == 0

@@ -42,6 +42,7 @@ def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_i
     assert B.device_status() == 0
     # the one-call layer is the two calls it is made of
     assert torch.equal(y, y2)
+    _check_values_schedule(dev, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, bias_t, y, ba, bw, fp8=False)
 
     rows_a = np.arange(M) if full_check else np.sort(rng.choice(M, min(M, n_rows_idx), replace=False))
     rows_w = np.arange(N) if full_check else np.sort(rng.choice(N, min(N, n_rows_idx), replace=False))
@@ -77,6 +78,28 @@ def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_i
         err = max(rel_frob(yg[rr], ref_r), rel_frob(yg[:, cc], ref_c))
         assert err <= GEMM_TOL, err
     return {"band_a": nb_a, "band_w": nb_w, "r_ulp": n_ulp, "gemm_rel": err}
+
+
+def _check_values_schedule(dev, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, bias_t, y, ba, bw, fp8):
+    """The values schedule against the codes one: the quantiser's values are
+    the codebook's values at the codes' indices (same norms), and the product
+    from those values equals the product from the codes bit for bit."""
+    d = xg.shape[1]
+    val, s_v = B.quantize_acts_values(plan, cb_a, xg, fp8=fp8)
+    u = B.unpack_indices(a_idx, d, ba).long()
+    if fp8:
+        tab = torch.from_numpy(cb_a.e4m3_bytes()).to(dev)
+        assert torch.equal(val, tab[u])
+    else:
+        tab = torch.from_numpy(cb_a.bf16_bits().view(np.int16)).to(dev)
+        assert torch.equal(val.view(torch.int16), tab[u])
+    assert torch.equal(s_v, s)
+    if bw == 3 and not fp8:
+        return
+    y3 = B.qgemm_values(cb_w, val, s_v, w_idx, w_r, bias=bias_t, fp8=fp8)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert torch.equal(y3, y)
 
 
 # multi-tile cases with ragged edges, checked in full
@@ -166,6 +189,8 @@ def test_fp8_variant_matches_oracle_on_e4m3_centroids(cuda_device, case):
     y = B.qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=bias_t)
     torch.cuda.synchronize()
     assert B.device_status() == 0
+    _check_values_schedule(cuda_device, plan, cb_a, cb_w, x.to(cuda_device), a_idx, s, w_idx, w_r, bias_t, y, ba, bw,
+                           fp8=True)
     ca = _e4m3_values(oracle.codebook(d, ba)[0], d)
     cw = _e4m3_values(oracle.codebook(d, bw)[0], d)
     ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
@@ -203,6 +228,8 @@ def test_fp8_variant_full_size_flux_qkv_sample(cuda_device):
     a_idx, s = B.quantize_acts(plan, cb_a, x.to(cuda_device))
     y = B.qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r)
     torch.cuda.synchronize()
+    _check_values_schedule(cuda_device, plan, cb_a, cb_w, x.to(cuda_device), a_idx, s, w_idx, w_r, None, y,
+                           w.bits_a, w.bits_w, fp8=True)
     rng = np.random.default_rng(5)
     rows = np.sort(rng.choice(w.M, 128, replace=False))
     cols = np.sort(rng.choice(w.N, 256, replace=False))
@@ -258,6 +285,26 @@ def test_three_bit_fp8_product_matches_oracle(cuda_device, bw, ba):
     ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
                          w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw)
     assert rel_frob(y.float().cpu().numpy().astype(np.float64), ref) <= GEMM_TOL
+
+
+def test_values_schedule_limits_are_reported(cuda_device):
+    cb3 = B.codebook(256, 3)
+    val = torch.zeros((8, 256), dtype=torch.bfloat16, device=cuda_device)
+    s = torch.ones(8, device=cuda_device)
+    w_idx = torch.zeros((16, 96), dtype=torch.uint8, device=cuda_device)
+    w_r = torch.ones(16, dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(B.OQError) as e:  # 3-bit weights: the fp8 product only
+        B.qgemm_values(cb3, val, s, w_idx, w_r)
+    assert e.value.status == 2
+    plan = B.rpbh_plan(192, 64, 3)
+    with pytest.raises(B.OQError) as e:  # e4m3 values need d % 128 == 0
+        B.quantize_acts_values(plan, B.codebook(192, 4), torch.zeros((4, 192), device=cuda_device), fp8=True)
+    assert e.value.status == 2
+    bad = torch.zeros(8 * 256 + 8, dtype=torch.bfloat16, device=cuda_device)[1:1 + 8 * 256].view(8, 256)
+    w4 = torch.zeros((16, 128), dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(B.OQError) as e:  # values not 16-byte aligned
+        B.qgemm_values(B.codebook(256, 4), bad, s, w4, w_r)
+    assert e.value.status == 3
 
 
 def test_three_bit_limits_are_reported(cuda_device):
