@@ -33,6 +33,8 @@
  *     bits = 4: two indices per byte (index k in bits 4*(k%2) of byte k/2);
  *     bits = 2: four per byte (bits 2*(k%4) of byte k/4);
  *     bits = 6: one index per byte (low 6 bits);
+ *     bits = 8: one index per byte (activations and weights are quantised;
+ *               the products take 8-bit activations as values only);
  *     bits = 3: a bit stream, index k in bits 3k..3k+2 of the row (eight
  *               indices per three bytes); needs h >= 32 and d % 128 == 0,
  *               and runs through the fp8 product variant only.
@@ -52,7 +54,7 @@ extern "C" {
 typedef enum {
     OQ_OK = 0,
     OQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, mismatched handles */
-    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,3,4,6}, d % 64 != 0 */
+    OQ_ERR_UNSUPPORTED = 2, /* d % h != 0, h not a power of two in [16, 128], bits not in {2,3,4,6,8}, d % 64 != 0 */
     OQ_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned */
     OQ_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
     OQ_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see oq_device_status) */
@@ -78,7 +80,8 @@ const char* oq_status_str(oq_status s);
 /* masses from the regularised incomplete beta function), then derives the */
 /* fp32 thresholds, bf16 centroids and the quantiser lookup table the      */
 /* kernels use.  Host-only: needs no GPU.                                  */
-/*   d    >= 3;  bits in {1..6} (the quantising calls accept {2, 4, 6}).   */
+/*   d    >= 3;  bits in {1..8} (the quantising calls accept               */
+/*   {2, 3, 4, 6, 8}).                                                     */
 /*   out  receives a library-owned handle (free with oq_codebook_free).    */
 oq_status oq_codebook(int d, int bits, oq_codebook_t** out);
 
@@ -167,7 +170,7 @@ oq_status oq_quantize_acts(const oq_plan_t* plan, const oq_codebook_t* cb_a, con
 /*           the product uses), row-major.                                 */
 /* The _fp8 form writes the e4m3 bytes of c sqrt(d) that oq_qgemm_fp8      */
 /* decodes to (oq_codebook_fp8); it needs d % 128 == 0.  Any bits in       */
-/* {2, 3, 4, 6}.  Used by the values schedule of oq_qlinear.               */
+/* {2, 3, 4, 6, 8}.  Used by the values schedule of oq_qlinear.            */
 oq_status oq_quantize_acts_values(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
                                   int M, uint16_t* val_out, float* s_out, void* stream);
 oq_status oq_quantize_acts_values_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const void* x, oq_dtype dtype,
@@ -186,7 +189,9 @@ oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, in
 /*   a_idx   device, [M, d*ba/8] packed activation indices; s device [M] f32. */
 /*   w_idx   device, [N, d*bw/8] packed weight indices; w_r device [N] bf16. */
 /*   bias    device [N] bf16 or NULL.   y device [M, N] bf16.              */
-/*   d % 64 == 0; bits_w, bits_a in {2, 4, 6}.  M >= 0, N > 0.              */
+/*   d % 64 == 0; bits_w, bits_a in {2, 4, 6} (8-bit codes: no in-kernel  */
+/*   decoder, OQ_ERR_UNSUPPORTED; 8-bit activations take the values        */
+/*   schedule).  M >= 0, N > 0.                                            */
 oq_status oq_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
                    const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                    void* stream);

@@ -46,9 +46,9 @@ static bool device_alloc(void** ptr, size_t bytes) {
 // true (once) if the next launch of `kernel` is to be starved
 bool take_starve(int kernel) { return (g_starve_mask.fetch_and(~kernel) & kernel) != 0; }
 
-bool quant_bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 6; }
+bool quant_bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 6 || bits == 8; }
 
-int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }
+int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }  // 8: one byte per code too
 
 // Launch the fused rotate/quantise kernel in one of its modes: 0 activation
 // codes, 1 weight codes, 2 rotation only, 3 / 4 activation values (bf16 /
@@ -188,7 +188,7 @@ const char* oq_status_str(oq_status s) {
 oq_status oq_codebook(int d, int bits, oq_codebook_t** out) {
     if (!out) return OQ_ERR_INVALID_ARG;
     *out = nullptr;
-    if (d < 3 || bits < 1 || bits > 6) return OQ_ERR_UNSUPPORTED;
+    if (d < 3 || bits < 1 || bits > 8) return OQ_ERR_UNSUPPORTED;
     oq_codebook_t* cb = new (std::nothrow) oq_codebook_s();
     if (!cb) return OQ_ERR_OOM;
     oq_status s = build_codebook(d, bits, cb);
@@ -347,6 +347,8 @@ static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
         return OQ_ERR_UNSUPPORTED;
     // 3-bit rows hold 24 bytes per 64 codes, too narrow for the bf16 kernel's TMA step
     if (!fp8 && (cb_a->bits == 3 || cb_w->bits == 3)) return OQ_ERR_UNSUPPORTED;
+    // 8-bit codes have no in-kernel decoder: 8-bit activations run in the values schedule
+    if (cb_a->bits == 8 || cb_w->bits == 8) return OQ_ERR_UNSUPPORTED;
     if (fp8 && (cb_a->bits == 3 || cb_w->bits == 3) && !((cb_a->bits == 3 || cb_a->bits == 4) && (cb_w->bits == 3 || cb_w->bits == 4)))
         return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;  // an empty batch: activation and output buffers may be null
@@ -382,7 +384,7 @@ static oq_status run_qgemm_values(const oq_codebook_t* cb_w, int M, int N, const
                                   void* stream, bool fp8) {
     if (!cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (!quant_bits_ok(cb_w->bits) || cb_w->d % (fp8 ? 128 : 64) != 0) return OQ_ERR_UNSUPPORTED;
-    if (!fp8 && cb_w->bits == 3) return OQ_ERR_UNSUPPORTED;
+    if ((!fp8 && cb_w->bits == 3) || cb_w->bits == 8) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
     if (!a_val || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
     if (!aligned16(a_val) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||

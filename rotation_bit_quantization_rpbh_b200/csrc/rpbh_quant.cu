@@ -430,6 +430,7 @@ cudaError_t launch_bits(const RpbhParams& p, int bits, int grid, cudaStream_t st
                 return cudaErrorInvalidValue;
             case 4: return launch_rpbh_t<InT, H, 4, MODE>(p, grid, stream);
             case 6: return launch_rpbh_t<InT, H, 6, MODE>(p, grid, stream);
+            case 8: return launch_rpbh_t<InT, H, 8, MODE>(p, grid, stream);
         }
         return cudaErrorInvalidValue;
     }

@@ -36,7 +36,7 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("d,bits", [(256, 4), (3072, 4), (12288, 4), (4096, 2), (4096, 4), (1536, 4), (1536, 6),
-                                    (64, 2), (64, 4), (64, 6), (512, 2), (8, 2), (3072, 3), (128, 3)])
+                                    (64, 2), (64, 4), (64, 6), (512, 2), (8, 2), (3072, 3), (128, 3), (256, 8)])
 def test_library_codebook_matches_oracle(d, bits):
     """Two independent solvers (library: Newton on the Lloyd-Max conditions
     with incomplete-beta cell masses; oracle: Lloyd iteration with
@@ -101,7 +101,7 @@ def test_argument_checks_on_host_calls():
     import ctypes
 
     h = ctypes.c_void_p()
-    assert L.oq_codebook(256, 7, ctypes.byref(h)) == 2  # UNSUPPORTED
+    assert L.oq_codebook(256, 9, ctypes.byref(h)) == 2  # UNSUPPORTED
     assert L.oq_codebook(2, 4, ctypes.byref(h)) == 2
     assert L.oq_codebook(256, 4, None) == 1  # INVALID_ARG
     perm = np.zeros(300, dtype=np.int32)
@@ -144,6 +144,9 @@ def test_workspace_size():
     ws3 = B.qlinear_workspace(10, 1536, 3)  # 3-bit: 8 codes per 3 bytes
     assert ws3 >= 10 * 1536 * 3 // 8 + 10 * 4 and ws3 % 256 == 0
     assert B.qlinear_workspace(10, 1536, 5) == 0
+    assert B.qlinear_workspace(10, 1536, 8) >= 10 * 1536 + 10 * 4  # 8-bit: one byte per code
+    wv = B.qlinear_workspace_values(4096, 3072)
+    assert wv >= 4096 * 3072 * 2 + 4096 * 4 and wv % 256 == 0
 
 
 def test_unpack_layout():

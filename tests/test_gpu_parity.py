@@ -320,3 +320,46 @@ def test_three_bit_limits_are_reported(cuda_device):
     with pytest.raises(B.OQError) as e:  # the bf16 kernel's 64-code step is 24 bytes of 3-bit codes
         B.qgemm(cb, cb, a_idx, s, w_idx, w_r)
     assert e.value.status == 2
+
+
+def test_eight_bit_activations_match_oracle(cuda_device):
+    """8-bit activation codes (one byte each) against the oracle, then the W4A8
+    layer, which runs in the values schedule (the codes product has no 8-bit
+    decoder), against the oracle's product on the same indices: bf16 and fp8."""
+    M, d, N, h, seed = 300, 256, 264, 64, 61
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, h, seed)
+    perm, sign = oracle.plan(d, h, seed)
+    cb_a, cb_w = B.codebook(d, 8), B.codebook(d, 4)
+    ocb_a, ocb_w = oracle.codebook(d, 8), oracle.codebook(d, 4)
+    xg = x.to(cuda_device)
+    a_idx, s = B.quantize_acts(plan, cb_a, xg)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert a_idx.shape == (M, d)
+    check_quantized_rows(a_idx, s, x, np.arange(M), h, perm, sign, cb_a, ocb_a, "acts")
+    with pytest.raises(B.OQError) as e:
+        B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r)
+    assert e.value.status == 2  # no in-kernel 8-bit decoder
+    with pytest.raises(B.OQError) as e:  # a codes-sized workspace leaves only the codes schedule
+        B.qlinear(plan, cb_a, cb_w, xg, w_idx, w_r, schedule="codes")
+    assert e.value.status == 2
+
+    ia = B.unpack_indices(a_idx, d, 8).cpu().numpy()
+    iw = B.unpack_indices(w_idx, d, 4).cpu().numpy()
+    s64 = s.cpu().numpy().astype(np.float64)
+    r64 = w_r.cpu().to(torch.float32).numpy().astype(np.float64)
+    for fp8 in (False, True):
+        y = B.qlinear(plan, cb_a, cb_w, xg, w_idx, w_r, fp8=fp8)
+        torch.cuda.synchronize()
+        assert B.device_status() == 0
+        _check_values_schedule(cuda_device, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, None, y, 8, 4, fp8=fp8)
+        if fp8:
+            ca, cw = _e4m3_values(ocb_a[0], d), _e4m3_values(ocb_w[0], d)
+        else:
+            ca, cw = oracle.round_bf16(ocb_a[0])[1], oracle.round_bf16(ocb_w[0])[1]
+        ref = gemm_reference(ia, s64, iw, r64, ca, cw)
+        assert rel_frob(y.float().cpu().numpy().astype(np.float64), ref) <= GEMM_TOL

@@ -19,7 +19,7 @@ import oracle
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 # (d, bits) pairs the five workloads need (activation and weight codebooks)
-CONFIG_CODEBOOKS = [(256, 4), (3072, 4), (12288, 4), (4096, 2), (4096, 4), (1536, 4), (1536, 6)]
+CONFIG_CODEBOOKS = [(256, 4), (3072, 4), (12288, 4), (4096, 2), (4096, 4), (1536, 4), (1536, 6), (256, 8)]
 
 
 # --------------------------------------------------------------------------
@@ -322,13 +322,13 @@ def test_permutation_makes_every_coordinate_variance_one_over_d():
 # --------------------------------------------------------------------------
 # quantiser
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("bits", [2, 4, 6])
-def test_threshold_count_is_the_nearest_centroid(bits):
-    """Brute force at d = 64 on 1e5 coordinates of random unit directions."""
-    d, h = 64, 64
+@pytest.mark.parametrize("d,bits", [(64, 2), (64, 4), (64, 6), (256, 8)])
+def test_threshold_count_is_the_nearest_centroid(d, bits):
+    """Brute force on 1e5 coordinates of random unit directions."""
+    h = 64
     c, t = oracle.codebook(d, bits)
     perm, sign = oracle.plan(d, h, 1)
-    x = np.random.default_rng(bits).standard_normal((1563, d))
+    x = np.random.default_rng(bits).standard_normal((100_032 // d, d))
     out = oracle.quantize_rows(x, h, perm, sign, t, decision=64, want_v=True)
     v = out["v"]
     brute = np.argmin(np.abs(v[..., None] - c[None, None, :]), axis=-1)
