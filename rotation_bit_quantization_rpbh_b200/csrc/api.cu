@@ -100,9 +100,9 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.G = (nb * R + 31) / 32 * 32;
     if (p.G > 128) return OQ_ERR_UNSUPPORTED;
     p.lut_n = mode != 2 ? (int)cb->lut.size() : 0;
-    // warp groups: as many (up to three) as shared memory holds
+    // warp groups: as many (up to four) as the launch bound and shared memory hold
     for (p.NG = kMaxGroups; p.NG > 1; --p.NG)
-        if (rpbh_smem_bytes(p) <= 227 * 1024) break;
+        if (p.NG * p.G <= kMaxThreads && rpbh_smem_bytes(p) <= 227 * 1024) break;
     p.T = p.NG * p.G;
     p.ntiles = (M + R - 1) / R;
     p.gtab = plan->dev.gtab;

@@ -8,7 +8,7 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM, each split into NG (1-3) warp groups that
+//   - persistent CTAs, one per SM, each split into NG (1-4) warp groups that
 //     take interleaved tiles of R rows and run out of phase (own staging buffers,
 //     mbarriers and named barriers), so one group's gathers overlap the
 //     others' butterflies and table lookups; a group stages its rows with
@@ -74,7 +74,7 @@ __device__ __forceinline__ void group_sync(int id, int count) {
 }
 
 template <typename InT, int H, int BITS, int MODE>
-__global__ void __launch_bounds__(384, 1) rpbh_quant_kernel(const RpbhParams p) {
+__global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);

@@ -32,7 +32,8 @@ struct RpbhParams {
     uint32_t mid_val;      // value outputs: the middle cell's value (bf16 bits or e4m3 byte)
 };
 
-constexpr int kMaxGroups = 3;  // warp groups per CTA (at most 128 threads each)
+constexpr int kMaxGroups = 4;    // warp groups per CTA (at most 128 threads each)
+constexpr int kMaxThreads = 384;  // per CTA: the kernel's launch bound (168 registers each)
 
 int rpbh_smem_bytes(const RpbhParams& p);
 
