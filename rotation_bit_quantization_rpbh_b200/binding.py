@@ -347,9 +347,10 @@ def qlinear_noalloc(plan, cb_a, cb_w, x, w_idx, w_r, y, bias=None, stream=None):
     """oq_qlinear without any device allocation inside the call, for callers
     that may not allocate device memory on their request path (a serving
     process that reserved all device memory at start-up).  The caller passes
-    the output ``y``; the packed activation codes go to the library's fixed
-    64 MiB per-device scratch array, shared by all calls: calls that overlap
-    on the GPU race on it, so keep them on one stream."""
+    the output ``y``; the activations' values (or, if they do not fit, their
+    packed codes) go to the library's fixed 128 MiB per-device scratch array,
+    shared by all calls: calls that overlap on the GPU race on it, so keep
+    them on one stream."""
     M, d = x.shape
     N = w_idx.shape[0]
     _check(lib().oq_qlinear_noalloc(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
