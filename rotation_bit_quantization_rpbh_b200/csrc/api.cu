@@ -121,9 +121,9 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.norm_out = norm_out;
     p.rsqrt_h = (float)(1.0 / std::sqrt((double)h));
     p.eps = (float)kEps;
-    p.starve = take_starve(OQ_STARVE_RPBH) ? 1 : 0;
     p.s_max = (float)(3.4028234663852886e38 / (2.0 * std::sqrt((double)h)));
     if (rpbh_smem_bytes(p) > 227 * 1024) return OQ_ERR_UNSUPPORTED;
+    p.starve = take_starve(OQ_STARVE_RPBH) ? 1 : 0;  // consumed by a launch that happens
     const int grid = p.ntiles < device_sms() ? p.ntiles : device_sms();
     cudaError_t e = launch_rpbh_quant(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, grid, st);
     return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
