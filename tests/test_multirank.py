@@ -77,3 +77,31 @@ def test_reference_arm_does_no_work_off_rank_zero(monkeypatch, capsys):
 
     bench.run_reference(A())
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
+    """Rank 0 of the reference arm (the oracle on the host cores) prints one
+    JSON line with the keys the bench contract asks of it."""
+    sys.path.insert(0, ROOT)
+    import json
+
+    import bench
+
+    monkeypatch.setenv("RANK", "0")
+
+    class A:
+        workload = "tiny_w4a4"
+        steps = 1
+        warmup = 0
+        gpus = 1
+
+    bench.run_reference(A())
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["metric"] == bench.METRIC and j["unit"] == "tokens/s"
+    assert j["value"] > 0 and j["higher_is_better"] is True and j["n_gpus"] == 1
+    assert j["config"]["workload"] == "tiny_w4a4"
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
