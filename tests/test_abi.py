@@ -159,3 +159,11 @@ def test_unpack_layout():
     assert B.unpack_indices(p2, 4, 2).tolist() == [[0, 1, 2, 3]]
     p6 = torch.tensor([[63, 5]], dtype=torch.uint8)
     assert B.unpack_indices(p6, 2, 6).tolist() == [[63, 5]]
+    p8 = torch.tensor([[255, 0, 128]], dtype=torch.uint8)
+    assert B.unpack_indices(p8, 3, 8).tolist() == [[255, 0, 128]]
+    # 3-bit: a bit stream, code k in bits 3k..3k+2 of the row (LSB first):
+    # codes 0..7 = 0,1,...,7 -> bits 000 001 010 011 100 101 110 111 from bit 0
+    stream = sum(k << (3 * k) for k in range(8))  # 24 bits
+    p3 = torch.tensor([[stream & 0xFF, (stream >> 8) & 0xFF, stream >> 16]], dtype=torch.uint8)
+    assert B.unpack_indices(p3, 8, 3).tolist() == [list(range(8))]
+    assert B.packed_row_bytes(1536, 8) == 1536 and B.packed_row_bytes(1536, 6) == 1536
