@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip timing the other large workloads (the per_workload block)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline sample")
     ap.add_argument("--fp8", action="store_true",
                     help="time the fp8 variant of the product (oq_qgemm_fp8: e4m3 centroid values)")
@@ -175,21 +177,21 @@ def job_throughput(world, tokens_per_rank, ms_per_step):
     return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
-def rpbh_bytes(w, schedule="codes", fp8=False):
-    """Algorithmic bytes of one quantiser launch: x read, then the packed
-    codes (codes schedule) or the centroid values (values schedule: 2 bytes
-    each, 1 in e4m3) written, plus s."""
+def rpbh_bytes(w):
+    """Algorithmic bytes of one quantiser launch as the method defines its
+    output: x read, the packed codes written (one byte per code at 6 bits),
+    and s.  The values schedule's 2-byte centroid values are this build's
+    layout for the product, not the method's output, so they count in the
+    measured traffic only."""
     esize = 4 if w.x_dtype == "f32" else 2
-    if schedule == "values":
-        out = w.d * (1 if fp8 else 2)
-    else:
-        out = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
+    out = w.d if w.bits_a in (6, 8) else w.d * w.bits_a // 8
     return w.M * (w.d * esize + out + 4)
 
 
-def cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, max_rows):
+def cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, max_rows, threads=0):
     """Times the oracle on `rows` tokens: rotate + quantise each row, then its
-    full output row of the quantised product.  Returns (tokens/s, rows, s, threads)."""
+    full output row of the quantised product, on `threads` threads (0: all).
+    Returns (tokens/s, rows, seconds, threads used, oracle codes and s of the rows)."""
     import numpy as np
 
     import oracle
@@ -203,20 +205,70 @@ def cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, max_rows):
 
     iw = B.unpack_indices(w_idx_cpu, w.d, w.bits_w).numpy()
     r64 = w_r_cpu.float().numpy().astype(np.float64)
+    oracle.set_num_threads(threads)
+    used = oracle.num_threads()
+    last = {}
 
     def run(rows):
         xs = x_cpu[:rows].float().numpy().astype(np.float64)
         t0 = time.perf_counter()
         q = oracle.quantize_rows(xs, w.h, perm, sign, ta, decision=32)
-        oracle.qlinear(q["idx"], q["s"], iw, r64, ca16, cw16)
-        return time.perf_counter() - t0
+        last["y"] = oracle.qlinear(q["idx"], q["s"], iw, r64, ca16, cw16)
+        dt = time.perf_counter() - t0
+        last["q"] = q
+        return dt
 
-    rows = 2
-    dt = run(rows)
-    while dt < target_s * 0.5 and rows < max_rows:
-        rows = min(max_rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
+    try:
+        rows = 2
         dt = run(rows)
-    return rows / dt, rows, dt, oracle.num_threads()
+        while dt < target_s * 0.5 and rows < max_rows:
+            rows = min(max_rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
+            dt = run(rows)
+    finally:
+        oracle.set_num_threads(0)
+    return rows / dt, rows, dt, used, last
+
+
+def cpu_baseline_block(w, x_cpu, w_idx_cpu, w_r_cpu, a_idx_gpu, s_gpu, y_gpu, target_s):
+    """The oracle as the CPU baseline, on the host's cores: the layer on a
+    bounded token sample (all threads, then one), the rotate-and-quantise
+    pass over the full batch (all threads), and the parity of the GPU's
+    codes, norms and product on the sampled rows."""
+    import numpy as np
+
+    import oracle
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+
+    tok_s, rows, dt, thr, last = cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, target_s, w.M)
+    tok_1, rows_1, dt_1, _, _ = cpu_oracle_sample(w, x_cpu, w_idx_cpu, w_r_cpu, max(2.0, target_s / 4), w.M, 1)
+    perm, sign = oracle.plan(w.d, w.h, w.plan_seed)
+    _, ta = oracle.codebook(w.d, w.bits_a)
+    x64 = x_cpu.float().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.quantize_rows(x64, w.h, perm, sign, ta, decision=32)
+    t_full = time.perf_counter() - t0
+    # parity on the sampled rows: codes, norms and product rows against the oracle
+    gi = B.unpack_indices(a_idx_gpu[:rows].cpu(), w.d, w.bits_a).numpy()
+    q = last["q"]
+    mism = int((gi != q["idx"]).sum())
+    s_rel = float(np.max(np.abs(s_gpu[:rows].cpu().numpy().astype(np.float64) - q["s"]) / np.maximum(q["s"], 1e-300)))
+    yg = y_gpu[:rows].float().cpu().numpy().astype(np.float64)
+    ref = last["y"]
+    rel = float(np.linalg.norm(yg - ref) / max(np.linalg.norm(ref), 1e-300))
+    return {"value": tok_s, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{rows} tokens of {w.name}: rotate+quantise each row, then its full {w.N}-wide output row "
+                      f"({dt:.1f} s on {thr} threads)",
+            "single_core": {"value": tok_1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{rows_1} tokens, same work ({dt_1:.1f} s)"},
+            "rpbh_quant_full_batch": {"seconds": t_full, "rows": w.M, "cores": thr,
+                                      "gbs": rpbh_bytes(w) / t_full / 1e9,
+                                      "note": "the oracle's rotate+split+quantise over all M rows (fp64, O(h) "
+                                              "direct sums per output)"},
+            "parity_on_sample": {"rows": rows, "code_mismatches": mism, "coordinates": rows * w.d,
+                                 "s_max_rel_diff": s_rel, "product_rel_frobenius": rel,
+                                 "note": "GPU codes (codes-mode launch) and GPU product rows against the oracle's "
+                                         "own codes and fp64 product; mismatches are threshold ties within "
+                                         "1e-6 relative (the parity tests check the band)"}}
 
 
 def run_reference(args):
@@ -227,10 +279,8 @@ def run_reference(args):
     if rank != 0:
         return
     import numpy as np
-    import torch
 
     import oracle
-    from rotation_bit_quantization_rpbh_b200 import binding as B
 
     w = I.WORKLOADS[args.workload]
     perm, sign = oracle.plan(w.d, w.h, w.plan_seed)
@@ -241,7 +291,9 @@ def run_reference(args):
     t_w = time.perf_counter()
     Wq = oracle.quantize_rows(I.make_w(w).float().numpy().astype(np.float64), w.h, perm, sign, tw, decision=32)
     t_w = time.perf_counter() - t_w
-    rows_per_step = max(1, min(w.M, 8))
+    threads = oracle.num_threads()
+    # four rows per thread keep every thread of the oracle's row loop busy
+    rows_per_step = max(1, min(w.M, 4 * threads))
     x = I.make_x(w, rows=np.arange(rows_per_step)).float().numpy().astype(np.float64)
 
     def step():
@@ -252,8 +304,8 @@ def run_reference(args):
     step()
     one = time.perf_counter() - t
     budget = 150.0
-    while rows_per_step > 1 and one * (args.steps + args.warmup) > budget:
-        rows_per_step //= 2
+    while rows_per_step > threads and one * (args.steps + args.warmup) > budget:
+        rows_per_step = max(threads, rows_per_step // 2)
         x = x[:rows_per_step]
         t = time.perf_counter()
         step()
@@ -270,12 +322,167 @@ def run_reference(args):
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": w.name, "tokens_per_step": rows_per_step, "M": w.M, "d": w.d, "N": w.N, "h": w.h,
                       "bits_w": w.bits_w, "bits_a": w.bits_a, "parallelism": "replicas"},
-           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                            "sample": f"{rows_per_step} tokens per step of {w.name} (rotate+quantise the rows, "
-                                      f"then their full {w.N}-wide output rows); offline weight pass "
-                                      f"{t_w:.1f} s untimed"},
+           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": f"{rows_per_step} tokens per step of {w.name} ({rows_per_step // threads} per "
+                                      f"thread; rotate+quantise the rows, then their full {w.N}-wide output rows); "
+                                      f"offline weight pass {t_w:.1f} s untimed"},
            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+class Layer:
+    """One workload's layer on the device: inputs, the offline weight pass,
+    the workspace and the two timed calls of a step (quantiser, product) in
+    the chosen schedule, plus a codes-mode quantiser launch."""
+
+    def __init__(self, w, dev, schedule, fp8):
+        import torch
+
+        from rotation_bit_quantization_rpbh_b200 import binding as B
+        from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+        self.w, self.schedule, self.fp8 = w, schedule, fp8
+        self.x_cpu = I.make_x(w)
+        W_cpu = I.make_w(w)
+        self.plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
+        self.cb_a, self.cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
+        self.x = self.x_cpu.to(dev)
+        self.w_idx, self.w_r = B.quantize_weights(self.plan, self.cb_w, W_cpu.to(dev))  # offline pass, untimed
+        del W_cpu
+        self.ws = torch.empty(max(B.qlinear_workspace(w.M, w.d, w.bits_a), B.qlinear_workspace_values(w.M, w.d)),
+                              dtype=torch.uint8, device=dev)
+        ws = self.ws
+        if schedule == "values":
+            vb = 1 if fp8 else 2
+            self.a_in = ws[: w.M * w.d * vb].view(w.M, w.d * vb)
+            if not fp8:
+                self.a_in = self.a_in.view(torch.bfloat16)
+            s_off = (w.M * w.d * vb + 255) // 256 * 256
+        else:
+            packed = B.packed_row_bytes(w.d, w.bits_a)
+            self.a_in = ws[: w.M * packed].view(w.M, packed)
+            s_off = (w.M * packed + 255) // 256 * 256
+        self.s = ws[s_off: s_off + 4 * w.M].view(torch.float32)
+        self.y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+        self.codes = torch.empty((w.M, B.packed_row_bytes(w.d, w.bits_a)), dtype=torch.uint8, device=dev)
+        self.s_codes = torch.empty(w.M, dtype=torch.float32, device=dev)
+
+    def quant(self, stream):
+        from rotation_bit_quantization_rpbh_b200 import binding as B
+
+        if self.schedule == "values":
+            B.quantize_acts_values(self.plan, self.cb_a, self.x, self.a_in, self.s, stream=stream, fp8=self.fp8)
+        else:
+            B.quantize_acts(self.plan, self.cb_a, self.x, self.a_in, self.s, stream=stream)
+
+    def gemm(self, stream):
+        from rotation_bit_quantization_rpbh_b200 import binding as B
+
+        if self.schedule == "values":
+            B.qgemm_values(self.cb_w, self.a_in, self.s, self.w_idx, self.w_r, y=self.y, stream=stream, fp8=self.fp8)
+        else:
+            (B.qgemm_fp8 if self.fp8 else B.qgemm)(self.cb_a, self.cb_w, self.a_in, self.s, self.w_idx, self.w_r,
+                                                    y=self.y, stream=stream)
+
+    def quant_codes(self, stream):
+        from rotation_bit_quantization_rpbh_b200 import binding as B
+
+        B.quantize_acts(self.plan, self.cb_a, self.x, self.codes, self.s_codes, stream=stream)
+
+
+def time_layer(L, steps, warmup, flush, stream):
+    """Event times (ms) of the whole step (quantiser then product, with
+    nothing between them in the stream, so the product's programmatic launch
+    overlaps the quantiser's end), then of the quantiser alone and of the
+    product alone, each over `steps` launches, L2 flushed before each
+    outside the events.  Returns (quantiser, product, step) lists."""
+    import torch
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        L.quant(stream)
+        L.gemm(stream)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    t_step = timed(lambda: (L.quant(stream), L.gemm(stream)))
+    t_rpbh = timed(lambda: L.quant(stream))
+    t_gemm = timed(lambda: L.gemm(stream))
+    return t_rpbh, t_gemm, t_step
+
+
+def time_codes_quantiser(L, steps, flush, stream):
+    """Event time (ms) per launch of the codes-mode quantiser (the method's
+    packed output), L2 flushed before each launch."""
+    import numpy as np
+    import torch
+
+    for _ in range(3):
+        flush.zero_()
+        L.quant_codes(stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        L.quant_codes(stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([e0.elapsed_time(e1) for e0, e1 in ev]))
+
+
+def host_call_overhead(L, stream, calls):
+    """Host time per oq_qlinear call (argument checks, marshalling and the
+    two launches), measured over `calls` back-to-back calls without a sync."""
+    import torch
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        B.qlinear(L.plan, L.cb_a, L.cb_w, L.x, L.w_idx, L.w_r, y=L.y, workspace=L.ws, stream=stream, fp8=L.fp8)
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    return (t1 - t0) / calls * 1e6
+
+
+def rooflines(w, peaks, fp8, ms_gemm, ms_rpbh, ms_codes, schedule, kernel_names):
+    flops = 2.0 * w.M * w.N * w.d
+    mma_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
+    rb = rpbh_bytes(w)
+    gemm_key, rpbh_key = kernel_names
+    out = {
+        "roofline": {"bound": "tensor", "kernel": gemm_key, "achieved": gemm_tflops, "peak": mma_peak,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / mma_peak,
+                     "traffic": committed_traffic(gemm_key, w.name),
+                     "peak_source": peaks["source"] + (" bf16 (burst) x nominal fp8/bf16 ratio 2" if fp8 else
+                                                       " (burst)"),
+                     "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
+        "roofline_rpbh": {"bound": "hbm", "kernel": rpbh_key, "achieved": rb / (ms_rpbh * 1e-3) / 1e9,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": rb / (ms_rpbh * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "traffic": committed_traffic(rpbh_key, w.name),
+                          "algorithmic": f"M*(d*in_bytes + packed codes + 4) = {rb} B per launch (the method's "
+                                         f"output; the {schedule} schedule's launch writes "
+                                         f"{'centroid values' if schedule == 'values' else 'the codes'})"},
+        "roofline_rpbh_codes": {"bound": "hbm", "kernel": "rpbh_quant", "achieved": rb / (ms_codes * 1e-3) / 1e9,
+                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": rb / (ms_codes * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "traffic": committed_traffic("rpbh_quant", w.name),
+                                "algorithmic": f"{rb} B per launch", "ms": ms_codes,
+                                "note": "the quantiser writing the packed codes (oq_quantize_acts), timed alone"},
+    }
+    return out, gemm_tflops
 
 
 def run_ours(args):
@@ -300,50 +507,15 @@ def run_ours(args):
     B.lib()
 
     w = I.WORKLOADS[args.workload]
-    x_cpu = I.make_x(w)
-    W_cpu = I.make_w(w)
-    plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
-    cb_a, cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
-    x = x_cpu.to(dev)
-    w_idx, w_r = B.quantize_weights(plan, cb_w, W_cpu.to(dev))  # offline pass, untimed
     schedule = "values" if args.schedule == "auto" else args.schedule  # the one oq_qlinear takes
-    ws = torch.empty(max(B.qlinear_workspace(w.M, w.d, w.bits_a), B.qlinear_workspace_values(w.M, w.d)),
-                     dtype=torch.uint8, device=dev)
-    if schedule == "values":
-        vb = 1 if args.fp8 else 2
-        a_in = ws[: w.M * w.d * vb].view(w.M, w.d * vb)
-        if not args.fp8:
-            a_in = a_in.view(torch.bfloat16)
-        s_off = (w.M * w.d * vb + 255) // 256 * 256
-    else:
-        packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
-        a_in = ws[: w.M * packed].view(w.M, packed)
-        s_off = (w.M * packed + 255) // 256 * 256
-    s = ws[s_off: s_off + 4 * w.M].view(torch.float32)
-    y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    L = Layer(w, dev, schedule, args.fp8)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
     stream = torch.cuda.current_stream()
 
-    if schedule == "values":
-        def quant():
-            B.quantize_acts_values(plan, cb_a, x, a_in, s, stream=stream, fp8=args.fp8)
-
-        def gemm():
-            B.qgemm_values(cb_w, a_in, s, w_idx, w_r, y=y, stream=stream, fp8=args.fp8)
-    else:
-        def quant():
-            B.quantize_acts(plan, cb_a, x, a_in, s, stream=stream)
-
-        def gemm():
-            (B.qgemm_fp8 if args.fp8 else B.qgemm)(cb_a, cb_w, a_in, s, w_idx, w_r, y=y, stream=stream)
-
-    def step():
-        quant()
-        gemm()
-
     for _ in range(max(3, args.warmup)):
         flush.zero_()
-        step()
+        L.quant(stream)
+        L.gemm(stream)
     torch.cuda.synchronize()
 
     uuid = None
@@ -353,33 +525,20 @@ def run_ours(args):
         pass
     sampler = ClockSampler(uuid)
     sampler.start()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.mark("start")
-    for i in range(args.steps):
-        flush.zero_()  # cold L2 for every step (outside the events)
-        ev[i][0].record(stream)
-        quant()
-        ev[i][1].record(stream)
-        gemm()
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
+    t_rpbh, t_gemm, t_step = time_layer(L, args.steps, 0, flush, stream)  # step first, then each kernel alone
     if world > 1:
         dist.barrier()
     sampler.mark("stop")
     clocks = sampler.stop()
     if B.device_status() != 0:
         raise SystemExit("a kernel reported a timeout")
-
-    t_rpbh = [e[0].elapsed_time(e[1]) for e in ev]
-    t_gemm = [e[1].elapsed_time(e[2]) for e in ev]
-    t_step = [e[0].elapsed_time(e[2]) for e in ev]
-    ms = float(np.mean(t_step))
-    ms_rpbh = float(np.mean(t_rpbh))
-    ms_gemm = float(np.mean(t_gemm))
-    ms, ms_rpbh, ms_gemm = reduce_max([ms, ms_rpbh, ms_gemm], world, dev)
+    ms, ms_rpbh, ms_gemm = reduce_max([float(np.mean(t_step)), float(np.mean(t_rpbh)), float(np.mean(t_gemm))],
+                                      world, dev)
+    ms_codes = reduce_max([time_codes_quantiser(L, max(5, min(args.steps, 20)), flush, stream)], world, dev)[0]
 
     # end to end through the public one-call API with host buffers: every
     # step copies its x in from pinned host memory, runs oq_qlinear and
@@ -387,14 +546,13 @@ def run_ours(args):
     # i+1 and copy-out of step i-1 overlap the layer of step i)
     e2e = None
     if not args.no_e2e:
-        x_pin = x_cpu.pin_memory()
+        x_pin = L.x_cpu.pin_memory()
         nbuf = 2
-        xs = [torch.empty_like(x) for _ in range(nbuf)]
-        ys = [torch.empty_like(y) for _ in range(nbuf)]
+        xs = [torch.empty_like(L.x) for _ in range(nbuf)]
+        ys = [torch.empty_like(L.y) for _ in range(nbuf)]
         # oq_qlinear takes its preferred schedule when the workspace holds it;
         # a codes-sized workspace makes it take the codes schedule
-        e2e_schedule = schedule
-        ws_e2e = ws.numel() if e2e_schedule == "values" else B.qlinear_workspace(w.M, w.d, w.bits_a)
+        ws_e2e = L.ws.numel() if schedule == "values" else B.qlinear_workspace(w.M, w.d, w.bits_a)
         wss = [torch.empty(ws_e2e, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
         y_pins = [torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
         s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -419,7 +577,8 @@ def run_ours(args):
             ev_in[b].record(s_in)
             s_cmp.wait_event(ev_in[b])
             s_cmp.wait_event(ev_out[b])  # the copy-out that last read ys[b] is done
-            B.qlinear(plan, cb_a, cb_w, xs[b], w_idx, w_r, y=ys[b], workspace=wss[b], stream=s_cmp, fp8=args.fp8)
+            B.qlinear(L.plan, L.cb_a, L.cb_w, xs[b], L.w_idx, L.w_r, y=ys[b], workspace=wss[b], stream=s_cmp,
+                      fp8=args.fp8)
             ev_cmp[b].record(s_cmp)
             s_out.wait_event(ev_cmp[b])
             with torch.cuda.stream(s_out):
@@ -431,23 +590,16 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = reduce_max([e0.elapsed_time(e1) / args.steps], world, dev)[0]
         e2e = {"value": job_throughput(world, w.M, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(x_cpu.numel() * x_cpu.element_size()),
-               "d2h_bytes_per_step": int(y.numel() * y.element_size()), "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(L.x_cpu.numel() * L.x_cpu.element_size()),
+               "d2h_bytes_per_step": int(L.y.numel() * L.y.element_size()), "ms_per_step": e2e_ms,
                "pipeline": "copy-in, oq_qlinear and copy-out on three streams, two buffers deep",
-               "schedule": e2e_schedule}
+               "schedule": schedule}
 
     peaks = measured_peaks()
-    # the fp8 variant's contraction peak: the measured bf16 peak times the
-    # nominal e4m3 / bf16 dense ratio (4.5 / 2.25 PFLOP/s)
-    mma_peak = peaks["bf16_tflops"] * (2.0 if args.fp8 else 1.0)
-    peak_note = peaks["source"] + (" bf16 (burst) x nominal fp8/bf16 ratio 2" if args.fp8 else " (burst)")
-    flops = 2.0 * w.M * w.N * w.d
-    gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
-    step_tflops = flops / (ms * 1e-3) / 1e12
-    rb = rpbh_bytes(w, schedule, args.fp8)
-    rpbh_gbs = rb / (ms_rpbh * 1e-3) / 1e9
     gemm_key = ("qgemm_values" if schedule == "values" else "qgemm") + ("_fp8" if args.fp8 else "")
     rpbh_key = "rpbh_quant" + (("_values_fp8" if args.fp8 else "_values") if schedule == "values" else "")
+    roof, gemm_tflops = rooflines(w, peaks, args.fp8, ms_gemm, ms_rpbh, ms_codes, schedule, (gemm_key, rpbh_key))
+    flops = 2.0 * w.M * w.N * w.d
     out = {
         "metric": METRIC, "value": job_throughput(world, w.M, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
@@ -456,27 +608,49 @@ def run_ours(args):
                    "bits_a": w.bits_a, "x_dtype": w.x_dtype, "tokens_per_gpu": w.M, "global_batch": world * w.M,
                    "parallelism": f"dp{world} (replicated packed W, no collective)", "schedule": schedule,
                    "l2": "flushed (256 MB write) before every timed step, outside the events"},
-        "tflops": step_tflops,
+        "tflops": flops / (ms * 1e-3) / 1e12,
         "breakdown": {"rpbh_quant_ms": ms_rpbh, "qgemm_ms": ms_gemm, "qgemm_tflops": gemm_tflops,
-                      "rpbh_quant_gbs": rpbh_gbs},
-        "roofline": {"bound": "tensor", "kernel": gemm_key, "achieved": gemm_tflops,
-                     "peak": mma_peak, "unit": "TFLOP/s", "frac": gemm_tflops / mma_peak,
-                     "traffic": committed_traffic(gemm_key, w.name), "peak_source": peak_note,
-                     "algorithmic": f"2*M*N*d = {flops:.4g} flop per launch"},
-        "roofline_rpbh": {"bound": "hbm", "kernel": rpbh_key, "achieved": rpbh_gbs, "peak": peaks["hbm_gbs"],
-                          "unit": "GB/s", "frac": rpbh_gbs / peaks["hbm_gbs"],
-                          "traffic": committed_traffic(rpbh_key, w.name),
-                          "algorithmic": f"M*(d*in_bytes + {'values' if schedule == 'values' else 'packed'} + 4) = "
-                                         f"{rb} B per launch"},
+                      "rpbh_quant_gbs": roof["roofline_rpbh"]["achieved"], "rpbh_quant_codes_ms": ms_codes,
+                      "overlap_ms": ms_rpbh + ms_gemm - ms,
+                      "note": "the step is timed as one unit (the product launches programmatically and overlaps "
+                              "the quantiser's end); each kernel is then timed alone over the same number of "
+                              "launches, L2 flushed before each"},
+        **roof,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "e2e": e2e,
     }
+    # host time per oq_qlinear call: flat in the number of calls (no per-call
+    # device allocation, synchronisation or tensor-map encoding)
+    out["host_us_per_call"] = {str(n): host_call_overhead(L, stream, n) for n in (10, 100)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, rows, dt, thr = cpu_oracle_sample(w, x_cpu, w_idx.cpu(), w_r.cpu(), args.cpu_seconds, w.M)
-        out["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-                               "sample": f"{rows} tokens of {w.name}: rotate+quantise each row, then its full "
-                                         f"{w.N}-wide output row ({dt:.1f} s)"}
+        L.quant_codes(stream)
+        torch.cuda.synchronize()
+        out["cpu_baseline"] = cpu_baseline_block(w, L.x_cpu, L.w_idx.cpu(), L.w_r.cpu(), L.codes, L.s_codes, L.y,
+                                                 args.cpu_seconds)
+    # the other large workloads, each timed the same way on this GPU
+    if world == 1 and not args.no_per_workload:
+        per = {}
+        for name in I.ORDER:
+            w2 = I.WORKLOADS[name]
+            if name == w.name or w2.M < 1024:
+                continue
+            L2 = Layer(w2, dev, schedule, args.fp8)
+            k2 = max(5, min(args.steps, 20))
+            tr, tg, ts = time_layer(L2, k2, 3, flush, stream)
+            mc = time_codes_quantiser(L2, k2, flush, stream)
+            if B.device_status() != 0:
+                raise SystemExit("a kernel reported a timeout")
+            r2, gt2 = rooflines(w2, peaks, args.fp8, float(np.mean(tg)), float(np.mean(tr)), mc, schedule,
+                                (gemm_key, rpbh_key))
+            per[name] = {"tokens_per_s": w2.M / (float(np.mean(ts)) * 1e-3), "ms_per_step": float(np.mean(ts)),
+                         "steps": k2, "qgemm_tflops": gt2, "qgemm_frac": r2["roofline"]["frac"],
+                         "rpbh_quant_ms": float(np.mean(tr)), "rpbh_quant_gbs": r2["roofline_rpbh"]["achieved"],
+                         "rpbh_quant_frac": r2["roofline_rpbh"]["frac"], "rpbh_quant_codes_ms": mc,
+                         "rpbh_quant_codes_frac": r2["roofline_rpbh_codes"]["frac"]}
+            del L2
+            torch.cuda.empty_cache()
+        out["per_workload"] = per
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -25,7 +25,12 @@
  *     their free functions.  A plan holds device tables on the device that
  *     was current when it was created.
  *   - Device work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
- *     default stream) and is asynchronous: the library never synchronises.
+ *     default stream) and is asynchronous.  Only set-up calls synchronise:
+ *     oq_rpbh_plan / oq_rotation_plan and oq_codebook_upload allocate and copy
+ *     their tables with a synchronous copy, and so does the first quantising
+ *     call of a codebook on a device that it was not uploaded to (call
+ *     oq_codebook_upload at set-up to keep the hot calls free of allocation
+ *     and synchronisation).  oq_device_status synchronises its stream.
  *     Launch failures are reported as OQ_ERR_CUDA.  A kernel that gives up a
  *     bounded wait records OQ_ERR_TIMEOUT in a device flag read by
  *     oq_device_status().
@@ -85,6 +90,13 @@ const char* oq_status_str(oq_status s);
 /*   out  receives a library-owned handle (free with oq_codebook_free).    */
 oq_status oq_codebook(int d, int bits, oq_codebook_t** out);
 
+/* Uploads the codebook's quantiser tables to the current device          */
+/* (allocation and a synchronous copy; once per codebook and device --     */
+/* later calls return at once).  The quantising calls do it themselves on  */
+/* first use; calling it at set-up keeps them free of both.  The tables    */
+/* are freed by oq_codebook_free.  OQ_ERR_OOM / OQ_ERR_CUDA on failure.    */
+oq_status oq_codebook_upload(const oq_codebook_t* cb);
+
 /* Copies the fp64 codebook: centroids[2^bits] ascending and               */
 /* thresholds[2^bits - 1] (midpoints of adjacent centroids; the middle one */
 /* is exactly 0).  Host pointers; either may be NULL.                       */
@@ -115,7 +127,9 @@ oq_status oq_rpbh_plan(int d, int h, uint64_t seed, oq_plan_t** out);
 /* sign[d] (int8, +-1).  Either may be NULL.                               */
 oq_status oq_rpbh_plan_export(const oq_plan_t* plan, int32_t* perm, int8_t* sign);
 
-/* Host-only plan generation (no device tables): same arrays as above. */
+/* Host-only plan generation (no device tables): same arrays as above.    */
+/* Accepts any d in [1, 32767] and any h >= 1 dividing d (the arrays do    */
+/* not depend on h); the device calls keep the limits of oq_rpbh_plan.     */
 oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign);
 
 /* Rotation variants for the page's rotation ablation [OrbitQuant, section */
@@ -267,12 +281,16 @@ oq_status oq_qlinear_fp8(const oq_plan_t* plan, const oq_codebook_t* cb_a, const
 /*   (OQ_NOALLOC_SCRATCH_BYTES, 128 MiB, held until the process exits),   */
 /*   in the values schedule when its workspace fits there, else in the    */
 /*   codes schedule.                                                       */
-/*   Requests needing more than that (oq_qlinear_workspace(M, d, bits_a)  */
-/*   > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE before any work. */
-/*   Nothing is allocated here: the plan and both codebooks must already  */
-/*   have their tables on this device (a plan gets them when created; a   */
-/*   codebook on its first oq_quantize_acts / oq_quantize_weights /       */
-/*   oq_qlinear call on the device), else OQ_ERR_INVALID_ARG.             */
+/*   The schedule is decided before any work: requests that fit neither   */
+/*   schedule the code widths allow (values: oq_qlinear_workspace_values; */
+/*   codes: oq_qlinear_workspace(M, d, bits_a)) within                     */
+/*   OQ_NOALLOC_SCRATCH_BYTES return OQ_ERR_TOO_LARGE, widths no product  */
+/*   supports OQ_ERR_UNSUPPORTED, and nothing runs.                        */
+/*   Nothing is allocated here: the plan and the activation codebook must */
+/*   already have their tables on this device (a plan gets them when      */
+/*   created; a codebook on oq_codebook_upload or on its first quantising  */
+/*   call on the device), else OQ_ERR_INVALID_ARG.  The weight codebook    */
+/*   reaches the product through launch parameters and needs no tables.   */
 /*   The first call on a device looks up the scratch array's device       */
 /*   address (once per device); make that first call before any stream   */
 /*   capture.  All calls share the one array and it keeps the last call's */
@@ -304,10 +322,17 @@ oq_status oq_device_status(int clear, int* out, void* stream);
 /*   returns without faulting; the context stays usable.  The output of     */
 /*   that launch is undefined.  The call itself still returns OQ_OK.        */
 /*   Each call replaces the pending set; mask 0 cancels.                    */
+/* oq_debug_rpbh_layout(rows_per_warp, slots): the rotate-and-quantise    */
+/*   kernel's work layout -- rows of x per warp (1, 2, 4 or 8) and staging  */
+/*   slots per warp team (1 or 2) -- is forced for the following launches   */
+/*   where it fits in shared memory (0 or another value: chosen by the      */
+/*   library, the default).  Results do not depend on it except for the    */
+/*   rounding order of the row norm's sum.  For tests and tuning.           */
 #define OQ_STARVE_RPBH 1 /* the rotate-and-quantise kernel (acts and weights) */
 #define OQ_STARVE_GEMM 2 /* the codebook-decode GEMM (bf16 and fp8)           */
 void oq_debug_fail_allocations(int n);
 void oq_debug_starve(int mask);
+void oq_debug_rpbh_layout(int rows_per_warp, int slots);
 
 #ifdef __cplusplus
 }

@@ -46,6 +46,7 @@ def lib():
         L.oracle_qlinear.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, ctypes.c_int, P,
                                      ctypes.c_int, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = L
     return _lib
 
@@ -168,6 +169,11 @@ def qlinear(ia, s, iw, r, ca, cw, rows=None, cols=None):
 
 def num_threads():
     return lib().oracle_num_threads()
+
+
+def set_num_threads(n):
+    """Threads of the oracle's parallel loops (n <= 0: the default)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def widen_bf16(bits_u16):

@@ -425,3 +425,16 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Thread count of the following parallel loops (timing the oracle on one
+ * core and on all of them); n <= 0 restores the default. */
+static int oracle_default_threads = 0;
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (!oracle_default_threads) oracle_default_threads = omp_get_max_threads();
+    omp_set_num_threads(n > 0 ? n : oracle_default_threads);
+#else
+    (void)n;
+#endif
+}

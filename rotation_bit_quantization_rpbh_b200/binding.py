@@ -33,7 +33,8 @@ EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf
            "oq_plan_free", "oq_quantize_weights", "oq_quantize_acts", "oq_rpbh_apply", "oq_qgemm",
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status",
            "oq_debug_fail_allocations", "oq_debug_starve", "oq_quantize_acts_values",
-           "oq_quantize_acts_values_fp8", "oq_qgemm_values", "oq_qgemm_values_fp8", "oq_qlinear_workspace_values"]
+           "oq_quantize_acts_values_fp8", "oq_qgemm_values", "oq_qgemm_values_fp8", "oq_qlinear_workspace_values",
+           "oq_debug_rpbh_layout", "oq_codebook_upload"]
 
 
 class OQError(RuntimeError):
@@ -64,6 +65,7 @@ def lib():
                     "oq_codebook_bf16": ([P, P], I),
                     "oq_codebook_shape": ([P, P, P], I),
                     "oq_codebook_free": ([P], None),
+                    "oq_codebook_upload": ([P], I),
                     "oq_rpbh_plan": ([I, I, U64, P], I),
                     "oq_rpbh_plan_export": ([P, P, P], I),
                     "oq_rpbh_plan_host": ([I, I, U64, P, P], I),
@@ -84,6 +86,7 @@ def lib():
                     "oq_device_status": ([I, P, P], I),
                     "oq_debug_fail_allocations": ([I], None),
                     "oq_debug_starve": ([I], None),
+                    "oq_debug_rpbh_layout": ([I, I], None),
                     "oq_quantize_acts_values": ([P, P, P, I, I, P, P, P], I),
                     "oq_quantize_acts_values_fp8": ([P, P, P, I, I, P, P, P], I),
                     "oq_qgemm_values": ([P, I, I, P, P, P, P, P, P, P], I),
@@ -122,7 +125,44 @@ def _dtype_code(t):
 
 
 def packed_row_bytes(d, bits):
-    return d if bits == 6 else d * bits // 8
+    """Bytes of one packed row of d codes: one code per byte at 6 and 8 bits,
+    else d * bits / 8 (3 bits: a bit stream, eight codes per three bytes)."""
+    return d if bits in (6, 8) else d * bits // 8
+
+
+def _need(t, name, shape, dtypes, device):
+    """The C ABI sees only pointers and sizes: a tensor of the wrong shape,
+    dtype, layout or device would make the kernels read or write out of
+    bounds.  Check each buffer here and raise ValueError instead."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    if not isinstance(dtypes, tuple):
+        dtypes = (dtypes,)
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _need_input(x, name, d):
+    """x: a contiguous [rows, d] bf16 or fp32 CUDA tensor; returns rows."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D torch.Tensor")
+    if x.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    _need(x, name, (x.shape[0], d), (torch.bfloat16, torch.float32), x.device)
+    return x.shape[0]
+
+
+def _need_opt(t, name, shape, dtypes, device):
+    if t is not None:
+        _need(t, name, shape, dtypes, device)
 
 
 class Codebook:
@@ -146,6 +186,12 @@ class Codebook:
         _check(lib().oq_codebook_values(self._h, c.ctypes.data_as(ctypes.c_void_p),
                                         t.ctypes.data_as(ctypes.c_void_p)), "oq_codebook_values")
         return c, t[: self.L - 1]
+
+    def upload(self):
+        """Put the quantiser tables on the current device now (set-up), so
+        the quantising calls neither allocate nor synchronise later."""
+        _check(lib().oq_codebook_upload(self._h), "oq_codebook_upload")
+        return self
 
     def e4m3_bytes(self):
         """The fp8 variant's centroid values: e4m3 bytes of c_j sqrt(d)."""
@@ -233,22 +279,28 @@ def rpbh_plan_host(d, h, seed):
 
 
 def quantize_weights(plan, cb_w, W, idx_out=None, r_out=None, stream=None):
-    N, d = W.shape
+    N = _need_input(W, "W", plan.d)
+    d = plan.d
     if idx_out is None:
         idx_out = torch.empty((N, packed_row_bytes(d, cb_w.bits)), dtype=torch.uint8, device=W.device)
     if r_out is None:
         r_out = torch.empty(N, dtype=torch.bfloat16, device=W.device)
+    _need(idx_out, "idx_out", (N, packed_row_bytes(d, cb_w.bits)), torch.uint8, W.device)
+    _need(r_out, "r_out", (N,), torch.bfloat16, W.device)
     _check(lib().oq_quantize_weights(plan.handle, cb_w.handle, _ptr(W), _dtype_code(W), N, _ptr(idx_out),
                                      _ptr(r_out), _stream(stream)), "oq_quantize_weights")
     return idx_out, r_out
 
 
 def quantize_acts(plan, cb_a, x, idx_out=None, s_out=None, stream=None):
-    M, d = x.shape
+    M = _need_input(x, "x", plan.d)
+    d = plan.d
     if idx_out is None:
         idx_out = torch.empty((M, packed_row_bytes(d, cb_a.bits)), dtype=torch.uint8, device=x.device)
     if s_out is None:
         s_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _need(idx_out, "idx_out", (M, packed_row_bytes(d, cb_a.bits)), torch.uint8, x.device)
+    _need(s_out, "s_out", (M,), torch.float32, x.device)
     _check(lib().oq_quantize_acts(plan.handle, cb_a.handle, _ptr(x), _dtype_code(x), M, _ptr(idx_out), _ptr(s_out),
                                   _stream(stream)), "oq_quantize_acts")
     return idx_out, s_out
@@ -258,11 +310,14 @@ def quantize_acts_values(plan, cb_a, x, val_out=None, s_out=None, stream=None, f
     """The online pass writing the centroid values C_a[idx] (a bf16 tensor
     [M, d]) instead of the codes; ``fp8=True`` writes the e4m3 bytes of
     c sqrt(d) (uint8)."""
-    M, d = x.shape
+    M = _need_input(x, "x", plan.d)
+    d = plan.d
     if val_out is None:
         val_out = torch.empty((M, d), dtype=torch.uint8 if fp8 else torch.bfloat16, device=x.device)
     if s_out is None:
         s_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _need(val_out, "val_out", (M, d), torch.uint8 if fp8 else torch.bfloat16, x.device)
+    _need(s_out, "s_out", (M,), torch.float32, x.device)
     fn, name = ((lib().oq_quantize_acts_values_fp8, "oq_quantize_acts_values_fp8") if fp8
                 else (lib().oq_quantize_acts_values, "oq_quantize_acts_values"))
     _check(fn(plan.handle, cb_a.handle, _ptr(x), _dtype_code(x), M, _ptr(val_out), _ptr(s_out), _stream(stream)), name)
@@ -270,20 +325,42 @@ def quantize_acts_values(plan, cb_a, x, val_out=None, s_out=None, stream=None, f
 
 
 def rpbh_apply(plan, x, x_rot=None, norm_out=None, stream=None):
-    M, d = x.shape
+    M = _need_input(x, "x", plan.d)
+    d = plan.d
     if x_rot is None:
         x_rot = torch.empty((M, d), dtype=torch.float32, device=x.device)
     if norm_out is None:
         norm_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _need(x_rot, "x_rot", (M, d), torch.float32, x.device)
+    _need(norm_out, "norm_out", (M,), torch.float32, x.device)
     _check(lib().oq_rpbh_apply(plan.handle, _ptr(x), _dtype_code(x), M, _ptr(x_rot), _ptr(norm_out),
                                _stream(stream)), "oq_rpbh_apply")
     return x_rot, norm_out
 
 
-def qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
-    M, N = a_idx.shape[0], w_idx.shape[0]
+def _need_product(cb_w, a, a_name, a_cols, a_dtype, s, w_idx, w_r, bias, y):
+    """Shapes of the product's buffers: a [M, a_cols], s [M] fp32, w_idx
+    [N, packed row of cb_w], w_r [N] bf16, bias [N] bf16 or None, y [M, N]
+    bf16 (allocated if None), all on a's CUDA device.  Returns (M, N, y)."""
+    if not isinstance(a, torch.Tensor) or a.dim() != 2 or a.device.type != "cuda":
+        raise ValueError(f"{a_name} must be a 2-D CUDA tensor")
+    if not isinstance(w_idx, torch.Tensor) or w_idx.dim() != 2:
+        raise ValueError("w_idx must be a 2-D tensor")
+    M, N, dev = a.shape[0], w_idx.shape[0], a.device
+    _need(a, a_name, (M, a_cols), a_dtype, dev)
+    _need(s, "s", (M,), torch.float32, dev)
+    _need(w_idx, "w_idx", (N, packed_row_bytes(cb_w.d, cb_w.bits)), torch.uint8, dev)
+    _need(w_r, "w_r", (N,), torch.bfloat16, dev)
+    _need_opt(bias, "bias", (N,), torch.bfloat16, dev)
     if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_idx.device)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "y", (M, N), torch.bfloat16, dev)
+    return M, N, y
+
+
+def qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
+    M, N, y = _need_product(cb_w, a_idx, "a_idx", packed_row_bytes(cb_a.d, cb_a.bits), torch.uint8, s,
+                            w_idx, w_r, bias, y)
     _check(lib().oq_qgemm(cb_a.handle, cb_w.handle, M, N, _ptr(a_idx), _ptr(s), _ptr(w_idx), _ptr(w_r), _ptr(bias),
                           _ptr(y), _stream(stream)), "oq_qgemm")
     return y
@@ -291,9 +368,8 @@ def qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
 
 def qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
     """oq_qgemm with e4m3 centroid values on the fp8 tensor cores."""
-    M, N = a_idx.shape[0], w_idx.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_idx.device)
+    M, N, y = _need_product(cb_w, a_idx, "a_idx", packed_row_bytes(cb_a.d, cb_a.bits), torch.uint8, s,
+                            w_idx, w_r, bias, y)
     _check(lib().oq_qgemm_fp8(cb_a.handle, cb_w.handle, M, N, _ptr(a_idx), _ptr(s), _ptr(w_idx), _ptr(w_r),
                               _ptr(bias), _ptr(y), _stream(stream)), "oq_qgemm_fp8")
     return y
@@ -302,9 +378,8 @@ def qgemm_fp8(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=None, y=None, stream=None):
 def qgemm_values(cb_w, a_val, s, w_idx, w_r, bias=None, y=None, stream=None, fp8=False):
     """The product with A given as centroid values (bf16 [M, d], or uint8
     e4m3 bytes with ``fp8=True``): only W is decoded in the kernel."""
-    M, N = a_val.shape[0], w_idx.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_val.device)
+    M, N, y = _need_product(cb_w, a_val, "a_val", cb_w.d, torch.uint8 if fp8 else torch.bfloat16, s, w_idx, w_r,
+                            bias, y)
     fn, name = (lib().oq_qgemm_values_fp8, "oq_qgemm_values_fp8") if fp8 else (lib().oq_qgemm_values,
                                                                                 "oq_qgemm_values")
     _check(fn(cb_w.handle, M, N, _ptr(a_val), _ptr(s), _ptr(w_idx), _ptr(w_r), _ptr(bias), _ptr(y), _stream(stream)),
@@ -320,15 +395,30 @@ def qlinear_workspace_values(M, d):
     return int(lib().oq_qlinear_workspace_values(M, d))
 
 
+def _need_layer(plan, cb_w, x, w_idx, w_r, bias, y, alloc_y):
+    """The layer's buffers: x [M, plan d] bf16/fp32, w_idx [N, packed row of
+    cb_w], w_r [N] bf16, bias [N] bf16 or None, y [M, N] bf16 (allocated
+    here if None and alloc_y).  Returns (M, N, y, d)."""
+    d = plan.d
+    M = _need_input(x, "x", d)
+    if not isinstance(w_idx, torch.Tensor) or w_idx.dim() != 2:
+        raise ValueError("w_idx must be a 2-D tensor")
+    N = w_idx.shape[0]
+    _need(w_idx, "w_idx", (N, packed_row_bytes(d, cb_w.bits)), torch.uint8, x.device)
+    _need(w_r, "w_r", (N,), torch.bfloat16, x.device)
+    _need_opt(bias, "bias", (N,), torch.bfloat16, x.device)
+    if y is None and alloc_y:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, "y", (M, N), torch.bfloat16, x.device)
+    return M, N, y, d
+
+
 def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, stream=None, fp8=False,
             schedule="auto"):
     """The full layer x -> y (oq_qlinear; oq_qlinear_fp8 with fp8=True).
     ``schedule`` sizes the workspace allocated here: "auto" (room for the
     values schedule, which the library then takes) or "codes"."""
-    M, d = x.shape
-    N = w_idx.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    M, N, y, d = _need_layer(plan, cb_w, x, w_idx, w_r, bias, y, alloc_y=True)
     if schedule not in ("auto", "codes"):
         raise ValueError(f"unknown schedule {schedule!r}")
     if schedule == "auto":
@@ -337,6 +427,9 @@ def qlinear(plan, cb_a, cb_w, x, w_idx, w_r, bias=None, y=None, workspace=None, 
         need = qlinear_workspace(M, d, cb_a.bits)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    if (not isinstance(workspace, torch.Tensor) or workspace.dtype != torch.uint8 or not workspace.is_contiguous()
+            or workspace.device != x.device):
+        raise ValueError("workspace must be a contiguous uint8 tensor on x's device")
     fn, name = (lib().oq_qlinear_fp8, "oq_qlinear_fp8") if fp8 else (lib().oq_qlinear, "oq_qlinear")
     _check(fn(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx), _ptr(w_r), N,
               _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)), name)
@@ -351,8 +444,7 @@ def qlinear_noalloc(plan, cb_a, cb_w, x, w_idx, w_r, y, bias=None, stream=None):
     packed codes) go to the library's fixed 128 MiB per-device scratch array,
     shared by all calls: calls that overlap on the GPU race on it, so keep
     them on one stream."""
-    M, d = x.shape
-    N = w_idx.shape[0]
+    M, N, y, _ = _need_layer(plan, cb_w, x, w_idx, w_r, bias, y, alloc_y=False)
     _check(lib().oq_qlinear_noalloc(plan.handle, cb_a.handle, cb_w.handle, _ptr(x), _dtype_code(x), M, _ptr(w_idx),
                                     _ptr(w_r), N, _ptr(bias), _ptr(y), _stream(stream)), "oq_qlinear_noalloc")
     return y
@@ -376,6 +468,13 @@ def debug_starve(mask):
     waits run out and ``device_status()`` reports OQ_ERR_TIMEOUT.  Replaces
     the pending set; 0 cancels."""
     lib().oq_debug_starve(int(mask))
+
+
+def debug_rpbh_layout(rows_per_warp=0, slots=0):
+    """Test and tuning hook: force the rotate-and-quantise kernel's rows per
+    warp (1, 2, 4, 8) and staging slots per warp team (1, 2) where they fit;
+    0 restores the library's choice."""
+    lib().oq_debug_rpbh_layout(int(rows_per_warp), int(slots))
 
 
 def unpack_indices(packed, d, bits):

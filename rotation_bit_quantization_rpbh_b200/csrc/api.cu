@@ -84,27 +84,23 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     }
     const int d = plan->d, h = plan->h, nb = d / h;
     const int esize = dtype == OQ_BF16 ? 2 : 4;
+    if (esize == 4 && d > 16384) return OQ_ERR_UNSUPPORTED;  // fp32 byte offsets of the gather table
+    const bool big = h > 128;  // blocks beyond the in-register kernel (rht_big.cu)
+    if (big && mode != 2 && cb->bits == 3) return OQ_ERR_UNSUPPORTED;
     RpbhParams p;
     std::memset(&p, 0, sizeof(p));
     p.x = x;
     p.M = M;
     p.d = d;
     p.nb = nb;
-    p.row_bytes = d * esize;
-    p.srow = d * esize + 16;  // +16 B: consecutive rows start 4 banks apart
-    int R = 1;
-    // rows per tile: a power of two, at most 128 threads per warp group,
-    // four staging buffers (two groups x two stages) within ~180 KB
-    while (R < 32 && 2 * R * nb <= 128 && 4 * (2 * R) * p.srow <= 180 * 1024) R *= 2;
-    p.R = R;
-    p.G = (nb * R + 31) / 32 * 32;
-    if (p.G > 128) return OQ_ERR_UNSUPPORTED;
     p.lut_n = mode != 2 ? (int)cb->lut.size() : 0;
-    // warp groups: as many (up to four) as the launch bound and shared memory hold
-    for (p.NG = kMaxGroups; p.NG > 1; --p.NG)
-        if (p.NG * p.G <= kMaxThreads && rpbh_smem_bytes(p) <= 227 * 1024) break;
-    p.T = p.NG * p.G;
-    p.ntiles = (M + R - 1) / R;
+    if (big) {
+        p.row_bytes = d * esize;
+        if (rht_big_smem_bytes(p) > kSmemLimit) return OQ_ERR_UNSUPPORTED;
+    } else {
+        if (!rpbh_choose_layout(p, h, esize)) return OQ_ERR_UNSUPPORTED;
+        p.nrs = (M + p.RW - 1) / p.RW;
+    }
     p.gtab = plan->dev.gtab;
     if (mode != 2) {
         p.lut = mode == 3 ? dcb->lut_vb : (mode == 4 ? dcb->lut_v8 : dcb->lut);
@@ -122,10 +118,19 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.rsqrt_h = (float)(1.0 / std::sqrt((double)h));
     p.eps = (float)kEps;
     p.s_max = (float)(3.4028234663852886e38 / (2.0 * std::sqrt((double)h)));
-    if (rpbh_smem_bytes(p) > 227 * 1024) return OQ_ERR_UNSUPPORTED;
     p.starve = take_starve(OQ_STARVE_RPBH) ? 1 : 0;  // consumed by a launch that happens
-    const int grid = p.ntiles < device_sms() ? p.ntiles : device_sms();
-    cudaError_t e = launch_rpbh_quant(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, grid, st);
+    cudaError_t e;
+    if (big) {
+        // one row per CTA at a time, as many CTAs per SM as shared memory holds (at most 8)
+        int per_sm = kSmemLimit / rht_big_smem_bytes(p);
+        per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+        const int cap = per_sm * device_sms();
+        e = launch_rht_big(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, M < cap ? M : cap, st);
+    } else {
+        const int per_cta = (p.nrs + p.tpc - 1) / p.tpc;
+        const int grid = per_cta < device_sms() ? per_cta : device_sms();
+        e = launch_rpbh_quant(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, grid, st);
+    }
     return e == cudaSuccess ? OQ_OK : OQ_ERR_CUDA;
 }
 
@@ -200,6 +205,12 @@ oq_status oq_codebook(int d, int bits, oq_codebook_t** out) {
     return OQ_OK;
 }
 
+oq_status oq_codebook_upload(const oq_codebook_t* cb) {
+    if (!cb) return OQ_ERR_INVALID_ARG;
+    const DeviceCodebook* dcb = nullptr;
+    return codebook_device(const_cast<oq_codebook_t*>(cb), &dcb);
+}
+
 oq_status oq_codebook_values(const oq_codebook_t* cb, double* centroids, double* thresholds) {
     if (!cb) return OQ_ERR_INVALID_ARG;
     if (centroids) std::memcpy(centroids, cb->c.data(), sizeof(double) * cb->L);
@@ -227,9 +238,12 @@ void oq_codebook_free(oq_codebook_t* cb) {
     delete cb;
 }
 
+// Device plans: h a power of two in [16, 16384] dividing d (h <= 128: the
+// in-register kernel; larger blocks, e.g. the ablation's Full RHT h = d: the
+// staged kernel of rht_big.cu).
 static oq_status check_plan_args(int d, int h) {
     if (d <= 0 || h <= 0) return OQ_ERR_INVALID_ARG;
-    if ((h & (h - 1)) != 0 || h < 16 || h > 128 || d % h != 0 || d > 32767 || d % 8 != 0) return OQ_ERR_UNSUPPORTED;
+    if ((h & (h - 1)) != 0 || h < 16 || h > 16384 || d % h != 0 || d > 32767 || d % 8 != 0) return OQ_ERR_UNSUPPORTED;
     return OQ_OK;
 }
 
@@ -238,8 +252,9 @@ oq_status oq_rpbh_plan_host(int d, int h, uint64_t seed, int32_t* perm, int8_t* 
 }
 
 oq_status oq_rotation_plan_host(int d, int h, uint64_t seed, int variant, int32_t* perm, int8_t* sign) {
-    oq_status s = check_plan_args(d, h);
-    if (s != OQ_OK) return s;
+    // no device tables: any d in [1, 32767] and any block size h >= 1 dividing d
+    if (d <= 0 || h <= 0) return OQ_ERR_INVALID_ARG;
+    if (d > 32767 || d % h != 0) return OQ_ERR_UNSUPPORTED;
     if (variant != OQ_ROT_RPBH && variant != OQ_ROT_BLOCK_RHT) return OQ_ERR_INVALID_ARG;
     std::vector<int32_t> pv(d);
     std::vector<int8_t> sv(d);
@@ -272,16 +287,16 @@ oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t**
     make_plan(d, h, seed, p->perm.data(), p->sign.data(), variant);
     build_gather_table(p, p->gtab_host);
     void* ptr = nullptr;
-    if (!device_alloc(&ptr, sizeof(uint16_t) * d)) {
+    if (!device_alloc(&ptr, sizeof(uint32_t) * d)) {
         delete p;
         return OQ_ERR_OOM;
     }
-    if (cudaMemcpy(ptr, p->gtab_host.data(), sizeof(uint16_t) * d, cudaMemcpyHostToDevice) != cudaSuccess) {
+    if (cudaMemcpy(ptr, p->gtab_host.data(), sizeof(uint32_t) * d, cudaMemcpyHostToDevice) != cudaSuccess) {
         cudaFree(ptr);
         delete p;
         return OQ_ERR_CUDA;
     }
-    p->dev.gtab = static_cast<uint16_t*>(ptr);
+    p->dev.gtab = static_cast<uint32_t*>(ptr);
     *out = p;
     return OQ_OK;
 }
@@ -338,19 +353,32 @@ oq_status oq_rpbh_apply(const oq_plan_t* plan, const void* x, oq_dtype dtype, in
                     static_cast<cudaStream_t>(stream));
 }
 
+// Whether the products support these code widths: the codes product
+// decodes both operands (2, 4 or 6 bits, or a pair of 3- and 4-bit codes),
+// the values product decodes W only (2, 3, 4 or 6 bits).  8-bit codes have no
+// in-kernel decoder (8-bit activations take the values schedule).  K steps
+// take d % 64 == 0 (bf16) or d % 128 == 0 (e4m3); 3-bit rows need
+// d % 128 == 0 (rows of whole 16-byte groups).
+static bool codes_product_ok(int ba, int bw, int d, bool fp8) {
+    if (d % (fp8 ? 128 : 64) != 0) return false;
+    if ((ba == 3 || bw == 3) && d % 128 != 0) return false;
+    auto ok246 = [](int b) { return b == 2 || b == 4 || b == 6; };
+    if (ok246(ba) && ok246(bw)) return true;
+    return (ba == 3 || ba == 4) && (bw == 3 || bw == 4);
+}
+
+static bool values_product_ok(int bw, int d, bool fp8) {
+    if (d % (fp8 ? 128 : 64) != 0) return false;
+    if (bw == 3) return d % 128 == 0;
+    return bw == 2 || bw == 4 || bw == 6;
+}
+
 static oq_status run_qgemm(const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M, int N, const uint8_t* a_idx,
                            const float* s, const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias,
                            uint16_t* y, void* stream, bool fp8) {
     if (!cb_a || !cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != cb_w->d) return OQ_ERR_INVALID_ARG;
-    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits) || cb_a->d % (fp8 ? 128 : 64) != 0)
-        return OQ_ERR_UNSUPPORTED;
-    // 3-bit rows hold 24 bytes per 64 codes, too narrow for the bf16 kernel's TMA step
-    if (!fp8 && (cb_a->bits == 3 || cb_w->bits == 3)) return OQ_ERR_UNSUPPORTED;
-    // 8-bit codes have no in-kernel decoder: 8-bit activations run in the values schedule
-    if (cb_a->bits == 8 || cb_w->bits == 8) return OQ_ERR_UNSUPPORTED;
-    if (fp8 && (cb_a->bits == 3 || cb_w->bits == 3) && !((cb_a->bits == 3 || cb_a->bits == 4) && (cb_w->bits == 3 || cb_w->bits == 4)))
-        return OQ_ERR_UNSUPPORTED;
+    if (!codes_product_ok(cb_a->bits, cb_w->bits, cb_a->d, fp8)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;  // an empty batch: activation and output buffers may be null
     if (!a_idx || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
     if (!aligned16(a_idx) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
@@ -383,8 +411,7 @@ static oq_status run_qgemm_values(const oq_codebook_t* cb_w, int M, int N, const
                                   const uint8_t* w_idx, const uint16_t* w_r, const uint16_t* bias, uint16_t* y,
                                   void* stream, bool fp8) {
     if (!cb_w || M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
-    if (!quant_bits_ok(cb_w->bits) || cb_w->d % (fp8 ? 128 : 64) != 0) return OQ_ERR_UNSUPPORTED;
-    if ((!fp8 && cb_w->bits == 3) || cb_w->bits == 8) return OQ_ERR_UNSUPPORTED;
+    if (!values_product_ok(cb_w->bits, cb_w->d, fp8)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
     if (!a_val || !s || !w_idx || !w_r || !y) return OQ_ERR_INVALID_ARG;
     if (!aligned16(a_val) || !aligned16(s) || !aligned16(w_idx) || !aligned16(w_r) || !aligned16(y) ||
@@ -454,6 +481,34 @@ size_t oq_qlinear_workspace_values(int M, int d) {
     return ((size_t)M * (size_t)d * 2 + 255) / 256 * 256 + ((size_t)M * sizeof(float) + 255) / 256 * 256;
 }
 
+static size_t values_workspace(int M, int d, bool fp8) {
+    return ((size_t)M * (size_t)d * (fp8 ? 1 : 2) + 255) / 256 * 256 + ((size_t)M * sizeof(float) + 255) / 256 * 256;
+}
+
+// The layer's schedule for a workspace of ws_bytes, decided before any
+// launch: values when the values product supports the widths and the
+// workspace holds the values; else codes when the workspace holds the codes
+// (OQ_ERR_UNSUPPORTED if the codes product does not support the widths);
+// else OQ_ERR_OOM, or OQ_ERR_UNSUPPORTED if neither product supports them.
+// *fits_larger tells whether a supported schedule would run with a larger
+// workspace.
+static oq_status choose_schedule(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w, int M,
+                                 size_t ws_bytes, bool fp8, bool* values, bool* fits_larger) {
+    const int d = plan->d;
+    const bool v_ok = values_product_ok(cb_w->bits, d, fp8);
+    const bool c_ok = codes_product_ok(cb_a->bits, cb_w->bits, d, fp8);
+    *fits_larger = v_ok || c_ok;
+    if (v_ok && ws_bytes >= values_workspace(M, d, fp8)) {
+        *values = true;
+        return OQ_OK;
+    }
+    if (ws_bytes >= oq_qlinear_workspace(M, d, cb_a->bits)) {
+        *values = false;
+        return c_ok ? OQ_OK : OQ_ERR_UNSUPPORTED;
+    }
+    return *fits_larger ? OQ_ERR_OOM : OQ_ERR_UNSUPPORTED;
+}
+
 static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, const oq_codebook_t* cb_w,
                              const void* x, oq_dtype dtype, int M, const uint8_t* w_idx, const uint16_t* w_r, int N,
                              const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream,
@@ -461,7 +516,7 @@ static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     if (!plan || !cb_a || !cb_w) return OQ_ERR_INVALID_ARG;
     if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
-    if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
+    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
     if (!workspace) return OQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return OQ_ERR_ALIGNMENT;
@@ -470,23 +525,21 @@ static oq_status run_qlinear(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     // for four (bf16) or two (e4m3) times the bytes of A to stream per tile;
     // with a deep A ring and N-fastest tiles it is the faster one on B200 at
     // every shape measured, so it is taken whenever the workspace holds it.
-    const size_t val_al = ((size_t)M * plan->d * (fp8 ? 1 : 2) + 255) / 256 * 256;
-    if (ws_bytes >= val_al + ((size_t)M * sizeof(float) + 255) / 256 * 256) {
-        if (fp8 && plan->d % 128 != 0) return OQ_ERR_UNSUPPORTED;
+    bool values = false, fits_larger = false;
+    oq_status st = choose_schedule(plan, cb_a, cb_w, M, ws_bytes, fp8, &values, &fits_larger);
+    if (st != OQ_OK) return st;
+    if (values) {
+        const size_t val_al = ((size_t)M * plan->d * (fp8 ? 1 : 2) + 255) / 256 * 256;
         float* s = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + val_al);
-        oq_status st = fp8 ? oq_quantize_acts_values_fp8(plan, cb_a, x, dtype, M, static_cast<uint8_t*>(workspace), s,
-                                                         stream)
-                           : oq_quantize_acts_values(plan, cb_a, x, dtype, M, static_cast<uint16_t*>(workspace), s,
-                                                     stream);
+        st = fp8 ? oq_quantize_acts_values_fp8(plan, cb_a, x, dtype, M, static_cast<uint8_t*>(workspace), s, stream)
+                 : oq_quantize_acts_values(plan, cb_a, x, dtype, M, static_cast<uint16_t*>(workspace), s, stream);
         if (st != OQ_OK) return st;
         return run_qgemm_values(cb_w, M, N, workspace, s, w_idx, w_r, bias, y, stream, fp8);
     }
-    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);
-    if (ws_bytes < need) return OQ_ERR_OOM;
     uint8_t* a_idx = static_cast<uint8_t*>(workspace);
     const size_t idx_al = ((size_t)M * packed_row_bytes(plan->d, cb_a->bits) + 255) / 256 * 256;
     float* s = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + idx_al);
-    oq_status st = oq_quantize_acts(plan, cb_a, x, dtype, M, a_idx, s, stream);
+    st = oq_quantize_acts(plan, cb_a, x, dtype, M, a_idx, s, stream);
     if (st != OQ_OK) return st;
     return run_qgemm(cb_a, cb_w, M, N, a_idx, s, w_idx, w_r, bias, y, stream, fp8);
 }
@@ -538,10 +591,13 @@ oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
     if (!plan || !cb_a || !cb_w) return OQ_ERR_INVALID_ARG;
     if (M < 0 || N <= 0) return OQ_ERR_INVALID_ARG;
     if (cb_a->d != plan->d || cb_w->d != plan->d) return OQ_ERR_INVALID_ARG;
-    if (!quant_bits_ok(cb_a->bits)) return OQ_ERR_UNSUPPORTED;
+    if (!quant_bits_ok(cb_a->bits) || !quant_bits_ok(cb_w->bits)) return OQ_ERR_UNSUPPORTED;
     if (M == 0) return OQ_OK;
-    const size_t need = oq_qlinear_workspace(M, plan->d, cb_a->bits);  // the codes schedule; values when they fit
-    if (need > OQ_NOALLOC_SCRATCH_BYTES) return OQ_ERR_TOO_LARGE;
+    // the schedule the scratch allows, decided before any work: values when
+    // they fit, else codes; a supported request that fits neither is too large
+    bool values = false, fits_larger = false;
+    const oq_status sched = choose_schedule(plan, cb_a, cb_w, M, OQ_NOALLOC_SCRATCH_BYTES, false, &values, &fits_larger);
+    if (sched != OQ_OK) return fits_larger ? OQ_ERR_TOO_LARGE : sched;
     if (current_device() != plan->device) return OQ_ERR_INVALID_ARG;
     // the activation codebook's tables must already be here (its upload would allocate)
     if (!codebook_resident(const_cast<oq_codebook_t*>(cb_a))) return OQ_ERR_INVALID_ARG;
@@ -555,6 +611,12 @@ oq_status oq_qlinear_noalloc(const oq_plan_t* plan, const oq_codebook_t* cb_a, c
 void oq_debug_fail_allocations(int n) { g_fail_allocs.store(n > 0 ? n : 0); }
 
 void oq_debug_starve(int mask) { g_starve_mask.store(mask & (OQ_STARVE_RPBH | OQ_STARVE_GEMM)); }
+
+void oq_debug_rpbh_layout(int rows_per_warp, int slots) {
+    const bool rw_ok = rows_per_warp == 0 || rows_per_warp == 1 || rows_per_warp == 2 || rows_per_warp == 4 ||
+                       rows_per_warp == 8;
+    rpbh_force_layout(rw_ok ? rows_per_warp : 0, (slots == 1 || slots == 2) ? slots : 0);
+}
 
 oq_status oq_device_status(int clear, int* out, void* stream) {
     if (!out) return OQ_ERR_INVALID_ARG;

@@ -242,13 +242,16 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb) {
     float G = (float)(1.0 / min_gap);
     if (L == 2) G = 4.0f;
     const float vmax = 1.0f + 1.0f / 16.0f;  // |v| <= 1 up to fp32 rounding for the rows the kernel quantises
-    for (int tries = 0; tries < 64; ++tries) {
-        bool ok = true;
+    bool separated = false;
+    for (int tries = 0; tries < 64 && !separated; ++tries) {
+        separated = true;
         for (int j = 0; j + 2 < L; ++j)
-            if (bin_of(cb->t32[j], G) >= bin_of(cb->t32[j + 1], G)) ok = false;
-        if (ok) break;
-        G *= 1.25f;
+            if (bin_of(cb->t32[j], G) >= bin_of(cb->t32[j + 1], G)) separated = false;
+        if (!separated) G *= 1.25f;
     }
+    // the kernels' one-compare lookup is exact only with at most one
+    // threshold per bin: refuse the codebook rather than build a wrong table
+    if (!separated) return OQ_ERR_NO_CONVERGENCE;
     cb->G = G;
     const int kmin = bin_of(-vmax, G), kmax = bin_of(vmax, G);
     cb->kmin = kmin;
@@ -317,18 +320,22 @@ void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int var
     for (int k = 0; k < d; ++k) sign[k] = (next() >> 63) ? (int8_t)-1 : (int8_t)1;
 }
 
-// Gather table: entry for post-permutation coordinate k = b*h + i is
-// pi(k) | 0x8000 * (sigma_k < 0).  Stored in 16-byte chunks of 8 entries,
-// chunk (c, b) (entries b*h + 8c .. b*h + 8c + 7) at chunk index c*nb + b, so
-// that threads working on neighbouring blocks read neighbouring chunks.
-void build_gather_table(const oq_plan_t* p, std::vector<uint16_t>& out) {
-    const int d = p->d, h = p->h, nb = d / h, nc = h / 8;
+// Gather table: the entry of post-permutation coordinate k = b*h + i is
+// (2 pi(k)) << 16 | 0x8000 * (sigma_k < 0): the byte offset of the bf16
+// element x[pi(k)] in its row (the fp32 kernel doubles it) and the sign of
+// D_k.  Stored in 16-byte chunks of 4 entries, chunk (c, b) (entries
+// b*h + 4c .. b*h + 4c + 3) at chunk index c*nb + b, so that lanes working on
+// neighbouring blocks read neighbouring chunks.  Offsets fit 16 bits since
+// d <= 32767.
+void build_gather_table(const oq_plan_t* p, std::vector<uint32_t>& out) {
+    const int d = p->d, h = p->h, nb = d / h, nc = h / 4;
     out.assign(d, 0);
     for (int b = 0; b < nb; ++b)
         for (int c = 0; c < nc; ++c)
-            for (int e = 0; e < 8; ++e) {
-                const int k = b * h + c * 8 + e;
-                out[(size_t)(c * nb + b) * 8 + e] = (uint16_t)(p->perm[k] | (p->sign[k] < 0 ? 0x8000 : 0));
+            for (int e = 0; e < 4; ++e) {
+                const int k = b * h + c * 4 + e;
+                out[(size_t)(c * nb + b) * 4 + e] =
+                    ((uint32_t)(2 * p->perm[k]) << 16) | (p->sign[k] < 0 ? 0x8000u : 0u);
             }
 }
 

@@ -29,7 +29,7 @@ struct DeviceCodebook {
 };
 
 struct DevicePlan {
-    uint16_t* gtab = nullptr;  // device gather table (see plan.cpp)
+    uint32_t* gtab = nullptr;  // device gather table (see build_gather_table)
 };
 
 }  // namespace oq
@@ -58,7 +58,7 @@ struct oq_plan_s {
     int device = -1;
     std::vector<int32_t> perm;
     std::vector<int8_t> sign;
-    std::vector<uint16_t> gtab_host;  // chunked gather table (see plan.cpp)
+    std::vector<uint32_t> gtab_host;  // chunked gather table (see build_gather_table)
     oq::DevicePlan dev;
 };
 
@@ -68,7 +68,7 @@ namespace oq {
 oq_status build_codebook(int d, int bits, oq_codebook_t* cb);
 void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int variant);
 uint8_t e4m3_round(double v);
-void build_gather_table(const oq_plan_t* p, std::vector<uint16_t>& out);
+void build_gather_table(const oq_plan_t* p, std::vector<uint32_t>& out);
 uint16_t bf16_round(double x);
 
 // device-side pieces (api.cu)

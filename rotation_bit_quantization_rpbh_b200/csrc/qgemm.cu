@@ -24,7 +24,8 @@
 //   warps 2-17  decoders, two groups taking alternate K steps: expand
 //               packed 2/3/4/6-bit codes to centroid values (register
 //               byte-permute lookups; 64-entry static shared tables for 6-bit
-//               codes; 3-bit codes in the fp8 variant only)
+//               codes; 3-bit codes from a 48-byte box per aligned
+//               pair of K steps in the bf16 variant)
 //               into a 4-stage ring in the 128-byte-swizzled K-major
 //               layout, then signal the leader's "stage full" barrier: the
 //               leader's own warps arrive, the peer's warps complete
@@ -86,7 +87,20 @@ constexpr int DEC_A = HM * 128, DEC_B = HN * 128, DEC_STAGE = DEC_A + DEC_B;
 // A K step fills one 128-byte row of each decoded operand: 64 bf16 values,
 // or 128 e4m3 values in the fp8 variant.
 __host__ __device__ constexpr int bk_codes(bool f8) { return f8 ? 128 : 64; }
-__host__ __device__ constexpr int pk_row_bytes(int bits, bool f8) { return bits == 6 ? bk_codes(f8) : bk_codes(f8) * bits / 8; }
+// Packed bytes per row and K step.  3-bit codes in the bf16 variant: 64
+// codes are 24 bytes, narrower than a TMA box may be, so each K step loads
+// the 48-byte box of the aligned step pair that holds it (128 codes) and
+// decodes its own half.
+__host__ __device__ constexpr bool pair_box(int bits, bool f8) { return bits == 3 && !f8; }
+__host__ __device__ constexpr int pk_row_bytes(int bits, bool f8) {
+    return pair_box(bits, f8) ? 48 : (bits == 6 ? bk_codes(f8) : bk_codes(f8) * bits / 8);
+}
+// byte coordinate of K step kb's box in a packed row
+__host__ __device__ constexpr int pk_box_x(int bits, bool f8, int kb) {
+    return pair_box(bits, f8) ? (kb >> 1) * 48 : kb * pk_row_bytes(bits, f8);
+}
+// offset of K step kb's codes inside its box
+__host__ __device__ constexpr int pk_half_off(int bits, bool f8, int kb) { return pair_box(bits, f8) ? (kb & 1) * 24 : 0; }
 // packed bytes behind one 16-byte decoded chunk (8 bf16 or 16 e4m3 values)
 __host__ __device__ constexpr int unit_bytes(int bits, bool f8) { return (f8 ? 16 : 8) * (bits == 6 ? 8 : bits) / 8; }
 // With A given as values (av) the decoded ring holds W only and the packed
@@ -410,7 +424,11 @@ template <int BITS, bool F8>
 __device__ __forceinline__ PackedU<BITS, F8> load_unit(const uint8_t* src) {
     PackedU<BITS, F8> u;
     constexpr int NB = PackedU<BITS, F8>::NB;
-    if constexpr (NB == 2) {
+    if constexpr (NB == 3) {  // 8 3-bit codes at any byte offset: the two words around them, funnel-shifted
+        const uintptr_t a = reinterpret_cast<uintptr_t>(src);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
+        u.w[0] = __funnelshift_r(w[0], w[1], (uint32_t)(a & 3u) * 8u) & 0xFFFFFFu;
+    } else if constexpr (NB == 2) {
         u.w[0] = *reinterpret_cast<const uint16_t*>(src);
     } else if constexpr (NB == 6) {  // 16 3-bit codes at a 2-byte-aligned offset
         const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
@@ -432,12 +450,29 @@ __device__ __forceinline__ PackedU<BITS, F8> load_unit(const uint8_t* src) {
     return u;
 }
 
+// 3-bit codes to bf16: the 24 bits of 8 codes are spread to 8 nibbles,
+// which select the high bytes of c_0..c_7 (tab words 0-1) and their low
+// bytes (words 2-3); two more permutes interleave them into bf16 pairs.
+__device__ __forceinline__ uint4 decode8_3bit(uint32_t x, const uint32_t tab[4]) {
+    const uint32_t y = spread3to4(x);
+    uint32_t out[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint32_t sel = half ? (y >> 16) : (y & 0xFFFFu);
+        const uint32_t hi = prmt(tab[0], tab[1], sel);
+        const uint32_t lo = prmt(tab[2], tab[3], sel);
+        out[2 * half] = prmt(lo, hi, 0x5140u);
+        out[2 * half + 1] = prmt(lo, hi, 0x7362u);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 template <int BITS, int TAB, bool F8>
 __device__ __forceinline__ uint4 decode_unit(const PackedU<BITS, F8>& u, const uint32_t tab[4]) {
-    static_assert(BITS != 3 || F8, "3-bit codes run in the fp8 variant only");
     if constexpr (!F8) {
         if constexpr (BITS == 4) return decode8_4bit(u.w[0], tab);
         else if constexpr (BITS == 2) return decode8_2bit(u.w[0], tab);
+        else if constexpr (BITS == 3) return decode8_3bit(u.w[0], tab);
         else return decode8_6bit<TAB>(u.w[0], u.w[1]);
     } else {
         if constexpr (BITS == 4) {
@@ -463,11 +498,14 @@ struct StageCodes {
 };
 
 // (AV: A arrives as values, so only W's codes are loaded and expanded)
+// (kb: the K step, which picks the half of a 3-bit pair box)
 template <int BA, int BW, bool F8, bool AV>
 __device__ __forceinline__ void load_codes(StageCodes<BA, BW, F8>& u, const uint8_t* pa, const uint8_t* pb, int srcA,
-                                           int srcB) {
+                                           int srcB, int kb) {
     constexpr int PKRA = pk_row_bytes(BA, F8), PKRB = pk_row_bytes(BW, F8);
     constexpr int NUA = AV ? 0 : DEC_UNITS;
+    pa += pk_half_off(BA, F8, kb);
+    pb += pk_half_off(BW, F8, kb);
 #pragma unroll
     for (int i = 0; i < NUA; ++i) u.a[i] = load_unit<BA, F8>(pa + srcA + i * DEC_ROWS * PKRA);
 #pragma unroll
@@ -604,6 +642,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above overlaps the end of the kernel before this one in the
+    // stream (launched with programmatic serialisation); every read of the
+    // operands, norms and bias and every write of y comes after this wait.
+    if (tid == 0) grid_launch_dependents();
+    grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -624,8 +667,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     }
                     mbar_arrive_expect_tx(&pk_full[ps.idx], PK_STAGE);
                     uint8_t* dst = pk + ps.idx * PK_STAGE;
-                    if constexpr (!AV) tma_load_2d(dst, &p.tmA, kb * pk_row_bytes(BA, F8), m0, &pk_full[ps.idx]);
-                    tma_load_2d(dst + PKA, &p.tmB, kb * pk_row_bytes(BW, F8), n0, &pk_full[ps.idx]);
+                    if constexpr (!AV) tma_load_2d(dst, &p.tmA, pk_box_x(BA, F8, kb), m0, &pk_full[ps.idx]);
+                    tma_load_2d(dst + PKA, &p.tmB, pk_box_x(BW, F8, kb), n0, &pk_full[ps.idx]);
                     ++issued;
                     ps.advance();
                     if constexpr (AV) {
@@ -749,7 +792,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         StageCodes<BA, BW, F8> cur;
         bool ok = grp < total && wait_or_abort<false>(&pk_full[ps.idx], 0u, abort_flag);
         if (ok) {
-            load_codes<BA, BW, F8, AV>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB);
+            load_codes<BA, BW, F8, AV>(cur, pk + ps.idx * PK_STAGE, pk + ps.idx * PK_STAGE + PKA, srcA, srcB,
+                                       grp % p.KB);
             __syncwarp();
             if (lane == 0) mbar_arrive(&pk_empty[ps.idx]);
         }
@@ -763,7 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 const uint8_t* pa = pk + ps.idx * PK_STAGE;
-                load_codes<BA, BW, F8, AV>(nxt, pa, pa + PKA, srcA, srcB);
+                load_codes<BA, BW, F8, AV>(nxt, pa, pa + PKA, srcA, srcB, (s + NGROUPS) % p.KB);
             }
             StageValues v;
             decode_codes<BA, BW, F8, AV>(v, cur, tab_a, tab_w);
@@ -891,8 +935,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows,
-               bool swizzle128 = false) {
+bool encode_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows,
+                 bool swizzle128) {
     auto fn = get_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
@@ -904,6 +948,46 @@ bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int b
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Tensor maps are encoded on the host (a driver call of a few microseconds);
+// layer calls repeat the same operands, so the last few encodings are kept,
+// keyed by everything that goes into them.  Device addresses are unique
+// across the process's devices (unified addressing).
+struct TmapKey {
+    const void* base;
+    int rows, row_bytes, box_cols, box_rows;
+    bool swizzle128;
+    bool operator==(const TmapKey& o) const {
+        return base == o.base && rows == o.rows && row_bytes == o.row_bytes && box_cols == o.box_cols &&
+               box_rows == o.box_rows && swizzle128 == o.swizzle128;
+    }
+};
+
+bool make_tmap(CUtensorMap* tm, const void* base, int rows, int row_bytes, int box_cols, int box_rows,
+               bool swizzle128 = false) {
+    constexpr int kSlots = 32;
+    static std::mutex mu;
+    static TmapKey keys[kSlots];
+    static CUtensorMap maps[kSlots];
+    static bool used[kSlots] = {false};
+    static int next = 0;
+    const TmapKey key{base, rows, row_bytes, box_cols, box_rows, swizzle128};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < kSlots; ++i)
+            if (used[i] && keys[i] == key) {
+                *tm = maps[i];
+                return true;
+            }
+    }
+    if (!encode_tmap(tm, base, rows, row_bytes, box_cols, box_rows, swizzle128)) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    keys[next] = key;
+    maps[next] = *tm;
+    used[next] = true;
+    next = (next + 1) % kSlots;
+    return true;
 }
 
 // Byte-permute tables of the register decoders (see decode8_4bit and
@@ -923,6 +1007,12 @@ void fill_tables(int bits, const uint16_t* cb, uint32_t tab[4], uint16_t* c6) {
         for (int j = 0; j < 4; ++j) {
             tab[0] |= (uint32_t)(cb[j] & 0xffu) << (8 * j);
             tab[1] |= (uint32_t)((cb[j] >> 8) & 0xffu) << (8 * j);
+        }
+    } else if (bits == 3) {
+        // high bytes of c_0..c_7 in words 0-1, low bytes in words 2-3 (see decode8_3bit)
+        for (int j = 0; j < 8; ++j) {
+            tab[j / 4] |= ((uint32_t)(cb[j] >> 8) & 0xffu) << (8 * (j % 4));
+            tab[2 + j / 4] |= ((uint32_t)cb[j] & 0xffu) << (8 * (j % 4));
         }
     } else {
         for (int j = 0; j < 64; ++j) c6[j] = cb[j];
@@ -950,9 +1040,10 @@ template <int BA, int BW, bool F8, bool AV = false>
 cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
     auto k = qgemm_kernel<BA, BW, F8, AV>;
     const int smem = smem_bytes(BA, BW, F8, AV);
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t e = ensure_smem_limit(k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, NTHREADS, smem, stream>>>(prm);
+    const cudaError_t le = launch_pdl(k, dim3(grid), dim3(NTHREADS), smem, stream, prm);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -962,15 +1053,13 @@ cudaError_t launch_bits(const QgemmArgs& a, QgemmParams& prm, int grid, cudaStre
         if (a.bits_w == 4) return launch_qgemm_t<0, 4, F8, true>(prm, grid, stream);
         if (a.bits_w == 2) return launch_qgemm_t<0, 2, F8, true>(prm, grid, stream);
         if (a.bits_w == 6) return launch_qgemm_t<0, 6, F8, true>(prm, grid, stream);
-        if constexpr (F8)
-            if (a.bits_w == 3) return launch_qgemm_t<0, 3, true, true>(prm, grid, stream);
+        if (a.bits_w == 3) return launch_qgemm_t<0, 3, F8, true>(prm, grid, stream);
         return cudaErrorInvalidValue;
     }
-    if constexpr (F8) {  // 3-bit codes: the fp8 variant only
-        if (a.bits_a == 3 && a.bits_w == 3) return launch_qgemm_t<3, 3, true>(prm, grid, stream);
-        if (a.bits_a == 3 && a.bits_w == 4) return launch_qgemm_t<3, 4, true>(prm, grid, stream);
-        if (a.bits_a == 4 && a.bits_w == 3) return launch_qgemm_t<4, 3, true>(prm, grid, stream);
-    }
+    // 3-bit codes pair with 3- or 4-bit codes
+    if (a.bits_a == 3 && a.bits_w == 3) return launch_qgemm_t<3, 3, F8>(prm, grid, stream);
+    if (a.bits_a == 3 && a.bits_w == 4) return launch_qgemm_t<3, 4, F8>(prm, grid, stream);
+    if (a.bits_a == 4 && a.bits_w == 3) return launch_qgemm_t<4, 3, F8>(prm, grid, stream);
 #define OQ_CASE(X, Y) \
     if (a.bits_a == X && a.bits_w == Y) return launch_qgemm_t<X, Y, F8>(prm, grid, stream);
     OQ_CASE(4, 4)

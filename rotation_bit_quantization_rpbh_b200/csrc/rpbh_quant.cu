@@ -8,20 +8,27 @@
 // W' = W Pi_d^T is Pi_d w_n) and stores r_n as bf16.
 //
 // Design (sm_100a, HBM-bound):
-//   - persistent CTAs, one per SM, each split into NG (1-4) warp groups that
-//     take interleaved tiles of R rows and run out of phase (own staging buffers,
-//     mbarriers and named barriers), so one group's gathers overlap the
-//     others' butterflies and table lookups; a group stages its rows with
-//     1-D bulk copies (cp.async.bulk), double buffered so its next tile
-//     streams in while this one is computed;
-//   - the gather and lookup tables arrive by bulk copy together with each
-//     group's first rows;
-//   - thread (r, b) owns row r's h-block b: it gathers the block's h inputs
-//     x[pi(k)] from the staged row (the sign D is the gather table entry's
-//     top bit, XORed into the bf16 sign) and runs the whole Walsh-Hadamard
-//     butterfly in registers (packed f32x2 adds).  The row norm is the norm
-//     of the gathered inputs (Pi_d is orthogonal, so ||x'|| = ||x||): its
-//     cross-warp reduction is posted before the butterflies and read after;
+//   - persistent CTAs, one per SM.  A lane owns one (row, h-block) unit: a
+//     warp covers RW rows x 32/RW blocks, and a team of warps covers all the
+//     blocks of a set of RW rows.  Teams run independently: each has its own
+//     staging slots (a row set arrives by one 1-D bulk copy per row into a
+//     slot, completing on that slot's mbarrier) and the team's first warp
+//     refills a slot with the team's next row set as soon as every warp of
+//     the team has gathered from it, so the copy overlaps the butterflies
+//     and the table lookups.  There is no CTA-wide barrier in the loop.
+//   - rows of a slot are padded so that the RW rows a warp gathers from fall
+//     on different banks; several rows per warp make the random gather of a
+//     warp touch fewer words per bank than 32 random columns of one row;
+//   - the gather table holds, per post-permutation coordinate k, the byte
+//     offset of x[pi(k)] in the row and the sign of D (bit 15), so the sign
+//     flip and the bf16 -> fp32 widening are one add and one shift; the RW
+//     lanes of one block read the same table words (a broadcast);
+//   - the lane runs the whole Walsh-Hadamard butterfly in registers (packed
+//     f32x2 adds).  The row norm is the norm of the gathered inputs (Pi_d is
+//     orthogonal, so ||x'|| = ||x||): it is summed across the block's lanes
+//     by shuffles and across the team's warps through shared memory and a
+//     per-team mbarrier, in a fixed order (deterministic), and the exchange
+//     overlaps the butterflies;
 //   - quantisation needs no search: bin(v) = rint(v G) (one fmaf with a
 //     magic constant) indexes a small table holding, per bin, the count of
 //     thresholds below it and the one threshold inside it, so
@@ -34,6 +41,9 @@
 //     centroid values of the bin's two possible cells (bf16 or e4m3 of
 //     c sqrt(d)), so the same compare selects C[index] itself, written as
 //     bf16 pairs or e4m3 quads, 16 bytes at a time.
+// Every mbarrier wait is bounded; a wait that runs out raises the device
+// error flag and a CTA-wide abort flag, every warp leaves its loop, and the
+// copies this CTA issued are drained (bounded) before it exits.
 #include <cuda_bf16.h>
 
 #include "device_util.cuh"
@@ -47,19 +57,22 @@ namespace {
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 struct SmemLayout {
-    int gtab, lut, stage, red, bar, total;
+    int gtab, lut, stage, part, bar, flag, total;
 };
 
-// gather table (u16 entries) | lookup table | NG groups x 2 staging buffers
-// of R rows | NG groups' norm partials | mbarriers (2 per group + tables)
+// gather table (u32 entries) | lookup table | tpc teams x slots x RW staged
+// rows | norm partials (tpc teams x 2 row sets x team warps x RW rows) |
+// mbarriers (tables, full and empty per slot, norm per team and parity) |
+// abort flag
 __host__ __device__ inline SmemLayout smem_layout(const RpbhParams& p) {
     SmemLayout L;
     L.gtab = 0;
-    L.lut = align_up(p.d * 2, 16);
+    L.lut = align_up(p.d * 4, 16);
     L.stage = align_up(L.lut + p.lut_n * 8, 128);
-    L.red = L.stage + p.NG * 2 * p.R * p.srow;
-    L.bar = align_up(L.red + p.NG * (p.G / 32) * p.R * 4, 8);
-    L.total = L.bar + 8 * (2 * p.NG + 1);
+    L.part = L.stage + p.tpc * p.slots * p.RW * p.srow;
+    L.bar = align_up(L.part + p.tpc * 2 * p.team * p.RW * 4, 8);
+    L.flag = L.bar + 8 * (1 + 2 * p.tpc * p.slots + 2 * p.tpc);
+    L.total = L.flag + 16;
     return L;
 }
 
@@ -69,163 +82,258 @@ __device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t se
     return d;
 }
 
-__device__ __forceinline__ void group_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+// Bounded wait that also gives up once another warp of the CTA aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicExch(&g_error_flag, kErrTimeout);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// The same, by every lane of the warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    const bool ok = wait_or_abort(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Lookup-table entry at a 32-bit shared-memory address: {T, base or values}.
+__device__ __forceinline__ void lut_ld(uint32_t addr, float& T, uint32_t& w) {
+    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T), "=r"(w) : "r"(addr));
+}
+
+// Shared-memory loads at 32-bit shared addresses (explicit ld.shared: the
+// staged rows change between iterations, so these are ordered after the
+// mbarrier waits by being volatile).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
 }
 
 template <typename InT, int H, int BITS, int MODE>
-__global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhParams p) {
+__global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid_constant__ RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
-    const uint16_t* s_gtab = reinterpret_cast<const uint16_t*>(smem + L.gtab);
-    __shared__ int s_abort[kMaxGroups];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+    uint64_t* tab_bar = bars;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flag);
 
-    // NG warp groups per CTA work through interleaved tiles independently
-    // (own staging buffers, mbarriers and named barrier), so one group's
-    // gathers overlap the others' butterflies and table lookups.
-    const int tid = threadIdx.x;
-    const int G = p.G, R = p.R, nb = p.nb, NG = p.NG;
-    const int grp = tid / G;
-    const int tg = tid - grp * G;
-    const int r = tg & (R - 1);
-    const int b = tg / R;
-    const bool active = b < nb;
-    const int lane = tg & 31, warp = tg >> 5, nwarps = G >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = warp / p.team, wt = warp - t * p.team;  // team, warp within the team
+    const int Bw = 1 << p.lbw;
+    const int j = lane & (Bw - 1), r = lane >> p.lbw;     // block within the warp, row within the set
+    const int b = wt * Bw + j;                            // h-block of this lane
+    const bool bact = b < p.nb;
+    const bool loader = wt == 0 && lane == 0;             // issues the team's row copies
+    uint64_t* my_full = bars + 1 + t * p.slots;
+    uint64_t* my_empty = bars + 1 + p.tpc * p.slots + t * p.slots;
+    uint64_t* my_norm = bars + 1 + 2 * p.tpc * p.slots + 2 * t;
+    uint8_t* my_stage = smem + L.stage + t * p.slots * p.RW * p.srow;
+    float* my_part = reinterpret_cast<float*>(smem + L.part) + t * 2 * p.team * p.RW;
     constexpr int ES = sizeof(InT);
-    uint8_t* s_stage = smem + L.stage + grp * 2 * R * p.srow;
-    float* s_red = reinterpret_cast<float*>(smem + L.red) + grp * nwarps * R;
-    uint64_t* all_bars = reinterpret_cast<uint64_t*>(smem + L.bar);
-    uint64_t* s_bar = all_bars + 2 * grp;
-    uint64_t* tab_bar = all_bars + 2 * NG;
+    constexpr int L2H = H / 2;
 
-    // returns whether a copy was issued; a starved launch (test hook) issues
-    // none, so the stage waits below run out and report a timeout
-    auto issue = [&](uint64_t* bars, uint8_t* stage, int tile, int st) -> int {
-        if (p.starve) return 0;
-        const int row0 = tile * R;
-        const int rows = min(R, p.M - row0);
-        mbar_arrive_expect_tx(&bars[st], (uint32_t)(rows * p.row_bytes));
-        const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
-        uint8_t* dst = stage + st * R * p.srow;
-        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, &bars[st]);
-        return 1;
-    };
+    // this team's row sets: g = k * (gridDim.x * tpc) + t * gridDim.x + blockIdx.x
+    const int stride = gridDim.x * p.tpc;
+    const int g0 = t * gridDim.x + blockIdx.x;
 
-    // this group's tiles: blockIdx.x + (NG k + grp) * gridDim.x
-    const int step = NG * gridDim.x;
-    int tile = blockIdx.x + grp * gridDim.x;
+    // Launched with programmatic serialisation: the set-up above may overlap
+    // the end of the kernel before this one in the stream; every global
+    // access (tables, rows, outputs) comes after this wait.
+    if (tid == 0) grid_launch_dependents();
+    grid_dependency_wait();
+
     if (tid == 0) {
-        for (int i = 0; i < 2 * NG + 1; ++i) mbar_init(&all_bars[i], 1);
+        const int nbar = 1 + 2 * p.tpc * p.slots + 2 * p.tpc;
+        for (int i = 0; i < nbar; ++i) {
+            const bool team_count = i >= 1 + p.tpc * p.slots;  // empty and norm barriers: one arrival per warp
+            mbar_init(&bars[i], team_count ? (uint32_t)p.team : 1u);
+        }
+        *abort_flag = 0;
         fence_mbar_init();
-        for (int g = 0; g < kMaxGroups; ++g) s_abort[g] = 0;
-        // gather and lookup tables, then each group's first rows: all in flight together
-        const uint32_t lut_bytes = (uint32_t)(p.lut_n * 8);
-        mbar_arrive_expect_tx(tab_bar, (uint32_t)(p.d * 2) + lut_bytes);
-        bulk_g2s(smem + L.gtab, p.gtab, (uint32_t)(p.d * 2), tab_bar);
-        if (lut_bytes) bulk_g2s(smem + L.lut, p.lut, lut_bytes, tab_bar);
-        for (int g = 0; g < NG; ++g) {
-            const int t0 = blockIdx.x + g * gridDim.x;
-            if (t0 < p.ntiles) issue(all_bars + 2 * g, smem + L.stage + g * 2 * R * p.srow, t0, 0);
+        if (!p.starve) {
+            const uint32_t gbytes = (uint32_t)(p.d * 4), lbytes = (uint32_t)(p.lut_n * 8);
+            mbar_arrive_expect_tx(tab_bar, gbytes + lbytes);
+            bulk_g2s(smem + L.gtab, p.gtab, gbytes, tab_bar);
+            if (lbytes) bulk_g2s(smem + L.lut, p.lut, lbytes, tab_bar);
         }
     }
     __syncthreads();  // barriers initialised
 
+    // loader: copy row set g into slot `slot` (a starved launch copies nothing)
+    int issued_k[2] = {-1, -1};  // iteration whose rows were last copied into each slot
+    auto issue = [&](int slot, int g, int k) {
+        if (p.starve) return;
+        const int row0 = g * p.RW;
+        const int rows = min(p.RW, p.M - row0);
+        uint64_t* bar = &my_full[slot];
+        mbar_arrive_expect_tx(bar, (uint32_t)(rows * p.row_bytes));
+        const uint8_t* src = static_cast<const uint8_t*>(p.x) + (size_t)row0 * p.row_bytes;
+        uint8_t* dst = my_stage + slot * p.RW * p.srow;
+        for (int i = 0; i < rows; ++i) bulk_g2s(dst + i * p.srow, src + (size_t)i * p.row_bytes, p.row_bytes, bar);
+        issued_k[slot] = k;
+    };
+    if (loader)
+        for (int i = 0; i < p.slots; ++i)
+            if (g0 + i * stride < p.nrs) issue(i, g0 + i * stride, i);
+
     const float2 G2 = make_float2(p.G_lut, p.G_lut);
     const float2 M2 = make_float2(kLutMagic, kLutMagic);
-    // shared address of lut[(bits of the magic-biased value) + lut_off], folded into one multiply-add
+    // shared address of lut[(bits of the magic-biased value) + lut_off]
     const uint32_t lut_addr0 = smem_u32(smem) + (uint32_t)L.lut + (uint32_t)p.lut_off * 8u;
-    constexpr int L2H = H / 2;
-    int pending_other = 0;  // group leader: a copy into the other stage is in flight
+    const uint32_t gtab_addr = smem_u32(smem) + (uint32_t)L.gtab;  // table chunks, 16 bytes each
+    const uint32_t stage_addr = smem_u32(my_stage);
 
-    for (int it = 0; tile < p.ntiles; tile += step, ++it) {
-        const int st = it & 1;
-        const int next = tile + step;
-        pending_other = 0;
-        if (tg == 0 && next < p.ntiles) {
-            pending_other = issue(s_bar, s_stage, next, st ^ 1);  // streams in while this tile is computed
+    // a slot refill that waits for the team's gathers (loader only)
+    int pend_slot = -1, pend_g = 0, pend_k = 0;
+    uint32_t pend_ph = 0;
+    int consumed_k = -1;  // last iteration whose rows this warp waited for
+    bool ok = true;
+    int k = 0;
+    for (int g = g0; g < p.nrs; g += stride, ++k) {
+        const int slot = p.slots == 1 ? 0 : (k & 1);
+        const uint32_t ph = (uint32_t)((p.slots == 1 ? k : (k >> 1)) & 1);
+        // a deferred refill must be issued before this wait (with one slot it is this one)
+        if (loader && pend_slot >= 0) {
+            if (wait_or_abort(&my_empty[pend_slot], pend_ph, abort_flag)) issue(pend_slot, pend_g, pend_k);
+            else ok = false;
+            pend_slot = -1;
         }
-        if (it == 0 && !mbar_wait_bounded(tab_bar, 0u)) s_abort[grp] = 1;
-        if (!mbar_wait_bounded(&s_bar[st], (uint32_t)((it >> 1) & 1))) s_abort[grp] = 1;
-        group_sync(1 + grp, G);
-        if (s_abort[grp]) {
-            // give the prefetch into the other stage (bounded) time to land
-            // before this CTA's shared memory goes away
-            if (tg == 0 && pending_other) mbar_wait_bounded(&s_bar[st ^ 1], (uint32_t)(((it + 1) >> 1) & 1));
+        if (wt == 0) ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (k == 0 && !warp_wait(tab_bar, 0u, abort_flag)) {
+            ok = false;
             break;
         }
+        if (!warp_wait(&my_full[slot], ph, abort_flag)) {
+            ok = false;
+            break;
+        }
+        consumed_k = k;
 
-        const int row = tile * R + r;
-        const bool valid = active && row < p.M;
+        const int row = g * p.RW + r;
+        const bool valid = bact && row < p.M;
 
-        // ---- A1 + A2: gather sigma_k x[pi(k)] (sign = top bit of the entry) ----
-        // and the sum of squares of the gathered values: ||x'|| = ||x|| since
-        // Pi_d is orthogonal, so the row norm is reduced across the row's
-        // threads while the butterflies run
+        // ---- A1 + A2: gather sigma_k x[pi(k)] and the sum of squares -------
+        // (||x'|| = ||x|| since Pi_d is orthogonal)
         float2 v2[L2H];
         float2 acc = make_float2(0.f, 0.f);
         if (valid) {
-            const uint32_t rowp = smem_u32(s_stage) + (uint32_t)(st * R * p.srow + r * p.srow);
+            const uint32_t rowp = stage_addr + (uint32_t)(slot * p.RW * p.srow + r * p.srow);
+            const uint32_t tabp = gtab_addr + (uint32_t)b * 16u;
 #pragma unroll
-            for (int c = 0; c < H / 8; ++c) {
-                const uint4 ch = reinterpret_cast<const uint4*>(s_gtab)[c * nb + b];
-                const uint32_t w[4] = {ch.x, ch.y, ch.z, ch.w};
+            for (int c4 = 0; c4 < H / 4; ++c4) {
+                // entries 4 c4 .. 4 c4 + 3 of block b (chunk c4 * nb + b)
+                const uint4 ch = lds_v4(tabp + (uint32_t)(c4 * p.nb) * 16u);
+                const uint32_t e[4] = {ch.x, ch.y, ch.z, ch.w};
+                float f[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t e0 = w[e], e1 = w[e] >> 16;  // entry k in the low half, k+1 in the high half
-                    float f0, f1;
+                for (int q = 0; q < 4; ++q) {
+                    // entry: byte offset of x[pi(k)] (bf16 element) in bits 16-31, sign of D in bit 15
                     if constexpr (ES == 2) {
-                        uint32_t r0, r1;
-                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r0) : "r"(rowp + ((e0 & 0x7fffu) << 1)));
-                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(r1) : "r"(rowp + ((e1 & 0x7fffu) << 1)));
-                        // bf16 -> fp32 with the sign flipped where the entry's top bit is set
-                        f0 = __uint_as_float((r0 ^ (e0 & 0x8000u)) << 16);
-                        f1 = __uint_as_float((r1 ^ (e1 & 0x8000u)) << 16);
+                        const uint32_t rv = lds_u16(rowp + (e[q] >> 16));
+                        f[q] = __uint_as_float((rv + e[q]) << 16);  // bit 15 of e flips the sign; the rest shifts out
                     } else {
-                        uint32_t r0, r1;
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r0) : "r"(rowp + ((e0 & 0x7fffu) << 2)));
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r1) : "r"(rowp + ((e1 & 0x7fffu) << 2)));
-                        f0 = __uint_as_float(r0 ^ ((e0 & 0x8000u) << 16));
-                        f1 = __uint_as_float(r1 ^ ((e1 & 0x8000u) << 16));
+                        const uint32_t rv = lds_u32(rowp + ((e[q] >> 16) << 1));
+                        f[q] = __uint_as_float(rv ^ (e[q] << 16));
                     }
-                    v2[c * 4 + e] = make_float2(f0, f1);
-                    acc = f2fma(v2[c * 4 + e], v2[c * 4 + e], acc);
                 }
+                v2[2 * c4] = make_float2(f[0], f[1]);
+                v2[2 * c4 + 1] = make_float2(f[2], f[3]);
+                acc = f2fma(v2[2 * c4], v2[2 * c4], acc);
+                acc = f2fma(v2[2 * c4 + 1], v2[2 * c4 + 1], acc);
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < L2H; ++j) v2[j] = make_float2(0.f, 0.f);
+            for (int i = 0; i < L2H; ++i) v2[i] = make_float2(0.f, 0.f);
+        }
+        // this warp is done with the slot
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&my_empty[slot]);
+        // loader: refill the slot with the team's row set k + slots once every
+        // warp has gathered from it (now if they have, else later)
+        const int gn = g + p.slots * stride;
+        if (loader && gn < p.nrs) {
+            if (mbar_try_wait(&my_empty[slot], ph)) {
+                issue(slot, gn, k + p.slots);
+            } else {
+                pend_slot = slot;
+                pend_ph = ph;
+                pend_g = gn;
+                pend_k = k + p.slots;
+            }
         }
 
-        // ---- A4 (first half): this block's sum of squares, summed over the
-        // row's blocks within the warp, one partial per warp and row ----------
+        // ---- A4 (first half): the row's sum of squares over this warp's blocks ----
         float ss = acc.x + acc.y;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
-            if (o >= R) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane < R) s_red[warp * R + lane] = ss;
+        for (int o = 1; o < Bw; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        float* part = my_part + (k & 1) * p.team * p.RW;
+        if (p.team > 1) {
+            if (j == 0) part[wt * p.RW + r] = ss;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&my_norm[k & 1]);
+        }
 
         // ---- A3: unnormalised Walsh-Hadamard butterflies, Sylvester order ------
 #pragma unroll
-        for (int j = 0; j < L2H; ++j) {
-            const float a = v2[j].x, c = v2[j].y;
-            v2[j] = make_float2(a + c, a - c);
+        for (int i = 0; i < L2H; ++i) {
+            const float a = v2[i].x, c = v2[i].y;
+            v2[i] = make_float2(a + c, a - c);
         }
 #pragma unroll
         for (int hl = 1; hl < L2H; hl <<= 1) {
 #pragma unroll
-            for (int j = 0; j < L2H; ++j) {
-                if ((j & hl) == 0) {
-                    const float2 a = v2[j], c = v2[j + hl];
-                    v2[j] = f2add(a, c);
-                    v2[j + hl] = f2sub(a, c);
+            for (int i = 0; i < L2H; ++i) {
+                if ((i & hl) == 0) {
+                    const float2 a = v2[i], c = v2[i + hl];
+                    v2[i] = f2add(a, c);
+                    v2[i + hl] = f2sub(a, c);
                 }
             }
         }
 
-        // ---- A4 (second half): the row norm s = ||x'|| ------------------------
-        group_sync(1 + grp, G);
-        float ssum = 0.f;
-        for (int w = 0; w < nwarps; ++w) ssum += s_red[w * R + r];
+        // a deferred refill may be possible by now
+        if (loader && pend_slot >= 0 && mbar_try_wait(&my_empty[pend_slot], pend_ph)) {
+            issue(pend_slot, pend_g, pend_k);
+            pend_slot = -1;
+        }
+
+        // ---- A4 (second half): the row norm s = ||x'||, summed in team order ----
+        float ssum = ss;
+        if (p.team > 1) {
+            if (!warp_wait(&my_norm[k & 1], (uint32_t)((k >> 1) & 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            ssum = 0.f;
+            const uint32_t pa = smem_u32(part) + (uint32_t)r * 4u;
+            for (int w2 = 0; w2 < p.team; ++w2) ssum += lds_f32(pa + (uint32_t)(w2 * p.RW) * 4u);
+        }
         const float s = __fsqrt_rn(ssum);
 
         if (valid) {
@@ -238,9 +346,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                 float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + b * H);
                 const float2 sc = make_float2(p.rsqrt_h, p.rsqrt_h);
 #pragma unroll
-                for (int j = 0; j < L2H; j += 2) {
-                    const float2 a = f2mul(v2[j], sc), c = f2mul(v2[j + 1], sc);
-                    yo[j >> 1] = make_float4(a.x, a.y, c.x, c.y);
+                for (int i = 0; i < L2H; i += 2) {
+                    const float2 a = f2mul(v2[i], sc), c = f2mul(v2[i + 1], sc);
+                    yo[i >> 1] = make_float4(a.x, a.y, c.x, c.y);
                 }
             } else if constexpr (MODE >= 3) {
                 // ---- A5 with the centroid values written instead of the codes:
@@ -252,15 +360,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                 if (s <= p.s_max) {
                     const float inv = p.rsqrt_h / (s + p.eps);
                     const float2 inv2 = make_float2(inv, inv);
-                    // table word of element pair j and the selector bits of its two values
-                    auto pick = [&](int j, uint32_t& val0, uint32_t& val1, uint32_t& ge0, uint32_t& ge1) {
-                        const float2 q = f2mul(v2[j], inv2);
+                    // table word of element pair i and the selector bits of its two values
+                    auto pick = [&](int i, uint32_t& val0, uint32_t& val1, uint32_t& ge0, uint32_t& ge1) {
+                        const float2 q = f2mul(v2[i], inv2);
                         const float2 z = f2fma(q, G2, M2);
                         float T0, T1;
-                        const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
-                        const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
-                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(val0) : "r"(a0));
-                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(val1) : "r"(a1));
+                        lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, val0);
+                        lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, val1);
                         ge0 = q.x >= T0 ? 1u : 0u;
                         ge1 = q.y >= T1 ? 1u : 0u;
                     };
@@ -308,6 +414,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                     else
                         reinterpret_cast<uint32_t*>(dst)[w0] = words[0];
                 };
+                // code of element pair i: (index of .x, index of .y)
+                auto code2 = [&](int i, float2 inv2, uint32_t& i0, uint32_t& i1) {
+                    const float2 q = f2mul(v2[i], inv2);
+                    const float2 z = f2fma(q, G2, M2);
+                    float T0, T1;
+                    uint32_t b0, b1;
+                    lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, b0);
+                    lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, b1);
+                    i0 = b0 + (q.x >= T0 ? 1u : 0u);
+                    i1 = b1 + (q.y >= T1 ? 1u : 0u);
+                };
                 // s <= s_max keeps every butterfly value below sqrt(h) s (finite),
                 // so |v| <= 1 up to rounding and the table index stays in range;
                 // larger, infinite and NaN norms take the middle cell
@@ -324,17 +441,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                         for (int gi = 0; gi < 4; ++gi) {
                             uint32_t acc_w = 0;
 #pragma unroll
-                            for (int k = 6; k >= 0; k -= 2) {
-                                const float2 q = f2mul(v2[(32 * g4 + 8 * gi + k) >> 1], inv2);
-                                const float2 z = f2fma(q, G2, M2);
-                                float T0, T1;
-                                int b0, b1;
-                                const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
-                                const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
-                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
-                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
-                                const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
-                                const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
+                            for (int kk = 6; kk >= 0; kk -= 2) {
+                                uint32_t i0, i1;
+                                code2((32 * g4 + 8 * gi + kk) >> 1, inv2, i0, i1);
                                 acc_w = (acc_w * 8u + i1) * 8u + i0;
                             }
                             grp[gi] = acc_w;
@@ -363,17 +472,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                             // codes of this word, highest position first: acc = acc * 2^bits + code
                             uint32_t acc_w = 0;
 #pragma unroll
-                            for (int k = PER - 2; k >= 0; k -= 2) {
-                                const float2 q = f2mul(v2[(wi * PER + k) >> 1], inv2);
-                                const float2 z = f2fma(q, G2, M2);
-                                float T0, T1;
-                                int b0, b1;
-                                const uint32_t a0 = __float_as_uint(z.x) * 8u + lut_addr0;
-                                const uint32_t a1 = __float_as_uint(z.y) * 8u + lut_addr0;
-                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T0), "=r"(b0) : "r"(a0));
-                                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T1), "=r"(b1) : "r"(a1));
-                                const uint32_t i0 = (uint32_t)(b0 + (q.x >= T0 ? 1 : 0));
-                                const uint32_t i1 = (uint32_t)(b1 + (q.y >= T1 ? 1 : 0));
+                            for (int kk = PER - 2; kk >= 0; kk -= 2) {
+                                uint32_t i0, i1;
+                                code2((wi * PER + kk) >> 1, inv2, i0, i1);
                                 acc_w = (acc_w * SH + i1) * SH + i0;
                             }
                             words[wj] = acc_w;
@@ -382,8 +483,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                     }
                 } else if (BITS == 3) {
                     // middle code 4 everywhere: the 3-bit stream repeats every 3 words
-                    constexpr uint32_t g = 04444'4444u;  // eight 3-bit fours (octal)
-                    const uint32_t pat[3] = {g | (g << 24), (g >> 8) | (g << 16), (g >> 16) | (g << 8)};
+                    constexpr uint32_t gm = 04444'4444u;  // eight 3-bit fours (octal)
+                    const uint32_t pat[3] = {gm | (gm << 24), (gm >> 8) | (gm << 16), (gm >> 16) | (gm << 8)};
 #pragma unroll
                     for (int w0 = 0; w0 < NW; w0 += CW) {
                         uint32_t ws[CW];
@@ -394,7 +495,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                 } else {
                     uint32_t wmid = 0;
 #pragma unroll
-                    for (int k = 0; k < PER; ++k) wmid = wmid * SH + (uint32_t)(p.L >> 1);
+                    for (int kk = 0; kk < PER; ++kk) wmid = wmid * SH + (uint32_t)(p.L >> 1);
                     uint32_t words[CW];
 #pragma unroll
                     for (int wj = 0; wj < CW; ++wj) words[wj] = wmid;
@@ -403,17 +504,28 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const RpbhPa
                 }
             }
         }
-        group_sync(1 + grp, G);  // this stage and the partials are free for reuse
     }
+
+    // Leaving (normally or after an abort): copies this CTA issued must land
+    // before its shared memory goes away.
+    if (loader) {
+        for (int sl = 0; sl < p.slots; ++sl)
+            if (issued_k[sl] > consumed_k) {
+                const int kk = issued_k[sl];
+                mbar_wait_bounded(&my_full[sl], (uint32_t)((p.slots == 1 ? kk : (kk >> 1)) & 1));
+            }
+    }
+    if (tid == 0 && !p.starve) mbar_wait_bounded(tab_bar, 0u);
 }
 
 template <typename InT, int H, int BITS, int MODE>
 cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
     auto k = rpbh_quant_kernel<InT, H, BITS, MODE>;
     const int smem = smem_layout(p).total;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t e = ensure_smem_limit(k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, p.T, smem, stream>>>(p);
+    const cudaError_t le = launch_pdl(k, dim3(grid), dim3(p.tpc * p.team * 32), smem, stream, p);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -450,6 +562,56 @@ cudaError_t launch_h(const RpbhParams& p, int h, int bits, int grid, cudaStream_
 }  // namespace
 
 int rpbh_smem_bytes(const RpbhParams& p) { return smem_layout(p).total; }
+
+// Layout choice.  More rows per warp spread the warp's random gather over
+// more banks: consecutive rows of a slot start 128 / RW bytes apart modulo
+// 128 (16 bytes at least, the bulk copies' alignment), so the RW rows' copies
+// of one column sit in RW different groups of 32 / RW banks and only the
+// warp's 32 / RW blocks can collide.  Larger RW costs larger slots and
+// larger teams.  Among the layouts that fit, the one with the most warps is
+// taken (they hide the gathers' latency), then the one with two slots per
+// team (the next row set streams in during the whole computation of this
+// one), then the one with the most rows per warp.  A forced layout (test
+// and tuning hook) is taken when it fits.
+static int g_force_rw = 0, g_force_slots = 0;
+
+void rpbh_force_layout(int rows_per_warp, int slots) {
+    g_force_rw = rows_per_warp;
+    g_force_slots = slots;
+}
+
+bool rpbh_choose_layout(RpbhParams& p, int h, int esize) {
+    const int nb = p.d / h;
+    p.row_bytes = p.d * esize;
+    RpbhParams best = p;
+    int best_key = -1;
+    for (int slots = 2; slots >= 1; --slots) {
+        for (int RW = 8; RW >= 1; RW >>= 1) {
+            if (g_force_rw && RW != g_force_rw) continue;
+            if (g_force_slots && slots != g_force_slots) continue;
+            const int Bw = 32 / RW;
+            const int team = (nb + Bw - 1) / Bw;
+            if (team > kMaxWarps) continue;
+            RpbhParams c = p;
+            c.RW = RW;
+            c.lbw = RW == 8 ? 2 : (RW == 4 ? 3 : (RW == 2 ? 4 : 5));
+            c.team = team;
+            c.slots = slots;
+            c.srow = c.row_bytes + (RW == 1 ? 16 : 128 / RW);
+            for (c.tpc = kMaxWarps / team; c.tpc >= 1; --c.tpc)
+                if (rpbh_smem_bytes(c) <= kSmemLimit) break;
+            if (c.tpc < 1) continue;
+            const int key = (c.tpc * team) * 100 + slots * 10 + RW;
+            if (key > best_key) {
+                best_key = key;
+                best = c;
+            }
+        }
+    }
+    if (best_key < 0) return false;
+    p = best;
+    return true;
+}
 
 cudaError_t launch_rpbh_quant(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
                               cudaStream_t stream) {

@@ -11,31 +11,52 @@ namespace oq {
 struct RpbhParams {
     const void* x;        // [M, d] rows, bf16 or fp32
     int M, d, nb;         // rows, dimension, h-blocks per row (d / h)
-    int R, T, G, NG;      // rows per tile (power of two), threads per CTA, threads per warp group, groups (T = NG G)
+    // Work layout.  A warp covers RW rows x (32 / RW) h-blocks (lane = row
+    // r * (32 / RW) + block j); a team of `team` warps covers all nb blocks
+    // of a set of RW rows; a CTA holds `tpc` teams, each with `slots`
+    // staging slots of RW rows.
+    int RW, lbw;          // rows per warp; log2 of the blocks per warp
+    int team, tpc, slots;
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
-    int ntiles;
-    const uint16_t* gtab;  // device gather table (chunked, see host.cpp)
-    const LutEntry* lut;   // device quantiser lookup table
-    int lut_n, lut_off;    // entries; index offset = -(magic bits) - kmin
-    float G_lut;           // lookup-table bins per unit of v
-    int L;                 // levels (2^bits)
-    uint8_t* idx_out;      // packed indices
+    int nrs;              // row sets: ceil(M / RW)
+    const uint32_t* gtab; // device gather table (see build_gather_table)
+    const LutEntry* lut;  // device quantiser lookup table
+    int lut_n, lut_off;   // entries; index offset = -(magic bits) - kmin
+    float G_lut;          // lookup-table bins per unit of v
+    int L;                // levels (2^bits)
+    uint8_t* idx_out;     // packed indices (or the centroid values)
     int out_row_bytes;
-    float* s_out;          // activations: s (fp32)
-    uint16_t* r_out;       // weights: r (bf16)
-    float* y_out;          // test hook: x' (fp32)
-    float* norm_out;       // test hook: ||x'||
-    float rsqrt_h;         // 1/sqrt(h)
-    float eps;             // the split's eps
-    float s_max;           // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
-    int starve;            // test hook: issue no row copies (the waits run out)
-    uint32_t mid_val;      // value outputs: the middle cell's value (bf16 bits or e4m3 byte)
+    float* s_out;         // activations: s (fp32)
+    uint16_t* r_out;      // weights: r (bf16)
+    float* y_out;         // test hook: x' (fp32)
+    float* norm_out;      // test hook: ||x'||
+    float rsqrt_h;        // 1/sqrt(h)
+    float eps;            // the split's eps
+    float s_max;          // FLT_MAX / (2 sqrt(h)): larger row norms take the middle cell
+    int starve;           // test hook: issue no copies (the waits run out)
+    uint32_t mid_val;     // value outputs: the middle cell's value (bf16 bits or e4m3 byte)
 };
 
-constexpr int kMaxGroups = 4;    // warp groups per CTA (at most 128 threads each)
-constexpr int kMaxThreads = 384;  // per CTA: the kernel's launch bound (168 registers each)
+constexpr int kMaxWarps = 12;                 // per CTA: the kernel's launch bound is 384 threads
+constexpr int kMaxThreads = kMaxWarps * 32;   // (168 registers each)
+constexpr int kSmemLimit = 227 * 1024;
 
 int rpbh_smem_bytes(const RpbhParams& p);
+
+// Chooses RW, team, tpc, slots and srow for a shape (the choice depends on d,
+// h, the input's element size and the lookup table only, so every output
+// mode of one shape takes the same layout and sums the row norm in the same
+// order).  Returns false if no layout fits in shared memory.
+bool rpbh_choose_layout(RpbhParams& p, int h, int esize);
+
+// Test and tuning hook: force rows per warp and slots per team (0: automatic).
+void rpbh_force_layout(int rows_per_warp, int slots);
+
+// The kernel for blocks of 256 ... 16384 (rht_big.cu): one row per CTA at a
+// time; RW, team, tpc, slots and srow are not used.
+int rht_big_smem_bytes(const RpbhParams& p);
+cudaError_t launch_rht_big(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
+                           cudaStream_t stream);
 
 // mode 0: activations (s fp32), 1: weights (r bf16), 2: rotation only (x', norm),
 // 3 / 4: activations as centroid values, bf16 / e4m3 of c sqrt(d) (s fp32)

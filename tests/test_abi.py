@@ -60,6 +60,20 @@ def test_library_plan_matches_oracle(d, h, seed):
     np.testing.assert_array_equal(s1, s2)
 
 
+def test_library_plan_matches_hand_derived_golden():
+    """The library's shuffle against the permutation derived by hand from the
+    published SplitMix64 outputs (tests/golden), independently of the oracle."""
+    import os
+
+    golden = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "fisher_yates_d5_seed1234567.txt")
+    with open(golden) as f:
+        rows = {ln.split()[0]: ln.split()[1:] for ln in f if ln.strip() and not ln.startswith("#")}
+    seed, d = int(rows["seed"][0]), int(rows["d"][0])
+    perm, sign = B.rpbh_plan_host(d, d, seed)
+    assert perm.tolist() == [int(v) for v in rows["perm"]]
+    assert int(sign[0]) == int(rows["sign0"][0])
+
+
 @pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (4096, 128, 3)])
 def test_library_block_rht_plan_matches_oracle(d, h, seed):
     p1, s1 = B.rotation_plan_host(d, h, seed, B.OQ_ROT_BLOCK_RHT)
@@ -109,8 +123,10 @@ def test_argument_checks_on_host_calls():
     P = perm.ctypes.data_as(ctypes.c_void_p)
     S = sign.ctypes.data_as(ctypes.c_void_p)
     assert L.oq_rpbh_plan_host(300, 128, 0, P, S) == 2  # d % h != 0
-    assert L.oq_rpbh_plan_host(256, 96, 0, P, S) == 2  # h not a power of two
-    assert L.oq_rpbh_plan_host(256, 256, 0, P, S) == 2  # h beyond the in-register block
+    assert L.oq_rpbh_plan_host(256, 96, 0, P, S) == 2  # d % h != 0
+    assert L.oq_rpbh_plan_host(256, 256, 0, P, S) == 0  # the host plan's arrays do not depend on h
+    assert L.oq_rpbh_plan_host(5, 5, 0, P, S) == 0
+    assert L.oq_rpbh_plan_host(40000, 8, 0, P, S) == 2  # beyond the 16-bit gather offsets
     assert L.oq_rpbh_plan_host(0, 64, 0, P, S) == 1
     assert L.oq_rpbh_plan_host(256, 64, 0, P, S) == 0
 
@@ -167,3 +183,30 @@ def test_unpack_layout():
     p3 = torch.tensor([[stream & 0xFF, (stream >> 8) & 0xFF, stream >> 16]], dtype=torch.uint8)
     assert B.unpack_indices(p3, 8, 3).tolist() == [list(range(8))]
     assert B.packed_row_bytes(1536, 8) == 1536 and B.packed_row_bytes(1536, 6) == 1536
+
+
+def test_binding_rejects_buffers_the_kernels_would_overrun():
+    """The C ABI sees only pointers and sizes, so the binding checks shapes,
+    dtypes, layout and device before any call (ValueError, no library call)."""
+    import torch
+
+    class FakePlan:  # only the dimension is read before the checks fail
+        d = 256
+        handle = None
+
+    class FakeCb:
+        d, bits = 256, 4
+        handle = None
+
+    x_cpu = torch.zeros((8, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.quantize_acts(FakePlan(), FakeCb(), x_cpu)  # not on a CUDA device
+    with pytest.raises(ValueError):
+        B.quantize_weights(FakePlan(), FakeCb(), torch.zeros((8, 256)))
+    with pytest.raises(ValueError):
+        B.rpbh_apply(FakePlan(), torch.zeros(256))  # not 2-D
+    with pytest.raises(ValueError):
+        B.qlinear(FakePlan(), FakeCb(), FakeCb(), x_cpu, torch.zeros((4, 128), dtype=torch.uint8),
+                  torch.zeros(4, dtype=torch.bfloat16))
+    assert B.packed_row_bytes(256, 3) == 96 and B.packed_row_bytes(256, 6) == 256
+    assert B.packed_row_bytes(256, 8) == 256 and B.packed_row_bytes(256, 2) == 64

@@ -113,3 +113,28 @@ def test_outputs_run_on_a_side_stream(layer, cuda_device):
     torch.cuda.current_stream().wait_stream(st)
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
+
+
+def test_binding_checks_buffers_before_the_call(layer, cuda_device):
+    """Wrong shapes, dtypes, layouts or devices are refused in the binding,
+    before the C ABI (which sees only pointers and sizes) could overrun them."""
+    plan, cb4, cb2, d = layer
+    x = torch.randn(16, d, device=cuda_device).to(torch.bfloat16)
+    W = torch.randn(32, d, device=cuda_device).to(torch.bfloat16)
+    w_idx, w_r = B.quantize_weights(plan, cb2, W)
+    with pytest.raises(ValueError):  # y of the wrong shape
+        B.qlinear(plan, cb4, cb2, x, w_idx, w_r, y=torch.empty((16, 31), dtype=torch.bfloat16, device=cuda_device))
+    with pytest.raises(ValueError):  # y of the wrong dtype
+        B.qlinear_noalloc(plan, cb4, cb2, x, w_idx, w_r, torch.empty((16, 32), dtype=torch.float32,
+                                                                   device=cuda_device))
+    with pytest.raises(ValueError):  # x not contiguous
+        B.quantize_acts(plan, cb4, torch.randn(d, 16, device=cuda_device).to(torch.bfloat16).t())
+    with pytest.raises(ValueError):  # x narrower than the plan's d
+        B.quantize_acts(plan, cb4, x[:, : d // 2].contiguous())
+    with pytest.raises(ValueError):  # packed W rows of another width
+        B.qlinear(plan, cb4, cb2, x, w_idx[:, :-1].contiguous(), w_r)
+    with pytest.raises(ValueError):  # norms of another dtype
+        B.qgemm(cb4, cb2, torch.zeros((16, d // 2), dtype=torch.uint8, device=cuda_device),
+                torch.ones(16, dtype=torch.float16, device=cuda_device), w_idx, w_r)
+    with pytest.raises(ValueError):  # an output on the host
+        B.quantize_acts(plan, cb4, x, s_out=torch.empty(16))

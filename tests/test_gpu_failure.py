@@ -131,3 +131,39 @@ def test_starved_layer_reports_timeout_from_both_kernels(layer):
     y = B.qlinear(L["plan"], L["cb4"], L["cb2"], L["x"], L["w_idx"], L["w_r"])
     assert torch.equal(y, L["y"])
     assert B.device_status() == 0
+
+
+def test_starved_quantizer_releases_the_dependent_gemm(layer):
+    """The product launches programmatically after the quantiser and waits
+    for it to finish before reading its output.  A quantiser whose waits run
+    out still finishes (bounded), so the product's dependency wait ends and
+    the layer call returns; the next call is exact again."""
+    L = layer
+    B.debug_starve(B.OQ_STARVE_RPBH)
+    try:
+        B.qlinear(L["plan"], L["cb4"], L["cb2"], L["x"], L["w_idx"], L["w_r"])
+        assert B.device_status(clear=True) == 5
+    finally:
+        _reset_hooks()
+    y = B.qlinear(L["plan"], L["cb4"], L["cb2"], L["x"], L["w_idx"], L["w_r"])
+    assert torch.equal(y, L["y"])
+    assert B.device_status() == 0
+
+
+def test_starved_large_block_quantizer_times_out_and_context_survives(cuda_device):
+    """The staged kernel for blocks beyond 128 (Full RHT) bounds its waits too."""
+    d = 1024
+    plan = B.rotation_plan(d, d, 5, B.OQ_ROT_BLOCK_RHT)
+    cb = B.codebook(d, 4)
+    x = torch.randn(20, d, device=cuda_device).to(torch.bfloat16)
+    ref_idx, ref_s = B.quantize_acts(plan, cb, x)
+    torch.cuda.synchronize()
+    B.debug_starve(B.OQ_STARVE_RPBH)
+    try:
+        B.quantize_acts(plan, cb, x)
+        assert B.device_status(clear=True) == 5
+    finally:
+        _reset_hooks()
+    idx, s = B.quantize_acts(plan, cb, x)
+    assert torch.equal(idx, ref_idx) and torch.equal(s, ref_s)
+    assert B.device_status() == 0

@@ -1,6 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
-the same seeded inputs -- multi-tile ragged cases checked in full, the five
-workload shapes at full size checked on sampled rows and columns.
+the same seeded inputs -- multi-tile ragged cases checked in full; at the
+five workload shapes at full size, the codes and norms of every activation
+and weight row, the rotation on 512 rows, and the product on 512 rows x all
+N plus all M x 256 columns.
 
 Tolerances are stated in tests/parity.py.
 """
@@ -14,13 +16,14 @@ import oracle
 from rotation_bit_quantization_rpbh_b200 import binding as B
 from rotation_bit_quantization_rpbh_b200 import inputs as I
 
-from parity import (GEMM_TOL, check_quantized_rows, check_rotation, gemm_reference, rel_frob, to_f64)
+from parity import (GEMM_TOL, check_product, check_quantized_rows, check_rotation, gemm_reference, rel_frob,
+                    to_f64)
 
 pytestmark = pytest.mark.gpu
 
 
-def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_idx=1024, n_rows_gemm=128,
-               n_cols_gemm=64, bias=False):
+def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rot=512, n_rows_gemm=512, n_cols_gemm=256,
+               bias=False):
     rng = np.random.default_rng(seed + 7)
     plan = B.rpbh_plan(d, h, seed)
     perm, sign = oracle.plan(d, h, seed)
@@ -44,12 +47,11 @@ def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_i
     assert torch.equal(y, y2)
     _check_values_schedule(dev, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, bias_t, y, ba, bw, fp8=False)
 
-    rows_a = np.arange(M) if full_check else np.sort(rng.choice(M, min(M, n_rows_idx), replace=False))
-    rows_w = np.arange(N) if full_check else np.sort(rng.choice(N, min(N, n_rows_idx), replace=False))
-    rot_rows = rows_a if full_check else rows_a[:64]
+    # codes and norms of every row of x and of W
+    rot_rows = np.arange(M) if full_check else np.sort(rng.choice(M, min(M, n_rot), replace=False))
     check_rotation(plan, x_cpu, rot_rows, h, perm, sign, dev)
-    nb_a, _ = check_quantized_rows(a_idx, s, x_cpu, rows_a, h, perm, sign, cb_a, ocb_a, "acts")
-    nb_w, n_ulp = check_quantized_rows(w_idx, w_r, W_cpu, rows_w, h, perm, sign, cb_w, ocb_w, "weights")
+    nb_a, _ = check_quantized_rows(a_idx, s, x_cpu, np.arange(M), h, perm, sign, cb_a, ocb_a, "acts")
+    nb_w, n_ulp = check_quantized_rows(w_idx, w_r, W_cpu, np.arange(N), h, perm, sign, cb_w, ocb_w, "weights")
 
     # product: oracle fp64 on the GPU's indices, norms and the bf16 centroid values
     ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
@@ -65,8 +67,7 @@ def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_i
         ref = gemm_reference(ia, s64, iw, r64, ca, cw)
         if b64 is not None:
             ref = ref + b64[None, :]
-        err = rel_frob(yg, ref)
-        assert err <= GEMM_TOL, err
+        err, _, worst = check_product(yg, ref)
     else:
         rr = np.sort(rng.choice(M, min(M, n_rows_gemm), replace=False))
         cc = np.sort(rng.choice(N, min(N, n_cols_gemm), replace=False))
@@ -75,9 +76,11 @@ def _run_layer(dev, M, d, N, h, bw, ba, x_cpu, W_cpu, seed, full_check, n_rows_i
         if b64 is not None:
             ref_r = ref_r + b64[None, :]
             ref_c = ref_c + b64[None, cc]
-        err = max(rel_frob(yg[rr], ref_r), rel_frob(yg[:, cc], ref_c))
-        assert err <= GEMM_TOL, err
-    return {"band_a": nb_a, "band_w": nb_w, "r_ulp": n_ulp, "gemm_rel": err}
+        e1, _, w1 = check_product(yg[rr], ref_r)
+        e2, _, w2 = check_product(yg[:, cc], ref_c)
+        err, worst = max(e1, e2), max(w1, w2)
+    return {"band_a": nb_a, "band_w": nb_w, "coords_a": M * d, "coords_w": N * d, "r_ulp": n_ulp, "gemm_rel": err,
+            "worst_elem_over_bound": worst}
 
 
 def _check_values_schedule(dev, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, bias_t, y, ba, bw, fp8):
@@ -156,6 +159,43 @@ def test_block_rht_variant_matches_oracle(cuda_device, M, d, h, ba):
     check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb_a, ocb_a, "acts")
 
 
+@pytest.mark.parametrize("M,d,h,variant,ba,dt", [
+    (70, 4096, 4096, "block_rht", 4, "bf16"),   # Full RHT: one Walsh-Hadamard block over d
+    (33, 1024, 1024, "block_rht", 2, "f32"),
+    (50, 3072, 1024, "block_rht", 6, "bf16"),   # the largest power-of-two block of d = 3 * 1024
+    (41, 2048, 512, "rpbh", 4, "bf16"),        # RPBH with blocks larger than the in-register kernel
+    (9, 16384, 16384, "block_rht", 4, "bf16"),
+])
+def test_large_block_rotation_matches_oracle(cuda_device, M, d, h, variant, ba, dt):
+    """Blocks of h > 128 (the rotation ablation's Full RHT, h = d) run in the
+    staged kernel: rotation, norms and codes against the oracle's direct
+    O(h) sums, and the value outputs equal to the codebook at the codes."""
+    seed = 70 + M
+    v = B.OQ_ROT_BLOCK_RHT if variant == "block_rht" else B.OQ_ROT_RPBH
+    plan = B.rotation_plan(d, h, seed, v)
+    perm, sign = oracle.plan(d, h, seed, variant=oracle.BLOCK_RHT if variant == "block_rht" else 0)
+    pe, se = plan.export()
+    np.testing.assert_array_equal(pe, perm)
+    np.testing.assert_array_equal(se, sign)
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))
+    x[:, torch.randint(0, d, (4,), generator=g)] *= 25.0
+    x = x.to(torch.bfloat16 if dt == "bf16" else torch.float32)
+    cb_a, ocb_a = B.codebook(d, ba), oracle.codebook(d, ba)
+    xg = x.to(cuda_device)
+    a_idx, s = B.quantize_acts(plan, cb_a, xg)
+    val, s_v = B.quantize_acts_values(plan, cb_a, xg)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    rows = np.arange(M)
+    check_rotation(plan, x, rows, h, perm, sign, cuda_device)
+    check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb_a, ocb_a, "acts")
+    u = B.unpack_indices(a_idx, d, ba).long()
+    tab = torch.from_numpy(cb_a.bf16_bits().view(np.int16)).to(cuda_device)
+    assert torch.equal(val.view(torch.int16), tab[u])
+    assert torch.equal(s_v, s)
+
+
 def _e4m3_values(c, d):
     """e4m3 centroid values of the fp8 variant, from the oracle's fp64 codebook:
     c_j sqrt(d) rounded once to e4m3 (torch's conversion), scaled back."""
@@ -201,7 +241,7 @@ def test_fp8_variant_matches_oracle_on_e4m3_centroids(cuda_device, case):
         ref = ref + bias_t.cpu().to(torch.float32).numpy().astype(np.float64)[None, :]
     got = y.float().cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(got))
-    assert rel_frob(got, ref) <= GEMM_TOL
+    check_product(got, ref)
 
 
 def test_fp8_variant_needs_d_multiple_of_128(cuda_device):
@@ -240,7 +280,7 @@ def test_fp8_variant_full_size_flux_qkv_sample(cuda_device):
     ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
                          w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw, rows, cols)
     got = y.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)]
-    assert rel_frob(got, ref) <= GEMM_TOL
+    check_product(got, ref)
 
 
 @pytest.mark.parametrize("M,d,h,seed", [(300, 512, 128, 51), (97, 384, 64, 52), (64, 256, 32, 53)])
@@ -284,16 +324,48 @@ def test_three_bit_fp8_product_matches_oracle(cuda_device, bw, ba):
     iw = B.unpack_indices(w_idx, d, bw).cpu().numpy()
     ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
                          w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw)
-    assert rel_frob(y.float().cpu().numpy().astype(np.float64), ref) <= GEMM_TOL
+    check_product(y.float().cpu().numpy().astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("bw,ba", [(3, 3), (3, 4), (4, 3)])
+def test_three_bit_bf16_product_matches_oracle(cuda_device, bw, ba):
+    """W3A3 (a setting of the page's ablation) and the mixed 3/4-bit pairs at
+    the bf16 centroid precision the rest of the layer uses: the codes product,
+    the values product and the one-call layer against the oracle's fp64
+    product on the same indices, norms and bf16 centroids."""
+    M, d, N, h, seed = 300, 768, 520, 128, 64 + bw + ba
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, h, seed)
+    cb_a, cb_w = B.codebook(d, ba), B.codebook(d, bw)
+    ocb_a, ocb_w = oracle.codebook(d, ba), oracle.codebook(d, bw)
+    xg = x.to(cuda_device)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    a_idx, s = B.quantize_acts(plan, cb_a, xg)
+    bias_t = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16).to(cuda_device)
+    y = B.qgemm(cb_a, cb_w, a_idx, s, w_idx, w_r, bias=bias_t)
+    y2 = B.qlinear(plan, cb_a, cb_w, xg, w_idx, w_r, bias=bias_t)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert torch.equal(y, y2)
+    _check_values_schedule(cuda_device, plan, cb_a, cb_w, xg, a_idx, s, w_idx, w_r, bias_t, y, ba, bw, fp8=False)
+    ia = B.unpack_indices(a_idx, d, ba).cpu().numpy()
+    iw = B.unpack_indices(w_idx, d, bw).cpu().numpy()
+    ca, cw = oracle.round_bf16(ocb_a[0])[1], oracle.round_bf16(ocb_w[0])[1]
+    ref = gemm_reference(ia, s.cpu().numpy().astype(np.float64), iw,
+                         w_r.cpu().to(torch.float32).numpy().astype(np.float64), ca, cw)
+    ref = ref + bias_t.cpu().to(torch.float32).numpy().astype(np.float64)[None, :]
+    check_product(y.float().cpu().numpy().astype(np.float64), ref)
 
 
 def test_values_schedule_limits_are_reported(cuda_device):
-    cb3 = B.codebook(256, 3)
-    val = torch.zeros((8, 256), dtype=torch.bfloat16, device=cuda_device)
+    cb3 = B.codebook(192, 3)  # 3-bit rows need d % 128 == 0
+    val = torch.zeros((8, 192), dtype=torch.bfloat16, device=cuda_device)
     s = torch.ones(8, device=cuda_device)
-    w_idx = torch.zeros((16, 96), dtype=torch.uint8, device=cuda_device)
+    w_idx = torch.zeros((16, 72), dtype=torch.uint8, device=cuda_device)
     w_r = torch.ones(16, dtype=torch.bfloat16, device=cuda_device)
-    with pytest.raises(B.OQError) as e:  # 3-bit weights: the fp8 product only
+    with pytest.raises(B.OQError) as e:
         B.qgemm_values(cb3, val, s, w_idx, w_r)
     assert e.value.status == 2
     plan = B.rpbh_plan(192, 64, 3)
@@ -302,8 +374,9 @@ def test_values_schedule_limits_are_reported(cuda_device):
     assert e.value.status == 2
     bad = torch.zeros(8 * 256 + 8, dtype=torch.bfloat16, device=cuda_device)[1:1 + 8 * 256].view(8, 256)
     w4 = torch.zeros((16, 128), dtype=torch.uint8, device=cuda_device)
+    s8 = torch.ones(8, device=cuda_device)
     with pytest.raises(B.OQError) as e:  # values not 16-byte aligned
-        B.qgemm_values(B.codebook(256, 4), bad, s, w4, w_r)
+        B.qgemm_values(B.codebook(256, 4), bad, s8, w4, w_r)
     assert e.value.status == 3
 
 
@@ -315,10 +388,11 @@ def test_three_bit_limits_are_reported(cuda_device):
         B.quantize_acts(B.rpbh_plan(d, 16, 1), cb, x)
     assert e.value.status == 2
     a_idx, s = B.quantize_acts(B.rpbh_plan(d, 64, 1), cb, x)
-    w_idx = torch.zeros((16, d * 3 // 8), dtype=torch.uint8, device=cuda_device)
+    cb2 = B.codebook(d, 2)
+    w_idx = torch.zeros((16, d // 4), dtype=torch.uint8, device=cuda_device)
     w_r = torch.ones(16, dtype=torch.bfloat16, device=cuda_device)
-    with pytest.raises(B.OQError) as e:  # the bf16 kernel's 64-code step is 24 bytes of 3-bit codes
-        B.qgemm(cb, cb, a_idx, s, w_idx, w_r)
+    with pytest.raises(B.OQError) as e:  # 3-bit codes pair with 3- or 4-bit codes only
+        B.qgemm(cb, cb2, a_idx, s, w_idx, w_r)
     assert e.value.status == 2
 
 
@@ -362,4 +436,4 @@ def test_eight_bit_activations_match_oracle(cuda_device):
         else:
             ca, cw = oracle.round_bf16(ocb_a[0])[1], oracle.round_bf16(ocb_w[0])[1]
         ref = gemm_reference(ia, s64, iw, r64, ca, cw)
-        assert rel_frob(y.float().cpu().numpy().astype(np.float64), ref) <= GEMM_TOL
+        check_product(y.float().cpu().numpy().astype(np.float64), ref)

@@ -100,6 +100,21 @@ def test_plan_is_a_bijection_with_rademacher_signs(d, h):
     assert abs(sign.mean()) < 5.0 / math.sqrt(d)
 
 
+def _golden_fisher_yates():
+    with open(os.path.join(GOLDEN, "fisher_yates_d5_seed1234567.txt")) as f:
+        rows = {ln.split()[0]: ln.split()[1:] for ln in f if ln.strip() and not ln.startswith("#")}
+    return int(rows["seed"][0]), int(rows["d"][0]), [int(v) for v in rows["perm"]], int(rows["sign0"][0])
+
+
+def test_plan_shuffle_order_matches_hand_derived_golden():
+    """The shuffle's loop direction and swap rule, pinned by a permutation
+    derived by hand from the published SplitMix64 outputs (golden file)."""
+    seed, d, perm_want, sign0 = _golden_fisher_yates()
+    perm, sign = oracle.plan(d, d, seed)
+    assert perm.tolist() == perm_want
+    assert int(sign[0]) == sign0
+
+
 def test_plan_permutation_is_uniform():
     """Fisher-Yates over SplitMix64 draws every permutation of 4 items equally often."""
     n = 24000
