@@ -34,7 +34,7 @@ EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status",
            "oq_debug_fail_allocations", "oq_debug_starve", "oq_quantize_acts_values",
            "oq_quantize_acts_values_fp8", "oq_qgemm_values", "oq_qgemm_values_fp8", "oq_qlinear_workspace_values",
-           "oq_debug_rpbh_layout", "oq_codebook_upload"]
+           "oq_debug_rpbh_layout", "oq_codebook_upload", "oq_debug_qgemm_tile_rows"]
 
 
 class OQError(RuntimeError):
@@ -86,7 +86,8 @@ def lib():
                     "oq_device_status": ([I, P, P], I),
                     "oq_debug_fail_allocations": ([I], None),
                     "oq_debug_starve": ([I], None),
-                    "oq_debug_rpbh_layout": ([I, I], None),
+                    "oq_debug_rpbh_layout": ([I, I, I], None),
+                    "oq_debug_qgemm_tile_rows": ([I], None),
                     "oq_quantize_acts_values": ([P, P, P, I, I, P, P, P], I),
                     "oq_quantize_acts_values_fp8": ([P, P, P, I, I, P, P, P], I),
                     "oq_qgemm_values": ([P, I, I, P, P, P, P, P, P, P], I),
@@ -470,11 +471,18 @@ def debug_starve(mask):
     lib().oq_debug_starve(int(mask))
 
 
-def debug_rpbh_layout(rows_per_warp=0, slots=0):
+def debug_rpbh_layout(rows_per_warp=0, slots=0, lanes_per_block=0):
     """Test and tuning hook: force the rotate-and-quantise kernel's rows per
-    warp (1, 2, 4, 8) and staging slots per warp team (1, 2) where they fit;
-    0 restores the library's choice."""
-    lib().oq_debug_rpbh_layout(int(rows_per_warp), int(slots))
+    warp (1, 2, 4, 8), staging slots per warp team (1, 2) and lanes per
+    h-block (2: two lanes share a block; bf16 inputs, h of 64 or 128) where
+    they fit; 0 restores the library's choice."""
+    lib().oq_debug_rpbh_layout(int(rows_per_warp), int(slots), int(lanes_per_block))
+
+
+def debug_qgemm_tile_rows(rows=0):
+    """Test and tuning hook: tiles of 256 or 512 rows of A in the A-values
+    product (0: the library's choice per shape)."""
+    lib().oq_debug_qgemm_tile_rows(int(rows))
 
 
 def unpack_indices(packed, d, bits):

@@ -612,10 +612,13 @@ void oq_debug_fail_allocations(int n) { g_fail_allocs.store(n > 0 ? n : 0); }
 
 void oq_debug_starve(int mask) { g_starve_mask.store(mask & (OQ_STARVE_RPBH | OQ_STARVE_GEMM)); }
 
-void oq_debug_rpbh_layout(int rows_per_warp, int slots) {
+void oq_debug_qgemm_tile_rows(int rows) { qgemm_force_tile_rows(rows); }
+
+void oq_debug_rpbh_layout(int rows_per_warp, int slots, int lanes_per_block) {
     const bool rw_ok = rows_per_warp == 0 || rows_per_warp == 1 || rows_per_warp == 2 || rows_per_warp == 4 ||
                        rows_per_warp == 8;
-    rpbh_force_layout(rw_ok ? rows_per_warp : 0, (slots == 1 || slots == 2) ? slots : 0);
+    rpbh_force_layout(rw_ok ? rows_per_warp : 0, (slots == 1 || slots == 2) ? slots : 0,
+                      lanes_per_block == 2 ? 2 : 0);
 }
 
 oq_status oq_device_status(int clear, int* out, void* stream) {

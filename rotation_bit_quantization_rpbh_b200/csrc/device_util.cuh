@@ -116,14 +116,16 @@ inline cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, int smem, cudaStr
 }
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` once per device
-// (cudaFuncSetAttribute is a host call that costs more than some launches);
-// one cache per kernel instantiation.  Benign races only repeat the call.
+// (cudaFuncSetAttribute is a host call that costs more than some launches).
+// `done` is the calling launch function's own per-device record -- one per
+// kernel instantiation (kernels of one signature share a function-pointer
+// type, so the record cannot live here).  Benign races only repeat the call.
+constexpr int kSmemRecordDevices = 64;
+
 template <typename K>
-inline cudaError_t ensure_smem_limit(K kernel, int bytes) {
-    constexpr int kDevs = 64;
-    static int done[kDevs] = {0};
+inline cudaError_t ensure_smem_limit(K kernel, int bytes, int (&done)[kSmemRecordDevices]) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSmemRecordDevices)
         return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (done[dev] >= bytes) return cudaSuccess;
     const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

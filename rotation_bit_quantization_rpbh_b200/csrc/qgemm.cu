@@ -109,26 +109,29 @@ __host__ __device__ constexpr int dec_stage_bytes(bool av) { return av ? DEC_B :
 __host__ __device__ constexpr int pk_stage_bytes(int ba, int bw, bool f8, bool av) {
     return (av ? 0 : HM * pk_row_bytes(ba, f8)) + HN * pk_row_bytes(bw, f8);
 }
-__host__ __device__ constexpr int av_stages(int bw, bool f8, bool av) {
+// A-values stages hold mb boxes (one per 256-row half of a 256 * mb row tile)
+__host__ __device__ constexpr int av_stages(int bw, bool f8, bool av, int mb = 1) {
     return !av ? 0
-               : ((227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) / DEC_A <
+               : ((227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) / (mb * DEC_A) <
                           AV_MAX
-                      ? (227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) / DEC_A
+                      ? (227 * 1024 - 3072 - d_stages(true) * DEC_B - PK_MIN_AV * HN * pk_row_bytes(bw, f8)) /
+                            (mb * DEC_A)
                       : AV_MAX);
 }
-__host__ __device__ constexpr int rings_bytes(int bw, bool f8, bool av) {
-    return d_stages(av) * dec_stage_bytes(av) + av_stages(bw, f8, av) * DEC_A;
+__host__ __device__ constexpr int rings_bytes(int bw, bool f8, bool av, int mb = 1) {
+    return d_stages(av) * dec_stage_bytes(av) + av_stages(bw, f8, av, mb) * mb * DEC_A;
 }
-__host__ __device__ constexpr int p_stages(int ba, int bw, bool f8, bool av) {
-    return (227 * 1024 - rings_bytes(bw, f8, av) - 3072) / pk_stage_bytes(ba, bw, f8, av) < P_MAX
-               ? (227 * 1024 - rings_bytes(bw, f8, av) - 3072) / pk_stage_bytes(ba, bw, f8, av)
+__host__ __device__ constexpr int p_stages(int ba, int bw, bool f8, bool av, int mb = 1) {
+    return (227 * 1024 - rings_bytes(bw, f8, av, mb) - 3072) / pk_stage_bytes(ba, bw, f8, av) < P_MAX
+               ? (227 * 1024 - rings_bytes(bw, f8, av, mb) - 3072) / pk_stage_bytes(ba, bw, f8, av)
                : P_MAX;
 }
 // decoded ring | A-values ring (av) | packed ring | epilogue r and bias of a
 // tile (1 KB) | barriers (512 B) | alignment slack (1 KB); the 6-bit tables
 // are static
-__host__ __device__ constexpr int smem_bytes(int ba, int bw, bool f8, bool av) {
-    return rings_bytes(bw, f8, av) + p_stages(ba, bw, f8, av) * pk_stage_bytes(ba, bw, f8, av) + 1024 + 512 + 1024;
+__host__ __device__ constexpr int smem_bytes(int ba, int bw, bool f8, bool av, int mb = 1) {
+    return rings_bytes(bw, f8, av, mb) + p_stages(ba, bw, f8, av, mb) * pk_stage_bytes(ba, bw, f8, av) + 1024 + 512 +
+           1024;
 }
 
 struct QgemmParams {
@@ -136,6 +139,7 @@ struct QgemmParams {
     CUtensorMap tmB;
     int M, N, KB, num_m, num_n, num_tiles;
     int n_fastest;                // tile order: N tiles fastest (A's values stay in L2 while W's codes cycle)
+    int mb;                       // 256-row A boxes per tile (2: 512-row tiles; A as values only)
     const float* s;
     const uint16_t* w_r;
     const uint16_t* bias;
@@ -564,7 +568,12 @@ struct RingPos {
 };
 
 // ----------------------------------------------------------------------------
-template <int BA, int BW, bool F8, bool AV>
+// MB: 256-row A boxes per tile (AV only).  With MB = 2 a pair computes a
+// 512 x 256 tile: each decoded W stage feeds the MMAs of two A boxes, into
+// the two TMEM accumulators, which halves the W decoding and the stage
+// hand-offs per flop; the accumulators are then not double-buffered across
+// tiles.
+template <int BA, int BW, bool F8, bool AV, int MB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     qgemm_kernel(const __grid_constant__ QgemmParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -572,16 +581,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int PKA = AV ? 0 : HM * pk_row_bytes(BA, F8);  // A's share of a packed stage
     constexpr int PK_STAGE = pk_stage_bytes(BA, BW, F8, AV);
-    constexpr int P_STAGES = p_stages(BA, BW, F8, AV);
+    static_assert(MB == 1 || (MB == 2 && AV), "two A boxes per tile with A given as values only");
+    constexpr int P_STAGES = p_stages(BA, BW, F8, AV, MB);
     constexpr int D_STAGES = d_stages(AV);
-    constexpr int AV_STAGES = AV ? av_stages(BW, F8, AV) : 1;
+    constexpr int AV_STAGES = AV ? av_stages(BW, F8, AV, MB) : 1;
+    constexpr int AV_STAGE = MB * DEC_A;         // bytes of one A-values stage
+    constexpr int TMT = TM * MB;                  // rows of A per tile
     static_assert(P_STAGES >= NGROUPS && D_STAGES >= NGROUPS && (!AV || AV_STAGES >= NGROUPS),
                   "each decoder group starts on a stage of its own");
     constexpr int DSTAGE = dec_stage_bytes(AV);  // decoded stage: A then W, or W alone (AV)
     constexpr int DOFF_B = AV ? 0 : DEC_A;       // offset of W's values in a decoded stage
     uint8_t* dec = smem;
     uint8_t* av = smem + D_STAGES * DSTAGE;      // A-values ring (AV): 1024-byte aligned stages for the swizzled TMA
-    uint8_t* pk = smem + rings_bytes(BW, F8, AV);
+    uint8_t* pk = smem + rings_bytes(BW, F8, AV, MB);
     uint16_t* epi_r = reinterpret_cast<uint16_t*>(pk + P_STAGES * PK_STAGE);  // r_n of the tile's 256 columns
     uint16_t* epi_b = epi_r + TN;   // bias of those columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_b + TN);
@@ -658,7 +670,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 int mt, nt;
                 tile_mn(p, tile, mt, nt);
-                const int m0 = mt * TM + (int)rank * HM;
+                const int m0 = mt * TMT + (int)rank * HM;
                 const int n0 = nt * TN + (int)rank * HN;
                 for (int kb = 0; kb < p.KB; ++kb) {
                     if (!wait_or_abort<false>(&pk_empty[ps.idx], ps.phase ^ 1u, abort_flag)) {
@@ -678,8 +690,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&av_full[as.idx], DEC_A);
-                        tma_load_2d(av + as.idx * DEC_A, &p.tmA, kb * 128, m0, &av_full[as.idx]);
+                        mbar_arrive_expect_tx(&av_full[as.idx], AV_STAGE);
+#pragma unroll
+                        for (int h = 0; h < MB; ++h)  // box h: rows 256 h + 128 rank of the tile
+                            tma_load_2d(av + as.idx * AV_STAGE + h * DEC_A, &p.tmA, kb * 128, m0 + h * TM,
+                                        &av_full[as.idx]);
                         ++issued_av;
                         as.advance();
                     }
@@ -703,8 +718,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             int acc_it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++acc_it) {
-                const int a = acc_it & 1;
-                if (!wait_or_abort<true>(&acc_empty[a], ((acc_it >> 1) & 1) ^ 1, abort_flag)) break;
+                // MB = 1: the accumulators alternate between tiles; MB = 2: box h
+                // of every tile accumulates into accumulator h
+                const int a = MB == 2 ? 0 : (acc_it & 1);
+                const uint32_t eph = MB == 2 ? ((uint32_t)acc_it & 1u) ^ 1u : (((uint32_t)acc_it >> 1) & 1u) ^ 1u;
+                if (!wait_or_abort<true>(&acc_empty[a], eph, abort_flag)) break;
+                if (MB == 2 && !wait_or_abort<true>(&acc_empty[1], eph, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(a * TN);
                 for (int kb = 0; kb < p.KB; ++kb) {
@@ -715,13 +734,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     tc_fence_after();
                     // (AV: the stage's "full" signal also covers A's values in both CTAs,
                     // since each CTA's decoders publish only after their A load landed)
-                    const uint32_t a_base = AV ? smem_u32(av + as.idx * DEC_A) : smem_u32(dec + ds.idx * DSTAGE);
+                    const uint32_t a_base = AV ? smem_u32(av + as.idx * AV_STAGE) : smem_u32(dec + ds.idx * DSTAGE);
                     const uint32_t b_base = smem_u32(dec + ds.idx * DSTAGE) + DOFF_B;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 32 bytes of each 128-byte row per MMA
-                        tc_mma_pair<F8>(d_tmem, sw128_desc(a_base + 32 * k), sw128_desc(b_base + 32 * k),
-                                        F8 ? kIdescE4m3 : kIdescBf16,
-                                    (kb | k) != 0 ? 1u : 0u);
+                    for (int h = 0; h < MB; ++h)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)  // 32 bytes of each 128-byte row per MMA
+                            tc_mma_pair<F8>(d_tmem + (uint32_t)(h * TN), sw128_desc(a_base + h * DEC_A + 32 * k),
+                                            sw128_desc(b_base + 32 * k), F8 ? kIdescE4m3 : kIdescBf16,
+                                            (kb | k) != 0 ? 1u : 0u);
                     tc_commit_pair(&dec_empty[ds.idx]);
                     if constexpr (AV) {
                         tc_commit_pair(&av_empty[as.idx]);
@@ -729,7 +750,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     }
                     ds.advance();
                 }
-                if (ok) tc_commit_pair(&acc_full[a]);
+                if (ok) {
+                    tc_commit_pair(&acc_full[a]);
+                    if (MB == 2) tc_commit_pair(&acc_full[1]);
+                }
             }
         }
     } else if (warp < 2 + NDEC_WARPS) {
@@ -845,9 +869,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int tile = pair; tile < p.num_tiles; tile += npairs, ++acc_it) {
             int mt, nt;
             tile_mn(p, tile, mt, nt);
-            const int m0 = mt * TM + (int)rank * HM, n0 = nt * TN;
-            const int a = acc_it & 1;
-            if (!wait_or_abort<false>(&acc_full[a], (acc_it >> 1) & 1, abort_flag)) break;
+            const int n0 = nt * TN;
+            // MB = 1: accumulator acc_it & 1, phase (acc_it >> 1) & 1; MB = 2:
+            // accumulators 0 and 1 (the tile's two 256-row halves), phase acc_it & 1
+            const int a0 = MB == 2 ? 0 : (acc_it & 1);
+            const uint32_t fph = MB == 2 ? ((uint32_t)acc_it & 1u) : (((uint32_t)acc_it >> 1) & 1u);
+            if (!wait_or_abort<false>(&acc_full[a0], fph, abort_flag)) break;
             tc_fence_after();
             epilogue_sync();  // the previous tile's reads of epi_r / epi_b are done
             for (int j = et; j < TN; j += 128) {
@@ -856,6 +883,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 epi_b[j] = (p.bias && n < p.N) ? p.bias[n] : (uint16_t)0;
             }
             epilogue_sync();
+            bool drained = true;
+            for (int h = 0; h < MB; ++h) {
+            const int a = a0 + h;
+            if (h > 0) {
+                if (!wait_or_abort<false>(&acc_full[a], fph, abort_flag)) {
+                    drained = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            const int m0 = mt * TMT + h * TM + (int)rank * HM;
             const int row = m0 + q * 32 + lane;
             const bool row_ok = row < p.M;
             const float sm = row_ok ? p.s[row] * p.out_scale : 0.f;
@@ -907,6 +945,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc_empty_leader + (uint32_t)(a * sizeof(uint64_t)));
+            }
+            if (!drained) break;
         }
     }
 
@@ -1036,11 +1076,12 @@ void fill_tables_e4m3(int bits, const uint8_t* e, uint32_t tab[4], uint8_t* c6) 
     }
 }
 
-template <int BA, int BW, bool F8, bool AV = false>
+template <int BA, int BW, bool F8, bool AV = false, int MB = 1>
 cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
-    auto k = qgemm_kernel<BA, BW, F8, AV>;
-    const int smem = smem_bytes(BA, BW, F8, AV);
-    const cudaError_t e = ensure_smem_limit(k, smem);
+    auto k = qgemm_kernel<BA, BW, F8, AV, MB>;
+    const int smem = smem_bytes(BA, BW, F8, AV, MB);
+    static int smem_done[kSmemRecordDevices] = {0};  // this instantiation's limit, per device
+    const cudaError_t e = ensure_smem_limit(k, smem, smem_done);
     if (e != cudaSuccess) return e;
     const cudaError_t le = launch_pdl(k, dim3(grid), dim3(NTHREADS), smem, stream, prm);
     if (le != cudaSuccess) return le;
@@ -1049,7 +1090,14 @@ cudaError_t launch_qgemm_t(QgemmParams& prm, int grid, cudaStream_t stream) {
 
 template <bool F8>
 cudaError_t launch_bits(const QgemmArgs& a, QgemmParams& prm, int grid, cudaStream_t stream) {
-    if (a.a_val) {  // A given as values: only W's width selects the kernel
+    if (a.a_val) {  // A given as values: only W's width (and the tile height) selects the kernel
+        if (prm.mb == 2) {
+            if (a.bits_w == 4) return launch_qgemm_t<0, 4, F8, true, 2>(prm, grid, stream);
+            if (a.bits_w == 2) return launch_qgemm_t<0, 2, F8, true, 2>(prm, grid, stream);
+            if (a.bits_w == 6) return launch_qgemm_t<0, 6, F8, true, 2>(prm, grid, stream);
+            if (a.bits_w == 3) return launch_qgemm_t<0, 3, F8, true, 2>(prm, grid, stream);
+            return cudaErrorInvalidValue;
+        }
         if (a.bits_w == 4) return launch_qgemm_t<0, 4, F8, true>(prm, grid, stream);
         if (a.bits_w == 2) return launch_qgemm_t<0, 2, F8, true>(prm, grid, stream);
         if (a.bits_w == 6) return launch_qgemm_t<0, 6, F8, true>(prm, grid, stream);
@@ -1086,6 +1134,10 @@ int qgemm_sm_count() {
 
 }  // namespace
 
+static int g_force_mb = 0;  // tuning hook: forced tile height (0: chosen per shape)
+
+void qgemm_force_tile_rows(int rows) { g_force_mb = rows == 512 ? 2 : (rows == 256 ? 1 : 0); }
+
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     QgemmParams prm;
     std::memset(&prm, 0, sizeof(prm));
@@ -1102,8 +1154,19 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     prm.M = a.M;
     prm.N = a.N;
     prm.KB = a.K / bk_codes(f8);
-    prm.num_m = (a.M + TM - 1) / TM;
     prm.num_n = (a.N + TN - 1) / TN;
+    // tile height: 512 rows (two A boxes per decoded W stage) when A arrives
+    // as values and the tiles still fill the SM pairs' waves about as well
+    // as 256-row tiles do (taken as forced by the tuning hook when set)
+    const int pairs_max = qgemm_sm_count() / 2;
+    auto wave_eff = [&](int tiles) {
+        const int waves = (tiles + pairs_max - 1) / pairs_max;
+        return (double)tiles / (double)(waves * pairs_max);
+    };
+    const int t1 = ((a.M + TM - 1) / TM) * prm.num_n, t2 = ((a.M + 2 * TM - 1) / (2 * TM)) * prm.num_n;
+    prm.mb = (a.a_val && wave_eff(t2) >= wave_eff(t1) - 0.02) ? 2 : 1;
+    if (a.a_val && g_force_mb) prm.mb = g_force_mb;
+    prm.num_m = (a.M + prm.mb * TM - 1) / (prm.mb * TM);
     prm.num_tiles = prm.num_m * prm.num_n;
     // A's values are 2 (e4m3: 1) bytes per element, more than L2 holds at the
     // larger shapes: N-fastest order keeps the few A tiles in use resident
@@ -1123,7 +1186,6 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
         if (!a.a_val) fill_tables(a.bits_a, a.ca_bf16, prm.tab_a, prm.c6a);
         fill_tables(a.bits_w, a.cw_bf16, prm.tab_w, prm.c6w);
     }
-    const int pairs_max = qgemm_sm_count() / 2;
     const int pairs = prm.num_tiles < pairs_max ? prm.num_tiles : pairs_max;
     return f8 ? launch_bits<true>(a, prm, 2 * pairs, stream) : launch_bits<false>(a, prm, 2 * pairs, stream);
 }

@@ -26,4 +26,8 @@ struct QgemmArgs {
 
 cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream);
 
+// Test and tuning hook: force the tile height of the A-values product
+// (256 or 512 rows; 0: chosen per shape).
+void qgemm_force_tile_rows(int rows);
+
 }  // namespace oq

@@ -275,7 +275,8 @@ template <typename InT, int BITS, int MODE>
 cudaError_t launch_big_t(const RpbhParams& p, int kh, int grid, cudaStream_t stream) {
     auto k = rht_big_kernel<InT, BITS, MODE>;
     const int smem = big_layout(p).total;
-    const cudaError_t e = ensure_smem_limit(k, smem);
+    static int smem_done[kSmemRecordDevices] = {0};  // this instantiation's limit, per device
+    const cudaError_t e = ensure_smem_limit(k, smem, smem_done);
     if (e != cudaSuccess) return e;
     const cudaError_t le = launch_pdl(k, dim3(grid), dim3(kBigThreads), smem, stream, p, kh);
     if (le != cudaSuccess) return le;

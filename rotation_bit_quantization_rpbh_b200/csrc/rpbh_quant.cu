@@ -104,39 +104,48 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Lookup-table entry at a 32-bit shared-memory address: {T, base or values}.
+// Its address depends on the gathered values, which are loaded after the
+// table's mbarrier wait, so it cannot move above that wait; it is left free
+// to be scheduled (and merged) otherwise.
 __device__ __forceinline__ void lut_ld(uint32_t addr, float& T, uint32_t& w) {
     asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(T), "=r"(w) : "r"(addr));
 }
 
-// Shared-memory loads at 32-bit shared addresses (explicit ld.shared: the
-// staged rows change between iterations, so these are ordered after the
-// mbarrier waits by being volatile).
+// Shared-memory loads at 32-bit shared addresses (explicit ld.shared).  The
+// tables and staged rows arrive by bulk copy, so every load that reads them
+// is volatile with a memory clobber: it stays after the mbarrier wait that
+// covers the copy (a load whose address depends on nothing loaded after the
+// wait could otherwise be moved above it, or out of the loop).
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
 }
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
 }
 
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
     uint4 v;
-    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
     return v;
 }
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
 }
 
-template <typename InT, int H, int BITS, int MODE>
-__global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid_constant__ RpbhParams p) {
+template <typename InT, int H, int BITS, int MODE, int SPL>
+__global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
+    rpbh_quant_kernel(const __grid_constant__ RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout(p);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
@@ -145,8 +154,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = warp / p.team, wt = warp - t * p.team;  // team, warp within the team
+    // SPL lanes per h-block: lane = ((r * Bw + j) * SPL + hf); with two, each
+    // lane holds half of the block's values (see the gather)
+    constexpr int LSPL = SPL == 2 ? 1 : 0;
+    const int hf = lane & (SPL - 1);
     const int Bw = 1 << p.lbw;
-    const int j = lane & (Bw - 1), r = lane >> p.lbw;     // block within the warp, row within the set
+    const int j = (lane >> LSPL) & (Bw - 1), r = lane >> (LSPL + p.lbw);  // block within the warp, row within the set
     const int b = wt * Bw + j;                            // h-block of this lane
     const bool bact = b < p.nb;
     const bool loader = wt == 0 && lane == 0;             // issues the team's row copies
@@ -156,7 +169,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
     uint8_t* my_stage = smem + L.stage + t * p.slots * p.RW * p.srow;
     float* my_part = reinterpret_cast<float*>(smem + L.part) + t * 2 * p.team * p.RW;
     constexpr int ES = sizeof(InT);
-    constexpr int L2H = H / 2;
+    static_assert(SPL == 1 || ES == 2, "two lanes per block exchange bf16 inputs");
+    constexpr int HL = H / SPL;  // values per lane
+    constexpr int L2H = HL / 2;
 
     // this team's row sets: g = k * (gridDim.x * tpc) + t * gridDim.x + blockIdx.x
     const int stride = gridDim.x * p.tpc;
@@ -243,7 +258,43 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
         // (||x'|| = ||x|| since Pi_d is orthogonal)
         float2 v2[L2H];
         float2 acc = make_float2(0.f, 0.f);
-        if (valid) {
+        if constexpr (SPL == 2) {
+            // the lane's half of the block: entries hf*HL .. hf*HL + HL-1, kept
+            // as signed bf16 pairs; the pair of lanes swaps them (every lane
+            // takes part in the shuffles) and runs the top butterfly stage
+            // across the pair: the low lane takes u_lo + u_hi, the high lane
+            // u_lo - u_hi (H_128 = [[H64, H64], [H64, -H64]])
+            uint32_t pk[L2H];
+            if (valid) {
+                const uint32_t rowp = stage_addr + (uint32_t)(slot * p.RW * p.srow + r * p.srow);
+                const uint32_t tabp = gtab_addr + (uint32_t)b * 16u + (uint32_t)(hf * (HL / 4) * p.nb) * 16u;
+#pragma unroll
+                for (int c4 = 0; c4 < HL / 4; ++c4) {
+                    const uint4 ch = lds_v4(tabp + (uint32_t)(c4 * p.nb) * 16u);
+                    const uint32_t e[4] = {ch.x, ch.y, ch.z, ch.w};
+                    uint32_t sv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sv[q] = lds_u16(rowp + (e[q] >> 16)) + e[q];  // bit 15: sign of D
+                    pk[2 * c4] = prmt_b32(sv[0], sv[1], 0x5410u);
+                    pk[2 * c4 + 1] = prmt_b32(sv[2], sv[3], 0x5410u);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < L2H; ++i) pk[i] = 0u;
+            }
+            const float2 sgn2 = hf ? make_float2(-1.f, -1.f) : make_float2(1.f, 1.f);
+#pragma unroll
+            for (int k2 = 0; k2 < L2H; ++k2) {
+                const uint32_t o = __shfl_xor_sync(0xffffffffu, pk[k2], 1);
+                const float2 own = make_float2(__uint_as_float(pk[k2] << 16), __uint_as_float(pk[k2] & 0xffff0000u));
+                const float2 oth = make_float2(__uint_as_float(o << 16), __uint_as_float(o & 0xffff0000u));
+                acc = f2fma(own, own, acc);
+                v2[k2] = f2fma(own, sgn2, oth);
+            }
+        } else if (!valid) {
+#pragma unroll
+            for (int i = 0; i < L2H; ++i) v2[i] = make_float2(0.f, 0.f);
+        } else {
             const uint32_t rowp = stage_addr + (uint32_t)(slot * p.RW * p.srow + r * p.srow);
             const uint32_t tabp = gtab_addr + (uint32_t)b * 16u;
 #pragma unroll
@@ -268,9 +319,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
                 acc = f2fma(v2[2 * c4], v2[2 * c4], acc);
                 acc = f2fma(v2[2 * c4 + 1], v2[2 * c4 + 1], acc);
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < L2H; ++i) v2[i] = make_float2(0.f, 0.f);
         }
         // this warp is done with the slot
         __syncwarp();
@@ -279,7 +327,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
         // warp has gathered from it (now if they have, else later)
         const int gn = g + p.slots * stride;
         if (loader && gn < p.nrs) {
-            if (mbar_try_wait(&my_empty[slot], ph)) {
+            if (mbar_test_wait(&my_empty[slot], ph)) {
                 issue(slot, gn, k + p.slots);
             } else {
                 pend_slot = slot;
@@ -291,10 +339,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
 
         // ---- A4 (first half): the row's sum of squares over this warp's blocks ----
         float ss = acc.x + acc.y;
-        for (int o = 1; o < Bw; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        for (int o = 1; o < (Bw << LSPL); o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         float* part = my_part + (k & 1) * p.team * p.RW;
         if (p.team > 1) {
-            if (j == 0) part[wt * p.RW + r] = ss;
+            if (j == 0 && hf == 0) part[wt * p.RW + r] = ss;
             __syncwarp();
             if (lane == 0) mbar_arrive(&my_norm[k & 1]);
         }
@@ -318,7 +366,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
         }
 
         // a deferred refill may be possible by now
-        if (loader && pend_slot >= 0 && mbar_try_wait(&my_empty[pend_slot], pend_ph)) {
+        if (loader && pend_slot >= 0 && mbar_test_wait(&my_empty[pend_slot], pend_ph)) {
             issue(pend_slot, pend_g, pend_k);
             pend_slot = -1;
         }
@@ -337,13 +385,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
         const float s = __fsqrt_rn(ssum);
 
         if (valid) {
-            if (b == 0) {
+            if (b == 0 && hf == 0) {
                 if constexpr (MODE == 0 || MODE >= 3) p.s_out[row] = s;
                 if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
                 if constexpr (MODE == 2) p.norm_out[row] = s;
             }
             if constexpr (MODE == 2) {
-                float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + b * H);
+                float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + b * H + hf * HL);
                 const float2 sc = make_float2(p.rsqrt_h, p.rsqrt_h);
 #pragma unroll
                 for (int i = 0; i < L2H; i += 2) {
@@ -356,7 +404,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
                 // give (the cell below the bin's threshold and the one above),
                 // so one compare selects c_index directly ----------------------
                 constexpr int VB = MODE == 3 ? 2 : 1;  // bytes per value: bf16, or e4m3
-                uint4* dst = reinterpret_cast<uint4*>(p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * H * VB);
+                uint4* dst = reinterpret_cast<uint4*>(p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * H * VB +
+                                                      (size_t)hf * HL * VB);
                 if (s <= p.s_max) {
                     const float inv = p.rsqrt_h / (s + p.eps);
                     const float2 inv2 = make_float2(inv, inv);
@@ -371,7 +420,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
                         ge1 = q.y >= T1 ? 1u : 0u;
                     };
 #pragma unroll
-                    for (int w0 = 0; w0 < H * VB / 4; w0 += 4) {
+                    for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) {
                         uint32_t words[4];
 #pragma unroll
                         for (int wj = 0; wj < 4; ++wj) {
@@ -396,16 +445,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
                     // the middle cell's value everywhere (see the codes branch)
                     const uint32_t wm = VB == 2 ? p.mid_val * 0x10001u : p.mid_val * 0x01010101u;
 #pragma unroll
-                    for (int w0 = 0; w0 < H * VB / 4; w0 += 4) dst[w0 >> 2] = make_uint4(wm, wm, wm, wm);
+                    for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) dst[w0 >> 2] = make_uint4(wm, wm, wm, wm);
                 }
             } else {
                 // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
-                constexpr int NB = BITS == 6 ? H : H * BITS / 8;  // packed bytes per h-block
+                constexpr int NB = BITS == 6 ? HL : HL * BITS / 8;  // packed bytes of the lane's codes
                 constexpr int NW = NB / 4;
                 constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
                 constexpr int PER = BITS == 6 ? 4 : (BITS == 3 ? 8 : 32 / BITS);  // codes per word (3-bit: per 24-bit group)
                 constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
-                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB;
+                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB * SPL + (size_t)hf * NB;
                 auto put = [&](int w0, const uint32_t (&words)[CW]) {
                     if constexpr (CW == 4)
                         reinterpret_cast<uint4*>(dst)[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
@@ -435,7 +484,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
                     const float2 inv2 = make_float2(inv, inv);
                     uint32_t words[NW];
 #pragma unroll
-                    for (int g4 = 0; g4 < H / 32; ++g4) {
+                    for (int g4 = 0; g4 < HL / 32; ++g4) {
                         uint32_t grp[4];
 #pragma unroll
                         for (int gi = 0; gi < 4; ++gi) {
@@ -518,15 +567,24 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rpbh_quant_kernel(const __grid
     if (tid == 0 && !p.starve) mbar_wait_bounded(tab_bar, 0u);
 }
 
-template <typename InT, int H, int BITS, int MODE>
-cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
-    auto k = rpbh_quant_kernel<InT, H, BITS, MODE>;
+template <typename InT, int H, int BITS, int MODE, int SPL>
+cudaError_t launch_rpbh_spl(const RpbhParams& p, int grid, cudaStream_t stream) {
+    auto k = rpbh_quant_kernel<InT, H, BITS, MODE, SPL>;
     const int smem = smem_layout(p).total;
-    const cudaError_t e = ensure_smem_limit(k, smem);
+    static int smem_done[kSmemRecordDevices] = {0};  // this instantiation's limit, per device
+    const cudaError_t e = ensure_smem_limit(k, smem, smem_done);
     if (e != cudaSuccess) return e;
     const cudaError_t le = launch_pdl(k, dim3(grid), dim3(p.tpc * p.team * 32), smem, stream, p);
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
+}
+
+// two lanes per block: bf16 inputs, blocks of 64 or 128
+template <typename InT, int H, int BITS, int MODE>
+cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
+    if constexpr (sizeof(InT) == 2 && H >= 64)
+        if (p.SPL == 2) return launch_rpbh_spl<InT, H, BITS, MODE, 2>(p, grid, stream);
+    return launch_rpbh_spl<InT, H, BITS, MODE, 1>(p, grid, stream);
 }
 
 template <typename InT, int H, int MODE>
@@ -573,11 +631,12 @@ int rpbh_smem_bytes(const RpbhParams& p) { return smem_layout(p).total; }
 // team (the next row set streams in during the whole computation of this
 // one), then the one with the most rows per warp.  A forced layout (test
 // and tuning hook) is taken when it fits.
-static int g_force_rw = 0, g_force_slots = 0;
+static int g_force_rw = 0, g_force_slots = 0, g_force_spl = 0;
 
-void rpbh_force_layout(int rows_per_warp, int slots) {
+void rpbh_force_layout(int rows_per_warp, int slots, int lanes_per_block) {
     g_force_rw = rows_per_warp;
     g_force_slots = slots;
+    g_force_spl = lanes_per_block;
 }
 
 bool rpbh_choose_layout(RpbhParams& p, int h, int esize) {
@@ -585,26 +644,36 @@ bool rpbh_choose_layout(RpbhParams& p, int h, int esize) {
     p.row_bytes = p.d * esize;
     RpbhParams best = p;
     int best_key = -1;
-    for (int slots = 2; slots >= 1; --slots) {
-        for (int RW = 8; RW >= 1; RW >>= 1) {
-            if (g_force_rw && RW != g_force_rw) continue;
-            if (g_force_slots && slots != g_force_slots) continue;
-            const int Bw = 32 / RW;
-            const int team = (nb + Bw - 1) / Bw;
-            if (team > kMaxWarps) continue;
-            RpbhParams c = p;
-            c.RW = RW;
-            c.lbw = RW == 8 ? 2 : (RW == 4 ? 3 : (RW == 2 ? 4 : 5));
-            c.team = team;
-            c.slots = slots;
-            c.srow = c.row_bytes + (RW == 1 ? 16 : 128 / RW);
-            for (c.tpc = kMaxWarps / team; c.tpc >= 1; --c.tpc)
-                if (rpbh_smem_bytes(c) <= kSmemLimit) break;
-            if (c.tpc < 1) continue;
-            const int key = (c.tpc * team) * 100 + slots * 10 + RW;
-            if (key > best_key) {
-                best_key = key;
-                best = c;
+    // two lanes per block (more warps per SM, half the registers) only for
+    // bf16 inputs and blocks of 64 or 128, and only when forced for now
+    const int spl_max = (esize == 2 && h >= 64 && g_force_spl == 2) ? 2 : 1;
+    for (int spl = spl_max; spl >= 1; --spl) {
+        const int max_warps = spl == 2 ? kMaxWarpsSplit : kMaxWarps;
+        for (int slots = 2; slots >= 1; --slots) {
+            for (int RW = 8; RW >= 1; RW >>= 1) {
+                if (g_force_rw && RW != g_force_rw) continue;
+                if (g_force_slots && slots != g_force_slots) continue;
+                const int Bw = 32 / (RW * spl);
+                if (Bw < 1) continue;
+                const int team = (nb + Bw - 1) / Bw;
+                if (team > max_warps) continue;
+                RpbhParams c = p;
+                c.SPL = spl;
+                c.RW = RW;
+                int lbw = 0;
+                while ((1 << lbw) < Bw) ++lbw;
+                c.lbw = lbw;
+                c.team = team;
+                c.slots = slots;
+                c.srow = c.row_bytes + (RW == 1 ? 16 : 128 / RW);
+                for (c.tpc = max_warps / team; c.tpc >= 1; --c.tpc)
+                    if (rpbh_smem_bytes(c) <= kSmemLimit) break;
+                if (c.tpc < 1) continue;
+                const int key = spl * 100000 + (c.tpc * team) * 100 + slots * 10 + RW;
+                if (key > best_key) {
+                    best_key = key;
+                    best = c;
+                }
             }
         }
     }

@@ -16,6 +16,7 @@ struct RpbhParams {
     // of a set of RW rows; a CTA holds `tpc` teams, each with `slots`
     // staging slots of RW rows.
     int RW, lbw;          // rows per warp; log2 of the blocks per warp
+    int SPL;              // lanes per h-block: 1, or 2 (each holds half the block's values)
     int team, tpc, slots;
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
     int nrs;              // row sets: ceil(M / RW)
@@ -39,6 +40,8 @@ struct RpbhParams {
 
 constexpr int kMaxWarps = 12;                 // per CTA: the kernel's launch bound is 384 threads
 constexpr int kMaxThreads = kMaxWarps * 32;   // (168 registers each)
+constexpr int kMaxWarpsSplit = 16;            // with two lanes per block: 512 threads
+constexpr int kMaxThreadsSplit = kMaxWarpsSplit * 32;  // (128 registers each)
 constexpr int kSmemLimit = 227 * 1024;
 
 int rpbh_smem_bytes(const RpbhParams& p);
@@ -49,8 +52,9 @@ int rpbh_smem_bytes(const RpbhParams& p);
 // order).  Returns false if no layout fits in shared memory.
 bool rpbh_choose_layout(RpbhParams& p, int h, int esize);
 
-// Test and tuning hook: force rows per warp and slots per team (0: automatic).
-void rpbh_force_layout(int rows_per_warp, int slots);
+// Test and tuning hook: force rows per warp, slots per team and lanes per
+// block (0: automatic).
+void rpbh_force_layout(int rows_per_warp, int slots, int lanes_per_block);
 
 // The kernel for blocks of 256 ... 16384 (rht_big.cu): one row per CTA at a
 // time; RW, team, tpc, slots and srow are not used.

@@ -437,3 +437,30 @@ def test_eight_bit_activations_match_oracle(cuda_device):
             ca, cw = oracle.round_bf16(ocb_a[0])[1], oracle.round_bf16(ocb_w[0])[1]
         ref = gemm_reference(ia, s64, iw, r64, ca, cw)
         check_product(y.float().cpu().numpy().astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("M,d,N,bw,fp8", [(300, 512, 520, 4, False), (700, 256, 264, 2, False),
+                                          (513, 384, 200, 6, False), (257, 512, 136, 4, True),
+                                          (1100, 768, 512, 3, False)])
+def test_tall_tiles_give_the_same_product(cuda_device, M, d, N, bw, fp8):
+    """The A-values product in 512-row tiles (two A boxes per decoded W
+    stage, both accumulators) against 256-row tiles: the same MMAs in the
+    same order per output element, so the same bits; ragged M and N."""
+    g = torch.Generator().manual_seed(M + N)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16)
+    plan = B.rpbh_plan(d, 128, 7)
+    cb_a, cb_w = B.codebook(d, 4), B.codebook(d, bw)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W.to(cuda_device))
+    val, s = B.quantize_acts_values(plan, cb_a, x.to(cuda_device), fp8=fp8)
+    bias = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16).to(cuda_device)
+    try:
+        B.debug_qgemm_tile_rows(256)
+        y1 = B.qgemm_values(cb_w, val, s, w_idx, w_r, bias=bias, fp8=fp8)
+        B.debug_qgemm_tile_rows(512)
+        y2 = B.qgemm_values(cb_w, val, s, w_idx, w_r, bias=bias, fp8=fp8)
+    finally:
+        B.debug_qgemm_tile_rows(0)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert torch.equal(y1, y2)
