@@ -658,12 +658,24 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+def full_rht_block(d):
+    """Full RHT: one Walsh-Hadamard block over all of d.  Sylvester matrices
+    exist for powers of two only, so for other d the largest power-of-two
+    block that divides d (3072 -> 1024, 12288 -> 4096, 1536 -> 512)."""
+    h = 1
+    while d % (2 * h) == 0 and 2 * h <= 16384:
+        h *= 2
+    return h
+
+
 def run_ablation(args):
     """The page's rotation ablation on one GPU: the fused rotate+quantise
-    kernel with the RPBH plan and with the Block-RHT plan (no permutation),
-    the rotation alone for both (oq_rpbh_apply), and a dense Haar rotation
-    (a cuBLAS bf16 GEMM against a random orthogonal d x d matrix).  Median
-    device time per call over --steps calls, L2 flushed before each."""
+    kernel and the rotation alone (oq_rpbh_apply) with the RPBH plan, the
+    Block-RHT plan (no permutation: each block read contiguously), the Full
+    RHT plan (no permutation, one block over d, or the largest power-of-two
+    block of d), and a dense Haar rotation (a cuBLAS bf16 GEMM against a
+    random orthogonal d x d matrix).  Median device time per call over
+    --steps calls, L2 flushed before each."""
     import numpy as np
     import torch
 
@@ -676,10 +688,11 @@ def run_ablation(args):
     w = I.WORKLOADS[args.workload]
     x = I.make_x(w).to(dev)
     cb_a = B.codebook(w.d, w.bits_a)
+    hf = full_rht_block(w.d)
     plans = {"rpbh": B.rpbh_plan(w.d, w.h, w.plan_seed),
-             "block_rht": B.rotation_plan(w.d, w.h, w.plan_seed, B.OQ_ROT_BLOCK_RHT)}
-    packed = w.d if w.bits_a == 6 else w.d * w.bits_a // 8
-    a_idx = torch.empty((w.M, packed), dtype=torch.uint8, device=dev)
+             "block_rht": B.rotation_plan(w.d, w.h, w.plan_seed, B.OQ_ROT_BLOCK_RHT),
+             "full_rht": B.rotation_plan(w.d, hf, w.plan_seed, B.OQ_ROT_BLOCK_RHT)}
+    a_idx = torch.empty((w.M, B.packed_row_bytes(w.d, w.bits_a)), dtype=torch.uint8, device=dev)
     s = torch.empty(w.M, dtype=torch.float32, device=dev)
     x_rot = torch.empty((w.M, w.d), dtype=torch.float32, device=dev)
     # Haar-distributed orthogonal matrix: QR of a Gaussian matrix with the
@@ -692,13 +705,11 @@ def run_ablation(args):
     y_haar = torch.empty((w.M, w.d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    calls = {
-        "rpbh_quant": lambda: B.quantize_acts(plans["rpbh"], cb_a, x, a_idx, s, stream=stream),
-        "block_rht_quant": lambda: B.quantize_acts(plans["block_rht"], cb_a, x, a_idx, s, stream=stream),
-        "rpbh_rotate": lambda: B.rpbh_apply(plans["rpbh"], x, x_rot, s, stream=stream),
-        "block_rht_rotate": lambda: B.rpbh_apply(plans["block_rht"], x, x_rot, s, stream=stream),
-        "haar_rotate_cublas": lambda: torch.matmul(xb, haar_t, out=y_haar),
-    }
+    calls = {}
+    for name, pl in plans.items():
+        calls[f"{name}_quant"] = (lambda pl=pl: B.quantize_acts(pl, cb_a, x, a_idx, s, stream=stream))
+        calls[f"{name}_rotate"] = (lambda pl=pl: B.rpbh_apply(pl, x, x_rot, s, stream=stream))
+    calls["haar_rotate_cublas"] = lambda: torch.matmul(xb, haar_t, out=y_haar)
     ms = {}
     for name, fn in calls.items():
         for _ in range(max(3, args.warmup)):
@@ -716,15 +727,22 @@ def run_ablation(args):
         raise SystemExit("a kernel reported a timeout")
     out = {
         "metric": "rotation ablation: device ms per call (median)",
-        "workload": w.name, "M": w.M, "d": w.d, "h": w.h, "bits_a": w.bits_a, "steps": args.steps,
+        "workload": w.name, "M": w.M, "d": w.d, "h": w.h, "full_rht_h": hf, "bits_a": w.bits_a, "steps": args.steps,
         "ms": ms,
         "ratios": {
             "rpbh_over_block_rht_quant": ms["rpbh_quant"] / ms["block_rht_quant"],
             "rpbh_over_block_rht_rotate": ms["rpbh_rotate"] / ms["block_rht_rotate"],
+            "full_rht_over_rpbh_rotate": ms["full_rht_rotate"] / ms["rpbh_rotate"],
             "haar_over_rpbh_rotate": ms["haar_rotate_cublas"] / ms["rpbh_rotate"],
-            "haar_over_rpbh_quant": ms["haar_rotate_cublas"] / ms["rpbh_quant"],
+            "haar_over_block_rht_rotate": ms["haar_rotate_cublas"] / ms["block_rht_rotate"],
+            "haar_over_full_rht_rotate": ms["haar_rotate_cublas"] / ms["full_rht_rotate"],
+            # the layer's cost of a dense rotation: the Haar GEMM, then a quantise
+            # pass over its output (the Block-RHT plan's launch stands in for a
+            # quantiser without a transform), against the fused RPBH launch
+            "haar_plus_quant_over_rpbh_quant": (ms["haar_rotate_cublas"] + ms["block_rht_quant"]) / ms["rpbh_quant"],
         },
-        "note": "rotate = oq_rpbh_apply (fp32 x' and norms out); quant = the fused rotate+split+quantise kernel; "
+        "note": "rotate = oq_rpbh_apply (fp32 x' and norms out); quant = the fused rotate+split+quantise kernel "
+                "(packed codes out); Block-RHT and Full RHT read each block contiguously (no permutation); "
                 "haar = bf16 x @ Q^T with a Haar-random Q, bf16 out (cuBLAS); L2 flushed before every call",
     }
     print(json.dumps(out), flush=True)

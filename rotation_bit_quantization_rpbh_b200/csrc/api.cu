@@ -94,6 +94,7 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.d = d;
     p.nb = nb;
     p.lut_n = mode != 2 ? (int)cb->lut.size() : 0;
+    p.contig = plan->variant == OQ_ROT_BLOCK_RHT ? 1 : 0;
     if (big) {
         p.row_bytes = d * esize;
         if (rht_big_smem_bytes(p) > kSmemLimit) return OQ_ERR_UNSUPPORTED;
@@ -282,6 +283,7 @@ oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t**
     p->h = h;
     p->seed = seed;
     p->device = dev;
+    p->variant = variant;
     p->perm.resize(d);
     p->sign.resize(d);
     make_plan(d, h, seed, p->perm.data(), p->sign.data(), variant);

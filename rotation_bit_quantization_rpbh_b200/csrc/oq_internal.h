@@ -56,6 +56,7 @@ struct oq_plan_s {
     int d = 0, h = 0;
     uint64_t seed = 0;
     int device = -1;
+    int variant = 0;  // OQ_ROT_RPBH or OQ_ROT_BLOCK_RHT (identity permutation)
     std::vector<int32_t> perm;
     std::vector<int8_t> sign;
     std::vector<uint32_t> gtab_host;  // chunked gather table (see build_gather_table)

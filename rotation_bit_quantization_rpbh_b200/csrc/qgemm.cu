@@ -1155,17 +1155,11 @@ cudaError_t launch_qgemm(const QgemmArgs& a, cudaStream_t stream) {
     prm.N = a.N;
     prm.KB = a.K / bk_codes(f8);
     prm.num_n = (a.N + TN - 1) / TN;
-    // tile height: 512 rows (two A boxes per decoded W stage) when A arrives
-    // as values and the tiles still fill the SM pairs' waves about as well
-    // as 256-row tiles do (taken as forced by the tuning hook when set)
+    // tile height: 256 rows.  512-row tiles (two A boxes per decoded W
+    // stage) give the same bits but measured about half the throughput at
+    // all four workload shapes, so they run only when the tuning hook asks.
     const int pairs_max = qgemm_sm_count() / 2;
-    auto wave_eff = [&](int tiles) {
-        const int waves = (tiles + pairs_max - 1) / pairs_max;
-        return (double)tiles / (double)(waves * pairs_max);
-    };
-    const int t1 = ((a.M + TM - 1) / TM) * prm.num_n, t2 = ((a.M + 2 * TM - 1) / (2 * TM)) * prm.num_n;
-    prm.mb = (a.a_val && wave_eff(t2) >= wave_eff(t1) - 0.02) ? 2 : 1;
-    if (a.a_val && g_force_mb) prm.mb = g_force_mb;
+    prm.mb = (a.a_val && g_force_mb) ? g_force_mb : 1;
     prm.num_m = (a.M + prm.mb * TM - 1) / (prm.mb * TM);
     prm.num_tiles = prm.num_m * prm.num_n;
     // A's values are 2 (e4m3: 1) bytes per element, more than L2 holds at the

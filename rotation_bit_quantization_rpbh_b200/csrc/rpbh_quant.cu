@@ -143,7 +143,10 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
-template <typename InT, int H, int BITS, int MODE, int SPL>
+// CONTIG: the plan's permutation is the identity (Block-RHT, the rotation
+// ablation without P_pi), so a block's inputs are contiguous and are read
+// 16 bytes at a time instead of gathered one by one.
+template <typename InT, int H, int BITS, int MODE, int SPL, bool CONTIG>
 __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
     rpbh_quant_kernel(const __grid_constant__ RpbhParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -154,12 +157,14 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = warp / p.team, wt = warp - t * p.team;  // team, warp within the team
-    // SPL lanes per h-block: lane = ((r * Bw + j) * SPL + hf); with two, each
-    // lane holds half of the block's values (see the gather)
+    // SPL lanes per h-block: lane = ((j * RW + r) * SPL + hf) -- block-major,
+    // so the 8 lanes of one phase of a 16-byte load are 8 rows of a block,
+    // whose row pads put them on different banks; with SPL = 2 each lane
+    // holds half of the block's values (see the gather)
     constexpr int LSPL = SPL == 2 ? 1 : 0;
     const int hf = lane & (SPL - 1);
     const int Bw = 1 << p.lbw;
-    const int j = (lane >> LSPL) & (Bw - 1), r = lane >> (LSPL + p.lbw);  // block within the warp, row within the set
+    const int r = (lane >> LSPL) & (p.RW - 1), j = lane >> (LSPL + p.lrw);  // row within the set, block within the warp
     const int b = wt * Bw + j;                            // h-block of this lane
     const bool bact = b < p.nb;
     const bool loader = wt == 0 && lane == 0;             // issues the team's row copies
@@ -294,6 +299,41 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
         } else if (!valid) {
 #pragma unroll
             for (int i = 0; i < L2H; ++i) v2[i] = make_float2(0.f, 0.f);
+        } else if constexpr (CONTIG) {
+            // identity permutation: the block's h inputs are contiguous in the
+            // row; 16-byte loads, the signs of D from the table's bit 15
+            const uint32_t rowp = stage_addr + (uint32_t)(slot * p.RW * p.srow + r * p.srow) + (uint32_t)(b * H * ES);
+            const uint32_t tabp = gtab_addr + (uint32_t)b * 16u;
+            constexpr int PER16 = 16 / ES;  // elements per 16-byte load
+#pragma unroll
+            for (int c = 0; c < H / PER16; ++c) {
+                const uint4 dv = lds_v4(rowp + (uint32_t)c * 16u);
+                const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+                float f[PER16];
+#pragma unroll
+                for (int c4 = 0; c4 < PER16 / 4; ++c4) {
+                    const int chunk = (c * PER16) / 4 + c4;  // table chunk of entries 4 chunk .. 4 chunk + 3
+                    const uint4 ch = lds_v4(tabp + (uint32_t)(chunk * p.nb) * 16u);
+                    const uint32_t e[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t sg = (e[q] & 0x8000u) << 16;  // sign of D_k in bit 31
+                        if constexpr (ES == 2) {
+                            const uint32_t w = dw[(4 * c4 + q) >> 1];
+                            const uint32_t bits = ((4 * c4 + q) & 1) ? (w & 0xffff0000u) : (w << 16);
+                            f[4 * c4 + q] = __uint_as_float(bits ^ sg);
+                        } else {
+                            f[4 * c4 + q] = __uint_as_float(dw[q] ^ sg);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < PER16; q += 2) {
+                    const int i2 = (c * PER16 + q) >> 1;
+                    v2[i2] = make_float2(f[q], f[q + 1]);
+                    acc = f2fma(v2[i2], v2[i2], acc);
+                }
+            }
         } else {
             const uint32_t rowp = stage_addr + (uint32_t)(slot * p.RW * p.srow + r * p.srow);
             const uint32_t tabp = gtab_addr + (uint32_t)b * 16u;
@@ -339,7 +379,8 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
 
         // ---- A4 (first half): the row's sum of squares over this warp's blocks ----
         float ss = acc.x + acc.y;
-        for (int o = 1; o < (Bw << LSPL); o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (SPL == 2) ss += __shfl_xor_sync(0xffffffffu, ss, 1);  // the block's two halves
+        for (int o = p.RW << LSPL; o < 32; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);  // the row's blocks
         float* part = my_part + (k & 1) * p.team * p.RW;
         if (p.team > 1) {
             if (j == 0 && hf == 0) part[wt * p.RW + r] = ss;
@@ -567,9 +608,9 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
     if (tid == 0 && !p.starve) mbar_wait_bounded(tab_bar, 0u);
 }
 
-template <typename InT, int H, int BITS, int MODE, int SPL>
+template <typename InT, int H, int BITS, int MODE, int SPL, bool CONTIG>
 cudaError_t launch_rpbh_spl(const RpbhParams& p, int grid, cudaStream_t stream) {
-    auto k = rpbh_quant_kernel<InT, H, BITS, MODE, SPL>;
+    auto k = rpbh_quant_kernel<InT, H, BITS, MODE, SPL, CONTIG>;
     const int smem = smem_layout(p).total;
     static int smem_done[kSmemRecordDevices] = {0};  // this instantiation's limit, per device
     const cudaError_t e = ensure_smem_limit(k, smem, smem_done);
@@ -579,12 +620,14 @@ cudaError_t launch_rpbh_spl(const RpbhParams& p, int grid, cudaStream_t stream) 
     return cudaGetLastError();
 }
 
-// two lanes per block: bf16 inputs, blocks of 64 or 128
+// contiguous blocks (identity permutation): one lane per block; two lanes
+// per block: bf16 inputs, blocks of 64 or 128
 template <typename InT, int H, int BITS, int MODE>
 cudaError_t launch_rpbh_t(const RpbhParams& p, int grid, cudaStream_t stream) {
+    if (p.contig) return launch_rpbh_spl<InT, H, BITS, MODE, 1, true>(p, grid, stream);
     if constexpr (sizeof(InT) == 2 && H >= 64)
-        if (p.SPL == 2) return launch_rpbh_spl<InT, H, BITS, MODE, 2>(p, grid, stream);
-    return launch_rpbh_spl<InT, H, BITS, MODE, 1>(p, grid, stream);
+        if (p.SPL == 2) return launch_rpbh_spl<InT, H, BITS, MODE, 2, false>(p, grid, stream);
+    return launch_rpbh_spl<InT, H, BITS, MODE, 1, false>(p, grid, stream);
 }
 
 template <typename InT, int H, int MODE>
@@ -646,7 +689,7 @@ bool rpbh_choose_layout(RpbhParams& p, int h, int esize) {
     int best_key = -1;
     // two lanes per block (more warps per SM, half the registers) only for
     // bf16 inputs and blocks of 64 or 128, and only when forced for now
-    const int spl_max = (esize == 2 && h >= 64 && g_force_spl == 2) ? 2 : 1;
+    const int spl_max = (esize == 2 && h >= 64 && g_force_spl == 2 && !p.contig) ? 2 : 1;
     for (int spl = spl_max; spl >= 1; --spl) {
         const int max_warps = spl == 2 ? kMaxWarpsSplit : kMaxWarps;
         for (int slots = 2; slots >= 1; --slots) {
@@ -660,9 +703,11 @@ bool rpbh_choose_layout(RpbhParams& p, int h, int esize) {
                 RpbhParams c = p;
                 c.SPL = spl;
                 c.RW = RW;
-                int lbw = 0;
+                int lbw = 0, lrw = 0;
                 while ((1 << lbw) < Bw) ++lbw;
+                while ((1 << lrw) < RW) ++lrw;
                 c.lbw = lbw;
+                c.lrw = lrw;
                 c.team = team;
                 c.slots = slots;
                 c.srow = c.row_bytes + (RW == 1 ? 16 : 128 / RW);

@@ -15,8 +15,9 @@ struct RpbhParams {
     // r * (32 / RW) + block j); a team of `team` warps covers all nb blocks
     // of a set of RW rows; a CTA holds `tpc` teams, each with `slots`
     // staging slots of RW rows.
-    int RW, lbw;          // rows per warp; log2 of the blocks per warp
+    int RW, lbw, lrw;     // rows per warp; log2 of the blocks per warp and of RW
     int SPL;              // lanes per h-block: 1, or 2 (each holds half the block's values)
+    int contig;           // identity permutation: blocks read contiguously (one lane per block)
     int team, tpc, slots;
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
     int nrs;              // row sets: ceil(M / RW)

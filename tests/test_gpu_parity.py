@@ -139,24 +139,31 @@ def test_workload_at_full_size(cuda_device, name):
     print(name, stats)
 
 
-@pytest.mark.parametrize("M,d,h,ba", [(300, 512, 128, 4), (96, 1536, 128, 6)])
-def test_block_rht_variant_matches_oracle(cuda_device, M, d, h, ba):
-    """The rotation ablation's Block-RHT plan (no permutation) through the
-    same kernels: rotation, norms and codes against the oracle's variant."""
+@pytest.mark.parametrize("M,d,h,ba,dt", [(300, 512, 128, 4, "bf16"), (96, 1536, 128, 6, "bf16"),
+                                         (130, 256, 64, 2, "f32"), (77, 3072, 128, 4, "bf16")])
+def test_block_rht_variant_matches_oracle(cuda_device, M, d, h, ba, dt):
+    """The rotation ablation's Block-RHT plan (no permutation; each block is
+    read contiguously): rotation, norms and codes against the oracle's
+    variant, and the value outputs equal to the codebook at the codes."""
     plan = B.rotation_plan(d, h, 21, B.OQ_ROT_BLOCK_RHT)
     perm, sign = oracle.plan(d, h, 21, variant=oracle.BLOCK_RHT)
     pe, se = plan.export()
     np.testing.assert_array_equal(pe, perm)
     np.testing.assert_array_equal(se, sign)
     g = torch.Generator().manual_seed(21)
-    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g)))
+    x = x.to(torch.bfloat16 if dt == "bf16" else torch.float32)
     cb_a, ocb_a = B.codebook(d, ba), oracle.codebook(d, ba)
     a_idx, s = B.quantize_acts(plan, cb_a, x.to(cuda_device))
+    val, s_v = B.quantize_acts_values(plan, cb_a, x.to(cuda_device))
     torch.cuda.synchronize()
     assert B.device_status() == 0
     rows = np.arange(M)
     check_rotation(plan, x, rows, h, perm, sign, cuda_device)
     check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb_a, ocb_a, "acts")
+    u = B.unpack_indices(a_idx, d, ba).long()
+    tab = torch.from_numpy(cb_a.bf16_bits().view(np.int16)).to(cuda_device)
+    assert torch.equal(val.view(torch.int16), tab[u]) and torch.equal(s_v, s)
 
 
 @pytest.mark.parametrize("M,d,h,variant,ba,dt", [
