@@ -710,6 +710,22 @@ def run_ablation(args):
         calls[f"{name}_quant"] = (lambda pl=pl: B.quantize_acts(pl, cb_a, x, a_idx, s, stream=stream))
         calls[f"{name}_rotate"] = (lambda pl=pl: B.rpbh_apply(pl, x, x_rot, s, stream=stream))
     calls["haar_rotate_cublas"] = lambda: torch.matmul(xb, haar_t, out=y_haar)
+
+    # the same two plans through one kernel family each: the team kernel
+    # (the Block-RHT plan's contiguous reads against the RPBH gather) and
+    # the warp-group kernel (both plans gathered through their tables)
+    def forced(family, fn):
+        def call():
+            B.debug_rpbh_kernel(family)
+            try:
+                fn()
+            finally:
+                B.debug_rpbh_kernel(0)
+        return call
+
+    calls["rpbh_quant_teams"] = forced(B.RPBH_KERNEL_TEAMS, calls["rpbh_quant"])
+    calls["rpbh_quant_groups"] = forced(B.RPBH_KERNEL_GROUPS, calls["rpbh_quant"])
+    calls["block_rht_quant_groups"] = forced(B.RPBH_KERNEL_GROUPS, calls["block_rht_quant"])
     ms = {}
     for name, fn in calls.items():
         for _ in range(max(3, args.warmup)):
@@ -731,6 +747,8 @@ def run_ablation(args):
         "ms": ms,
         "ratios": {
             "rpbh_over_block_rht_quant": ms["rpbh_quant"] / ms["block_rht_quant"],
+            "rpbh_over_block_rht_quant_team_kernel": ms["rpbh_quant_teams"] / ms["block_rht_quant"],
+            "rpbh_over_block_rht_quant_group_kernel": ms["rpbh_quant_groups"] / ms["block_rht_quant_groups"],
             "rpbh_over_block_rht_rotate": ms["rpbh_rotate"] / ms["block_rht_rotate"],
             "full_rht_over_rpbh_rotate": ms["full_rht_rotate"] / ms["rpbh_rotate"],
             "haar_over_rpbh_rotate": ms["haar_rotate_cublas"] / ms["rpbh_rotate"],
@@ -742,7 +760,9 @@ def run_ablation(args):
             "haar_plus_quant_over_rpbh_quant": (ms["haar_rotate_cublas"] + ms["block_rht_quant"]) / ms["rpbh_quant"],
         },
         "note": "rotate = oq_rpbh_apply (fp32 x' and norms out); quant = the fused rotate+split+quantise kernel "
-                "(packed codes out); Block-RHT and Full RHT read each block contiguously (no permutation); "
+                "(packed codes out), each plan on its default kernel; _teams / _groups = forced onto the team or "
+                "the warp-group kernel; Block-RHT and Full RHT read each block contiguously (no permutation) "
+                "except on the warp-group kernel, which gathers through the identity table; "
                 "haar = bf16 x @ Q^T with a Haar-random Q, bf16 out (cuBLAS); L2 flushed before every call",
     }
     print(json.dumps(out), flush=True)

@@ -322,8 +322,8 @@ oq_status oq_device_status(int clear, int* out, void* stream);
 /*   returns without faulting; the context stays usable.  The output of     */
 /*   that launch is undefined.  The call itself still returns OQ_OK.        */
 /*   Each call replaces the pending set; mask 0 cancels.                    */
-/* oq_debug_rpbh_layout(rows_per_warp, slots, lanes_per_block): the       */
-/*   rotate-and-quantise kernel's work layout -- rows of x per warp (1, 2, */
+/* oq_debug_rpbh_layout(rows_per_warp, slots, lanes_per_block): the team  */
+/*   kernel's work layout -- rows of x per warp (1, 2, */
 /*   4 or 8), staging slots per warp team (1 or 2) and lanes per h-block   */
 /*   (2: each lane holds half of a block; bf16 inputs, h of 64 or 128) --  */
 /*   is forced for the following launches where it fits in shared memory   */
@@ -332,15 +332,23 @@ oq_status oq_device_status(int clear, int* out, void* stream);
 /*   and of the butterflies.  For tests and tuning.                         */
 /* oq_debug_qgemm_tile_rows(rows): the product with A given as values     */
 /*   (oq_qgemm_values, the values schedule) uses tiles of `rows` = 256 or  */
-/*   512 rows of A for the following launches (0 or another value: chosen */
-/*   by the library per shape, the default).  The result does not depend   */
-/*   on it.  For tests and tuning.                                          */
+/*   512 rows of A for the following launches (0 or another value: 256,   */
+/*   the default).  The result does not depend on it.  For tests and       */
+/*   tuning.                                                                */
+/* oq_debug_rpbh_kernel(which): the rotate-and-quantise kernel family for  */
+/*   plans with h <= 128 in the following launches: 1 the warp-group       */
+/*   kernel, 2 the team kernel (whose work layout oq_debug_rpbh_layout     */
+/*   forces), 0 or another value: chosen by the library (the warp-group    */
+/*   kernel for permuted plans with d <= 8192, else the team kernel).      */
+/*   Results do not depend on it except for the rounding order of the row   */
+/*   norm's sum.  For tests and tuning.                                     */
 #define OQ_STARVE_RPBH 1 /* the rotate-and-quantise kernel (acts and weights) */
 #define OQ_STARVE_GEMM 2 /* the codebook-decode GEMM (bf16 and fp8)           */
 void oq_debug_fail_allocations(int n);
 void oq_debug_starve(int mask);
 void oq_debug_rpbh_layout(int rows_per_warp, int slots, int lanes_per_block);
 void oq_debug_qgemm_tile_rows(int rows);
+void oq_debug_rpbh_kernel(int which);
 
 #ifdef __cplusplus
 }

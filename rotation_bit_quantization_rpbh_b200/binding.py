@@ -34,7 +34,8 @@ EXPORTS = ["oq_status_str", "oq_codebook", "oq_codebook_values", "oq_codebook_bf
            "oq_qlinear_workspace", "oq_qlinear", "oq_qlinear_noalloc", "oq_device_status",
            "oq_debug_fail_allocations", "oq_debug_starve", "oq_quantize_acts_values",
            "oq_quantize_acts_values_fp8", "oq_qgemm_values", "oq_qgemm_values_fp8", "oq_qlinear_workspace_values",
-           "oq_debug_rpbh_layout", "oq_codebook_upload", "oq_debug_qgemm_tile_rows"]
+           "oq_debug_rpbh_layout", "oq_codebook_upload", "oq_debug_qgemm_tile_rows",
+           "oq_debug_rpbh_kernel"]
 
 
 class OQError(RuntimeError):
@@ -88,6 +89,7 @@ def lib():
                     "oq_debug_starve": ([I], None),
                     "oq_debug_rpbh_layout": ([I, I, I], None),
                     "oq_debug_qgemm_tile_rows": ([I], None),
+                    "oq_debug_rpbh_kernel": ([I], None),
                     "oq_quantize_acts_values": ([P, P, P, I, I, P, P, P], I),
                     "oq_quantize_acts_values_fp8": ([P, P, P, I, I, P, P, P], I),
                     "oq_qgemm_values": ([P, I, I, P, P, P, P, P, P, P], I),
@@ -472,7 +474,7 @@ def debug_starve(mask):
 
 
 def debug_rpbh_layout(rows_per_warp=0, slots=0, lanes_per_block=0):
-    """Test and tuning hook: force the rotate-and-quantise kernel's rows per
+    """Test and tuning hook: force the team kernel's rows per
     warp (1, 2, 4, 8), staging slots per warp team (1, 2) and lanes per
     h-block (2: two lanes share a block; bf16 inputs, h of 64 or 128) where
     they fit; 0 restores the library's choice."""
@@ -481,8 +483,17 @@ def debug_rpbh_layout(rows_per_warp=0, slots=0, lanes_per_block=0):
 
 def debug_qgemm_tile_rows(rows=0):
     """Test and tuning hook: tiles of 256 or 512 rows of A in the A-values
-    product (0: the library's choice per shape)."""
+    product (0: the default, 256)."""
     lib().oq_debug_qgemm_tile_rows(int(rows))
+
+
+RPBH_KERNEL_AUTO, RPBH_KERNEL_GROUPS, RPBH_KERNEL_TEAMS = 0, 1, 2
+
+
+def debug_rpbh_kernel(which=RPBH_KERNEL_AUTO):
+    """Test and tuning hook: the rotate-and-quantise kernel family for
+    h <= 128 (1: warp groups, 2: teams; 0: the library's choice per shape)."""
+    lib().oq_debug_rpbh_kernel(int(which))
 
 
 def unpack_indices(packed, d, bits):

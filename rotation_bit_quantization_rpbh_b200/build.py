@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "liboq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 SOURCES = ["liboq.cu", "host.cpp"]
-DEPS = ["liboq.cu", "host.cpp", "api.cu", "rpbh_quant.cu", "rht_big.cu", "qgemm.cu", "device_util.cuh", "oq_internal.h",
+DEPS = ["liboq.cu", "host.cpp", "api.cu", "rpbh_quant.cu", "rpbh_groups.cu", "rht_big.cu", "qgemm.cu", "device_util.cuh", "oq_internal.h",
         "rpbh_quant.cuh", "qgemm.cuh"]
 
 

@@ -53,6 +53,10 @@ int packed_row_bytes(int d, int bits) { return bits == 6 ? d : d * bits / 8; }  
 // Launch the fused rotate/quantise kernel in one of its modes: 0 activation
 // codes, 1 weight codes, 2 rotation only, 3 / 4 activation values (bf16 /
 // e4m3 of c sqrt(d)) written to idx_out.
+// Tuning hook: 0 chooses the kernel family per shape, 1 forces the
+// warp-group kernel, 2 the team kernel (blocks of at most 128).
+std::atomic<int> g_force_kernel{0};
+
 oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_dtype dtype, int M, int mode,
                    uint8_t* idx_out, float* s_out, uint16_t* r_out, float* y_out, float* norm_out, cudaStream_t st) {
     if (!plan || M < 0) return OQ_ERR_INVALID_ARG;
@@ -95,14 +99,25 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
     p.nb = nb;
     p.lut_n = mode != 2 ? (int)cb->lut.size() : 0;
     p.contig = plan->variant == OQ_ROT_BLOCK_RHT ? 1 : 0;
+    // Kernel family for blocks of at most 128: the warp-group kernel for
+    // permuted plans up to d = 8192 (measured faster there), the team kernel
+    // above that and for Block-RHT plans (its contiguous read path); the
+    // tuning hook may force either.
+    bool groups = false;
     if (big) {
         p.row_bytes = d * esize;
         if (rht_big_smem_bytes(p) > kSmemLimit) return OQ_ERR_UNSUPPORTED;
     } else {
-        if (!rpbh_choose_layout(p, h, esize)) return OQ_ERR_UNSUPPORTED;
-        p.nrs = (M + p.RW - 1) / p.RW;
+        const int force = g_force_kernel.load();
+        groups = force == 1 || (force == 0 && !p.contig && d <= 8192);
+        if (groups && !rpbh_choose_groups(p, esize)) groups = false;
+        if (!groups) {
+            if (!rpbh_choose_layout(p, h, esize)) return OQ_ERR_UNSUPPORTED;
+            p.nrs = (M + p.RW - 1) / p.RW;
+        }
     }
     p.gtab = plan->dev.gtab;
+    p.gtab16 = plan->dev.gtab16;
     if (mode != 2) {
         p.lut = mode == 3 ? dcb->lut_vb : (mode == 4 ? dcb->lut_v8 : dcb->lut);
         p.lut_off = -(int)kLutMagicBits - cb->kmin;
@@ -127,6 +142,9 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
         per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
         const int cap = per_sm * device_sms();
         e = launch_rht_big(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, M < cap ? M : cap, st);
+    } else if (groups) {
+        const int grid = p.ntiles < device_sms() ? p.ntiles : device_sms();
+        e = launch_rpbh_groups(p, dtype == OQ_BF16, h, mode == 2 ? 4 : cb->bits, mode, grid, st);
     } else {
         const int per_cta = (p.nrs + p.tpc - 1) / p.tpc;
         const int grid = per_cta < device_sms() ? per_cta : device_sms();
@@ -288,17 +306,23 @@ oq_status oq_rotation_plan(int d, int h, uint64_t seed, int variant, oq_plan_t**
     p->sign.resize(d);
     make_plan(d, h, seed, p->perm.data(), p->sign.data(), variant);
     build_gather_table(p, p->gtab_host);
+    build_gather_table16(p, p->gtab16_host);
+    // one allocation: the 32-bit table, then the 16-bit one (16-byte aligned: 4 d bytes in)
     void* ptr = nullptr;
-    if (!device_alloc(&ptr, sizeof(uint32_t) * d)) {
+    const size_t b32 = sizeof(uint32_t) * d, b16 = sizeof(uint16_t) * d;
+    if (!device_alloc(&ptr, b32 + b16)) {
         delete p;
         return OQ_ERR_OOM;
     }
-    if (cudaMemcpy(ptr, p->gtab_host.data(), sizeof(uint32_t) * d, cudaMemcpyHostToDevice) != cudaSuccess) {
+    uint8_t* base = static_cast<uint8_t*>(ptr);
+    if (cudaMemcpy(base, p->gtab_host.data(), b32, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base + b32, p->gtab16_host.data(), b16, cudaMemcpyHostToDevice) != cudaSuccess) {
         cudaFree(ptr);
         delete p;
         return OQ_ERR_CUDA;
     }
-    p->dev.gtab = static_cast<uint32_t*>(ptr);
+    p->dev.gtab = reinterpret_cast<uint32_t*>(base);
+    p->dev.gtab16 = reinterpret_cast<uint16_t*>(base + b32);
     *out = p;
     return OQ_OK;
 }
@@ -615,6 +639,8 @@ void oq_debug_fail_allocations(int n) { g_fail_allocs.store(n > 0 ? n : 0); }
 void oq_debug_starve(int mask) { g_starve_mask.store(mask & (OQ_STARVE_RPBH | OQ_STARVE_GEMM)); }
 
 void oq_debug_qgemm_tile_rows(int rows) { qgemm_force_tile_rows(rows); }
+
+void oq_debug_rpbh_kernel(int which) { g_force_kernel.store(which == 1 || which == 2 ? which : 0); }
 
 void oq_debug_rpbh_layout(int rows_per_warp, int slots, int lanes_per_block) {
     const bool rw_ok = rows_per_warp == 0 || rows_per_warp == 1 || rows_per_warp == 2 || rows_per_warp == 4 ||

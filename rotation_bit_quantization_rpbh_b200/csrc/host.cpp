@@ -339,4 +339,19 @@ void build_gather_table(const oq_plan_t* p, std::vector<uint32_t>& out) {
             }
 }
 
+// The warp-group kernel's gather table: the entry of coordinate k = b*h + i
+// is pi(k) | 0x8000 * (sigma_k < 0) (the element index, 15 bits since
+// d <= 32767, and the sign of D_k), in 16-byte chunks of 8 entries, chunk
+// (c, b) (entries b*h + 8c .. b*h + 8c + 7) at chunk index c*nb + b.
+void build_gather_table16(const oq_plan_t* p, std::vector<uint16_t>& out) {
+    const int d = p->d, h = p->h, nb = d / h, nc = h / 8;
+    out.assign(d, 0);
+    for (int b = 0; b < nb; ++b)
+        for (int c = 0; c < nc; ++c)
+            for (int e = 0; e < 8; ++e) {
+                const int k = b * h + c * 8 + e;
+                out[(size_t)(c * nb + b) * 8 + e] = (uint16_t)(p->perm[k] | (p->sign[k] < 0 ? 0x8000 : 0));
+            }
+}
+
 }  // namespace oq

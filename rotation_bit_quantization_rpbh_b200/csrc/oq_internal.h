@@ -29,7 +29,8 @@ struct DeviceCodebook {
 };
 
 struct DevicePlan {
-    uint32_t* gtab = nullptr;  // device gather table (see build_gather_table)
+    uint32_t* gtab = nullptr;    // device gather table (see build_gather_table)
+    uint16_t* gtab16 = nullptr;  // the 16-bit one (see build_gather_table16), same allocation
 };
 
 }  // namespace oq
@@ -59,7 +60,8 @@ struct oq_plan_s {
     int variant = 0;  // OQ_ROT_RPBH or OQ_ROT_BLOCK_RHT (identity permutation)
     std::vector<int32_t> perm;
     std::vector<int8_t> sign;
-    std::vector<uint32_t> gtab_host;  // chunked gather table (see build_gather_table)
+    std::vector<uint32_t> gtab_host;    // chunked gather table (see build_gather_table)
+    std::vector<uint16_t> gtab16_host;  // 16-bit entries (see build_gather_table16)
     oq::DevicePlan dev;
 };
 
@@ -70,6 +72,7 @@ oq_status build_codebook(int d, int bits, oq_codebook_t* cb);
 void make_plan(int d, int h, uint64_t seed, int32_t* perm, int8_t* sign, int variant);
 uint8_t e4m3_round(double v);
 void build_gather_table(const oq_plan_t* p, std::vector<uint32_t>& out);
+void build_gather_table16(const oq_plan_t* p, std::vector<uint16_t>& out);
 uint16_t bf16_round(double x);
 
 // device-side pieces (api.cu)

@@ -143,6 +143,184 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
+// A5 for one lane's HL values of row `row`: v2 holds the unnormalised
+// butterfly outputs of columns unit*HL .. unit*HL + HL-1 and s the row norm.
+// Writes the norm (the lane of unit 0), then the rotation (test mode), the
+// centroid values or the packed codes of those columns.
+template <int HL, int BITS, int MODE>
+__device__ __forceinline__ void store_unit(const RpbhParams& p, float2 (&v2)[HL / 2], float s, int row, int unit,
+                                           uint32_t lut_addr0) {
+    constexpr int L2H = HL / 2;
+    const float2 G2 = make_float2(p.G_lut, p.G_lut);
+    const float2 M2 = make_float2(kLutMagic, kLutMagic);
+    if (unit == 0) {
+        if constexpr (MODE == 0 || MODE >= 3) p.s_out[row] = s;
+        if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+        if constexpr (MODE == 2) p.norm_out[row] = s;
+    }
+    if constexpr (MODE == 2) {
+        float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + (size_t)unit * HL);
+        const float2 sc = make_float2(p.rsqrt_h, p.rsqrt_h);
+#pragma unroll
+        for (int i = 0; i < L2H; i += 2) {
+            const float2 a = f2mul(v2[i], sc), c = f2mul(v2[i + 1], sc);
+            yo[i >> 1] = make_float4(a.x, a.y, c.x, c.y);
+        }
+    } else if constexpr (MODE >= 3) {
+        // ---- A5 with the centroid values written instead of the codes:
+        // the table entry holds the values of both cells its bin can
+        // give (the cell below the bin's threshold and the one above),
+        // so one compare selects c_index directly ----------------------
+        constexpr int VB = MODE == 3 ? 2 : 1;  // bytes per value: bf16, or e4m3
+        uint4* dst = reinterpret_cast<uint4*>(p.idx_out + (size_t)row * p.out_row_bytes + (size_t)unit * HL * VB);
+        if (s <= p.s_max) {
+            const float inv = p.rsqrt_h / (s + p.eps);
+            const float2 inv2 = make_float2(inv, inv);
+            // table word of element pair i and the selector bits of its two values
+            auto pick = [&](int i, uint32_t& val0, uint32_t& val1, uint32_t& ge0, uint32_t& ge1) {
+                const float2 q = f2mul(v2[i], inv2);
+                const float2 z = f2fma(q, G2, M2);
+                float T0, T1;
+                lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, val0);
+                lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, val1);
+                ge0 = q.x >= T0 ? 1u : 0u;
+                ge1 = q.y >= T1 ? 1u : 0u;
+            };
+#pragma unroll
+            for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) {
+                uint32_t words[4];
+#pragma unroll
+                for (int wj = 0; wj < 4; ++wj) {
+                    if constexpr (VB == 2) {
+                        // bf16 pair: (lo or hi half of entry 0, lo or hi half of entry 1)
+                        uint32_t val0, val1, ge0, ge1;
+                        pick(w0 + wj, val0, val1, ge0, ge1);
+                        words[wj] = prmt_b32(val0, val1, 0x5410u + ge0 * 0x22u + ge1 * 0x2200u);
+                    } else {
+                        // four e4m3 bytes: byte 0 or 1 of each entry's value word
+                        uint32_t val0, val1, val2, val3, ge0, ge1, ge2, ge3;
+                        pick(2 * (w0 + wj), val0, val1, ge0, ge1);
+                        pick(2 * (w0 + wj) + 1, val2, val3, ge2, ge3);
+                        const uint32_t lo = prmt_b32(val0, val1, 0x40u + ge0 + ge1 * 0x10u);
+                        const uint32_t hi = prmt_b32(val2, val3, 0x40u + ge2 + ge3 * 0x10u);
+                        words[wj] = prmt_b32(lo, hi, 0x5410u);
+                    }
+                }
+                dst[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
+            }
+        } else {
+            // the middle cell's value everywhere (see the codes branch)
+            const uint32_t wm = VB == 2 ? p.mid_val * 0x10001u : p.mid_val * 0x01010101u;
+#pragma unroll
+            for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) dst[w0 >> 2] = make_uint4(wm, wm, wm, wm);
+        }
+    } else {
+        // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
+        constexpr int NB = BITS == 6 ? HL : HL * BITS / 8;  // packed bytes of the lane's codes
+        constexpr int NW = NB / 4;
+        constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
+        constexpr int PER = BITS == 6 ? 4 : (BITS == 3 ? 8 : 32 / BITS);  // codes per word (3-bit: per 24-bit group)
+        constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
+        uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)unit * NB;
+        auto put = [&](int w0, const uint32_t (&words)[CW]) {
+            if constexpr (CW == 4)
+                reinterpret_cast<uint4*>(dst)[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
+            else if constexpr (CW == 2)
+                reinterpret_cast<uint2*>(dst)[w0 >> 1] = make_uint2(words[0], words[1]);
+            else
+                reinterpret_cast<uint32_t*>(dst)[w0] = words[0];
+        };
+        // code of element pair i: (index of .x, index of .y)
+        auto code2 = [&](int i, float2 inv2, uint32_t& i0, uint32_t& i1) {
+            const float2 q = f2mul(v2[i], inv2);
+            const float2 z = f2fma(q, G2, M2);
+            float T0, T1;
+            uint32_t b0, b1;
+            lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, b0);
+            lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, b1);
+            i0 = b0 + (q.x >= T0 ? 1u : 0u);
+            i1 = b1 + (q.y >= T1 ? 1u : 0u);
+        };
+        // s <= s_max keeps every butterfly value below sqrt(h) s (finite),
+        // so |v| <= 1 up to rounding and the table index stays in range;
+        // larger, infinite and NaN norms take the middle cell
+        if (BITS == 3 && s <= p.s_max) {
+            // 3-bit: codes 8g..8g+7 form a 24-bit group (LSB first); four
+            // groups fill three words
+            const float inv = p.rsqrt_h / (s + p.eps);
+            const float2 inv2 = make_float2(inv, inv);
+            uint32_t words[NW];
+#pragma unroll
+            for (int g4 = 0; g4 < HL / 32; ++g4) {
+                uint32_t grp[4];
+#pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    uint32_t acc_w = 0;
+#pragma unroll
+                    for (int kk = 6; kk >= 0; kk -= 2) {
+                        uint32_t i0, i1;
+                        code2((32 * g4 + 8 * gi + kk) >> 1, inv2, i0, i1);
+                        acc_w = (acc_w * 8u + i1) * 8u + i0;
+                    }
+                    grp[gi] = acc_w;
+                }
+                words[3 * g4] = grp[0] | (grp[1] << 24);
+                words[3 * g4 + 1] = (grp[1] >> 8) | (grp[2] << 16);
+                words[3 * g4 + 2] = (grp[2] >> 16) | (grp[3] << 8);
+            }
+#pragma unroll
+            for (int w0 = 0; w0 < NW; w0 += CW) {
+                uint32_t ws[CW];
+#pragma unroll
+                for (int wj = 0; wj < CW; ++wj) ws[wj] = words[w0 + wj];
+                put(w0, ws);
+            }
+        } else if (BITS != 3 && s <= p.s_max) {
+            // x'/(s+eps) = (H u / sqrt(h)) / (s + eps): one multiplier for the unnormalised butterflies
+            const float inv = p.rsqrt_h / (s + p.eps);
+            const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+            for (int w0 = 0; w0 < NW; w0 += CW) {
+                uint32_t words[CW];
+#pragma unroll
+                for (int wj = 0; wj < CW; ++wj) {
+                    const int wi = w0 + wj;
+                    // codes of this word, highest position first: acc = acc * 2^bits + code
+                    uint32_t acc_w = 0;
+#pragma unroll
+                    for (int kk = PER - 2; kk >= 0; kk -= 2) {
+                        uint32_t i0, i1;
+                        code2((wi * PER + kk) >> 1, inv2, i0, i1);
+                        acc_w = (acc_w * SH + i1) * SH + i0;
+                    }
+                    words[wj] = acc_w;
+                }
+                put(w0, words);
+            }
+        } else if (BITS == 3) {
+            // middle code 4 everywhere: the 3-bit stream repeats every 3 words
+            constexpr uint32_t gm = 04444'4444u;  // eight 3-bit fours (octal)
+            const uint32_t pat[3] = {gm | (gm << 24), (gm >> 8) | (gm << 16), (gm >> 16) | (gm << 8)};
+#pragma unroll
+            for (int w0 = 0; w0 < NW; w0 += CW) {
+                uint32_t ws[CW];
+#pragma unroll
+                for (int wj = 0; wj < CW; ++wj) ws[wj] = pat[(w0 + wj) % 3];
+                put(w0, ws);
+            }
+        } else {
+            uint32_t wmid = 0;
+#pragma unroll
+            for (int kk = 0; kk < PER; ++kk) wmid = wmid * SH + (uint32_t)(p.L >> 1);
+            uint32_t words[CW];
+#pragma unroll
+            for (int wj = 0; wj < CW; ++wj) words[wj] = wmid;
+#pragma unroll
+            for (int w0 = 0; w0 < NW; w0 += CW) put(w0, words);
+        }
+    }
+}
+
 // CONTIG: the plan's permutation is the identity (Block-RHT, the rotation
 // ablation without P_pi), so a block's inputs are contiguous and are read
 // 16 bytes at a time instead of gathered one by one.
@@ -222,8 +400,6 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
         for (int i = 0; i < p.slots; ++i)
             if (g0 + i * stride < p.nrs) issue(i, g0 + i * stride, i);
 
-    const float2 G2 = make_float2(p.G_lut, p.G_lut);
-    const float2 M2 = make_float2(kLutMagic, kLutMagic);
     // shared address of lut[(bits of the magic-biased value) + lut_off]
     const uint32_t lut_addr0 = smem_u32(smem) + (uint32_t)L.lut + (uint32_t)p.lut_off * 8u;
     const uint32_t gtab_addr = smem_u32(smem) + (uint32_t)L.gtab;  // table chunks, 16 bytes each
@@ -425,175 +601,7 @@ __global__ void __launch_bounds__(SPL == 2 ? kMaxThreadsSplit : kMaxThreads, 1)
         }
         const float s = __fsqrt_rn(ssum);
 
-        if (valid) {
-            if (b == 0 && hf == 0) {
-                if constexpr (MODE == 0 || MODE >= 3) p.s_out[row] = s;
-                if constexpr (MODE == 1) p.r_out[row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-                if constexpr (MODE == 2) p.norm_out[row] = s;
-            }
-            if constexpr (MODE == 2) {
-                float4* yo = reinterpret_cast<float4*>(p.y_out + (size_t)row * p.d + b * H + hf * HL);
-                const float2 sc = make_float2(p.rsqrt_h, p.rsqrt_h);
-#pragma unroll
-                for (int i = 0; i < L2H; i += 2) {
-                    const float2 a = f2mul(v2[i], sc), c = f2mul(v2[i + 1], sc);
-                    yo[i >> 1] = make_float4(a.x, a.y, c.x, c.y);
-                }
-            } else if constexpr (MODE >= 3) {
-                // ---- A5 with the centroid values written instead of the codes:
-                // the table entry holds the values of both cells its bin can
-                // give (the cell below the bin's threshold and the one above),
-                // so one compare selects c_index directly ----------------------
-                constexpr int VB = MODE == 3 ? 2 : 1;  // bytes per value: bf16, or e4m3
-                uint4* dst = reinterpret_cast<uint4*>(p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * H * VB +
-                                                      (size_t)hf * HL * VB);
-                if (s <= p.s_max) {
-                    const float inv = p.rsqrt_h / (s + p.eps);
-                    const float2 inv2 = make_float2(inv, inv);
-                    // table word of element pair i and the selector bits of its two values
-                    auto pick = [&](int i, uint32_t& val0, uint32_t& val1, uint32_t& ge0, uint32_t& ge1) {
-                        const float2 q = f2mul(v2[i], inv2);
-                        const float2 z = f2fma(q, G2, M2);
-                        float T0, T1;
-                        lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, val0);
-                        lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, val1);
-                        ge0 = q.x >= T0 ? 1u : 0u;
-                        ge1 = q.y >= T1 ? 1u : 0u;
-                    };
-#pragma unroll
-                    for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) {
-                        uint32_t words[4];
-#pragma unroll
-                        for (int wj = 0; wj < 4; ++wj) {
-                            if constexpr (VB == 2) {
-                                // bf16 pair: (lo or hi half of entry 0, lo or hi half of entry 1)
-                                uint32_t val0, val1, ge0, ge1;
-                                pick(w0 + wj, val0, val1, ge0, ge1);
-                                words[wj] = prmt_b32(val0, val1, 0x5410u + ge0 * 0x22u + ge1 * 0x2200u);
-                            } else {
-                                // four e4m3 bytes: byte 0 or 1 of each entry's value word
-                                uint32_t val0, val1, val2, val3, ge0, ge1, ge2, ge3;
-                                pick(2 * (w0 + wj), val0, val1, ge0, ge1);
-                                pick(2 * (w0 + wj) + 1, val2, val3, ge2, ge3);
-                                const uint32_t lo = prmt_b32(val0, val1, 0x40u + ge0 + ge1 * 0x10u);
-                                const uint32_t hi = prmt_b32(val2, val3, 0x40u + ge2 + ge3 * 0x10u);
-                                words[wj] = prmt_b32(lo, hi, 0x5410u);
-                            }
-                        }
-                        dst[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
-                    }
-                } else {
-                    // the middle cell's value everywhere (see the codes branch)
-                    const uint32_t wm = VB == 2 ? p.mid_val * 0x10001u : p.mid_val * 0x01010101u;
-#pragma unroll
-                    for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) dst[w0 >> 2] = make_uint4(wm, wm, wm, wm);
-                }
-            } else {
-                // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
-                constexpr int NB = BITS == 6 ? HL : HL * BITS / 8;  // packed bytes of the lane's codes
-                constexpr int NW = NB / 4;
-                constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
-                constexpr int PER = BITS == 6 ? 4 : (BITS == 3 ? 8 : 32 / BITS);  // codes per word (3-bit: per 24-bit group)
-                constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
-                uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)b * NB * SPL + (size_t)hf * NB;
-                auto put = [&](int w0, const uint32_t (&words)[CW]) {
-                    if constexpr (CW == 4)
-                        reinterpret_cast<uint4*>(dst)[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
-                    else if constexpr (CW == 2)
-                        reinterpret_cast<uint2*>(dst)[w0 >> 1] = make_uint2(words[0], words[1]);
-                    else
-                        reinterpret_cast<uint32_t*>(dst)[w0] = words[0];
-                };
-                // code of element pair i: (index of .x, index of .y)
-                auto code2 = [&](int i, float2 inv2, uint32_t& i0, uint32_t& i1) {
-                    const float2 q = f2mul(v2[i], inv2);
-                    const float2 z = f2fma(q, G2, M2);
-                    float T0, T1;
-                    uint32_t b0, b1;
-                    lut_ld(__float_as_uint(z.x) * 8u + lut_addr0, T0, b0);
-                    lut_ld(__float_as_uint(z.y) * 8u + lut_addr0, T1, b1);
-                    i0 = b0 + (q.x >= T0 ? 1u : 0u);
-                    i1 = b1 + (q.y >= T1 ? 1u : 0u);
-                };
-                // s <= s_max keeps every butterfly value below sqrt(h) s (finite),
-                // so |v| <= 1 up to rounding and the table index stays in range;
-                // larger, infinite and NaN norms take the middle cell
-                if (BITS == 3 && s <= p.s_max) {
-                    // 3-bit: codes 8g..8g+7 form a 24-bit group (LSB first); four
-                    // groups fill three words
-                    const float inv = p.rsqrt_h / (s + p.eps);
-                    const float2 inv2 = make_float2(inv, inv);
-                    uint32_t words[NW];
-#pragma unroll
-                    for (int g4 = 0; g4 < HL / 32; ++g4) {
-                        uint32_t grp[4];
-#pragma unroll
-                        for (int gi = 0; gi < 4; ++gi) {
-                            uint32_t acc_w = 0;
-#pragma unroll
-                            for (int kk = 6; kk >= 0; kk -= 2) {
-                                uint32_t i0, i1;
-                                code2((32 * g4 + 8 * gi + kk) >> 1, inv2, i0, i1);
-                                acc_w = (acc_w * 8u + i1) * 8u + i0;
-                            }
-                            grp[gi] = acc_w;
-                        }
-                        words[3 * g4] = grp[0] | (grp[1] << 24);
-                        words[3 * g4 + 1] = (grp[1] >> 8) | (grp[2] << 16);
-                        words[3 * g4 + 2] = (grp[2] >> 16) | (grp[3] << 8);
-                    }
-#pragma unroll
-                    for (int w0 = 0; w0 < NW; w0 += CW) {
-                        uint32_t ws[CW];
-#pragma unroll
-                        for (int wj = 0; wj < CW; ++wj) ws[wj] = words[w0 + wj];
-                        put(w0, ws);
-                    }
-                } else if (BITS != 3 && s <= p.s_max) {
-                    // x'/(s+eps) = (H u / sqrt(h)) / (s + eps): one multiplier for the unnormalised butterflies
-                    const float inv = p.rsqrt_h / (s + p.eps);
-                    const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-                    for (int w0 = 0; w0 < NW; w0 += CW) {
-                        uint32_t words[CW];
-#pragma unroll
-                        for (int wj = 0; wj < CW; ++wj) {
-                            const int wi = w0 + wj;
-                            // codes of this word, highest position first: acc = acc * 2^bits + code
-                            uint32_t acc_w = 0;
-#pragma unroll
-                            for (int kk = PER - 2; kk >= 0; kk -= 2) {
-                                uint32_t i0, i1;
-                                code2((wi * PER + kk) >> 1, inv2, i0, i1);
-                                acc_w = (acc_w * SH + i1) * SH + i0;
-                            }
-                            words[wj] = acc_w;
-                        }
-                        put(w0, words);
-                    }
-                } else if (BITS == 3) {
-                    // middle code 4 everywhere: the 3-bit stream repeats every 3 words
-                    constexpr uint32_t gm = 04444'4444u;  // eight 3-bit fours (octal)
-                    const uint32_t pat[3] = {gm | (gm << 24), (gm >> 8) | (gm << 16), (gm >> 16) | (gm << 8)};
-#pragma unroll
-                    for (int w0 = 0; w0 < NW; w0 += CW) {
-                        uint32_t ws[CW];
-#pragma unroll
-                        for (int wj = 0; wj < CW; ++wj) ws[wj] = pat[(w0 + wj) % 3];
-                        put(w0, ws);
-                    }
-                } else {
-                    uint32_t wmid = 0;
-#pragma unroll
-                    for (int kk = 0; kk < PER; ++kk) wmid = wmid * SH + (uint32_t)(p.L >> 1);
-                    uint32_t words[CW];
-#pragma unroll
-                    for (int wj = 0; wj < CW; ++wj) words[wj] = wmid;
-#pragma unroll
-                    for (int w0 = 0; w0 < NW; w0 += CW) put(w0, words);
-                }
-            }
-        }
+        if (valid) store_unit<HL, BITS, MODE>(p, v2, s, row, b * SPL + hf, lut_addr0);
     }
 
     // Leaving (normally or after an abort): copies this CTA issued must land

@@ -21,7 +21,11 @@ struct RpbhParams {
     int team, tpc, slots;
     int row_bytes, srow;  // bytes per input row; shared-memory row stride
     int nrs;              // row sets: ceil(M / RW)
+    // Warp-group kernel (rpbh_groups.cu): NG groups of G threads per CTA,
+    // tiles of R rows, thread (r, b) of a group on row r's h-block b.
+    int R, G, NG, ntiles;
     const uint32_t* gtab; // device gather table (see build_gather_table)
+    const uint16_t* gtab16; // the same with 16-bit entries (see build_gather_table16)
     const LutEntry* lut;  // device quantiser lookup table
     int lut_n, lut_off;   // entries; index offset = -(magic bits) - kmin
     float G_lut;          // lookup-table bins per unit of v
@@ -56,6 +60,14 @@ bool rpbh_choose_layout(RpbhParams& p, int h, int esize);
 // Test and tuning hook: force rows per warp, slots per team and lanes per
 // block (0: automatic).
 void rpbh_force_layout(int rows_per_warp, int slots, int lanes_per_block);
+
+// The warp-group kernel (rpbh_groups.cu) for permuted plans with h <= 128.
+// rpbh_choose_groups sets R, G, NG, srow, row_bytes and ntiles (p.M, p.d,
+// p.nb and p.lut_n set); false if the shape has no group layout.
+constexpr int kMaxGroups = 4;
+bool rpbh_choose_groups(RpbhParams& p, int esize);
+cudaError_t launch_rpbh_groups(const RpbhParams& p, bool in_bf16, int h, int bits, int mode, int grid,
+                               cudaStream_t stream);
 
 // The kernel for blocks of 256 ... 16384 (rht_big.cu): one row per CTA at a
 // time; RW, team, tpc, slots and srow are not used.

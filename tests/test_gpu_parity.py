@@ -471,3 +471,47 @@ def test_tall_tiles_give_the_same_product(cuda_device, M, d, N, bw, fp8):
     torch.cuda.synchronize()
     assert B.device_status() == 0
     assert torch.equal(y1, y2)
+
+
+# (kernel family, team layout (rows per warp, slots, lanes per block) or None)
+_FAMILIES = [(B.RPBH_KERNEL_GROUPS, None), (B.RPBH_KERNEL_TEAMS, None), (B.RPBH_KERNEL_TEAMS, (1, 1, 1)),
+             (B.RPBH_KERNEL_TEAMS, (8, 2, 1)), (B.RPBH_KERNEL_TEAMS, (4, 2, 2))]
+
+
+@pytest.mark.parametrize("family,layout", _FAMILIES)
+@pytest.mark.parametrize("M,d,h,ba,dt", [(301, 1536, 128, 4, "bf16"), (130, 256, 64, 2, "f32"),
+                                         (77, 3072, 128, 3, "bf16"), (45, 640, 32, 6, "bf16")])
+def test_kernel_families_match_oracle(cuda_device, family, layout, M, d, h, ba, dt):
+    """Both rotate-and-quantise kernel families (warp groups; teams under
+    several forced work layouts) against the oracle on the same ragged
+    inputs: rotation and norms, codes for activations and weights, and the
+    value outputs equal to the codebook at the codes."""
+    g = torch.Generator().manual_seed(d + M)
+    x = torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))
+    x = x.to(torch.bfloat16 if dt == "bf16" else torch.float32)
+    plan = B.rpbh_plan(d, h, 33)
+    perm, sign = oracle.plan(d, h, 33)
+    cb, ocb = B.codebook(d, ba), oracle.codebook(d, ba)
+    xg = x.to(cuda_device)
+    try:
+        B.debug_rpbh_kernel(family)
+        if layout:
+            B.debug_rpbh_layout(*layout)
+        a_idx, s = B.quantize_acts(plan, cb, xg)
+        w_idx, r = B.quantize_weights(plan, cb, xg)
+        val = None
+        if ba != 3:
+            val, s_v = B.quantize_acts_values(plan, cb, xg)
+        rows = np.arange(M)
+        check_rotation(plan, x, rows, h, perm, sign, cuda_device)
+        torch.cuda.synchronize()
+    finally:
+        B.debug_rpbh_kernel(0)
+        B.debug_rpbh_layout(0, 0, 0)
+    assert B.device_status() == 0
+    check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb, ocb, "acts")
+    check_quantized_rows(w_idx, r, x, rows, h, perm, sign, cb, ocb, "weights")
+    if val is not None:
+        u = B.unpack_indices(a_idx, d, ba).long()
+        tab = torch.from_numpy(cb.bf16_bits().view(np.int16)).to(cuda_device)
+        assert torch.equal(val.view(torch.int16), tab[u]) and torch.equal(s_v, s)
