@@ -61,26 +61,34 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-KERNEL_SOURCES = {"qgemm": "qgemm.cu", "qgemm_fp8": "qgemm.cu", "qgemm_values": "qgemm.cu",
-                  "qgemm_values_fp8": "qgemm.cu", "rpbh_quant": "rpbh_quant.cu", "rpbh_quant_values": "rpbh_quant.cu",
-                  "rpbh_quant_values_fp8": "rpbh_quant.cu"}
+_RPBH_SOURCES = ("rpbh_quant.cu", "rpbh_groups.cu")  # the team and the warp-group kernel (and their shared epilogue)
+KERNEL_SOURCES = {"qgemm": ("qgemm.cu",), "qgemm_fp8": ("qgemm.cu",), "qgemm_values": ("qgemm.cu",),
+                  "qgemm_values_fp8": ("qgemm.cu",), "rpbh_quant": _RPBH_SOURCES, "rpbh_quant_values": _RPBH_SOURCES,
+                  "rpbh_quant_values_fp8": _RPBH_SOURCES}
+
+
+def kernel_code_md5(kernel):
+    """md5 of the kernel's sources (code_only, concatenated in order)."""
+    import hashlib
+
+    parts = []
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "rotation_bit_quantization_rpbh_b200", "csrc", name), encoding="utf-8") as f:
+            parts.append(code_only(f.read()))
+    return hashlib.md5("\n".join(parts).encode()).hexdigest()
 
 
 def committed_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if one exists for
     this kernel and workload and the kernel source is unchanged since the
     counters were taken (null otherwise)."""
-    import hashlib
-
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f).get(kernel, {})
-    src = os.path.join(ROOT, "rotation_bit_quantization_rpbh_b200", "csrc", KERNEL_SOURCES[kernel])
-    with open(src, encoding="utf-8") as f:
-        if hashlib.md5(code_only(f.read()).encode()).hexdigest() != j.get("code_md5"):
-            return None
+    if kernel_code_md5(kernel) != j.get("code_md5"):
+        return None
     return j.get(workload)
 
 
