@@ -127,6 +127,7 @@ oq_status run_rpbh(const oq_plan_t* plan, oq_codebook_t* cb, const void* x, oq_d
         p.mid_val = mode == 3 ? cb->c_bf16[cb->L / 2] : (mode == 4 ? cb->c_e4m3[cb->L / 2] : 0u);
     }
     p.idx_out = idx_out;
+    p.st32 = (reinterpret_cast<uintptr_t>(idx_out) % 32 == 0 && p.out_row_bytes % 32 == 0) ? 1 : 0;
     p.s_out = s_out;
     p.r_out = r_out;
     p.y_out = y_out;

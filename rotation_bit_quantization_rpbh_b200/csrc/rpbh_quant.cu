@@ -143,6 +143,24 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
+// 32 bytes of output at a 32-byte-aligned global address: one 256-bit
+// store when the launch's output rows are 32-byte aligned throughout
+// (p.st32: the base and the row pitch), else two 16-byte stores.  A lane
+// writes its own h-block, so the stores of a warp go to 32 different rows
+// or blocks; whole 32-byte sectors halve the store instructions and the L2
+// sector updates against 16-byte halves.
+__device__ __forceinline__ void st_32B(uint8_t* dst, const uint32_t (&w)[8], int st32) {
+    if (st32) {
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(__cvta_generic_to_global(dst)),
+                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    } else {
+        uint4* d = reinterpret_cast<uint4*>(dst);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
 // A5 for one lane's HL values of row `row`: v2 holds the unnormalised
 // butterfly outputs of columns unit*HL .. unit*HL + HL-1 and s the row norm.
 // Writes the norm (the lane of unit 0), then the rotation (test mode), the
@@ -186,11 +204,12 @@ __device__ __forceinline__ void store_unit(const RpbhParams& p, float2 (&v2)[HL 
                 ge0 = q.x >= T0 ? 1u : 0u;
                 ge1 = q.y >= T1 ? 1u : 0u;
             };
+            constexpr int SW = (HL * VB) % 32 == 0 ? 8 : 4;  // words per store: 32 bytes where the unit holds them
 #pragma unroll
-            for (int w0 = 0; w0 < HL * VB / 4; w0 += 4) {
-                uint32_t words[4];
+            for (int w0 = 0; w0 < HL * VB / 4; w0 += SW) {
+                uint32_t words[SW];
 #pragma unroll
-                for (int wj = 0; wj < 4; ++wj) {
+                for (int wj = 0; wj < SW; ++wj) {
                     if constexpr (VB == 2) {
                         // bf16 pair: (lo or hi half of entry 0, lo or hi half of entry 1)
                         uint32_t val0, val1, ge0, ge1;
@@ -206,7 +225,10 @@ __device__ __forceinline__ void store_unit(const RpbhParams& p, float2 (&v2)[HL 
                         words[wj] = prmt_b32(lo, hi, 0x5410u);
                     }
                 }
-                dst[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
+                if constexpr (SW == 8)
+                    st_32B(reinterpret_cast<uint8_t*>(dst + (w0 >> 2)), words, p.st32);
+                else
+                    dst[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
             }
         } else {
             // the middle cell's value everywhere (see the codes branch)
@@ -218,12 +240,14 @@ __device__ __forceinline__ void store_unit(const RpbhParams& p, float2 (&v2)[HL 
         // ---- A5: v = x'/(s+eps) in fp32, index = #{ t_j <= v }, pack -----
         constexpr int NB = BITS == 6 ? HL : HL * BITS / 8;  // packed bytes of the lane's codes
         constexpr int NW = NB / 4;
-        constexpr int CW = NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1);  // words per store
+        constexpr int CW = NB % 32 == 0 ? 8 : (NB % 16 == 0 ? 4 : (NB % 8 == 0 ? 2 : 1));  // words per store
         constexpr int PER = BITS == 6 ? 4 : (BITS == 3 ? 8 : 32 / BITS);  // codes per word (3-bit: per 24-bit group)
         constexpr uint32_t SH = BITS == 6 ? 256u : (1u << BITS);
         uint8_t* dst = p.idx_out + (size_t)row * p.out_row_bytes + (size_t)unit * NB;
         auto put = [&](int w0, const uint32_t (&words)[CW]) {
-            if constexpr (CW == 4)
+            if constexpr (CW == 8)
+                st_32B(dst + (size_t)w0 * 4, words, p.st32);
+            else if constexpr (CW == 4)
                 reinterpret_cast<uint4*>(dst)[w0 >> 2] = make_uint4(words[0], words[1], words[2], words[3]);
             else if constexpr (CW == 2)
                 reinterpret_cast<uint2*>(dst)[w0 >> 1] = make_uint2(words[0], words[1]);

@@ -32,6 +32,7 @@ struct RpbhParams {
     int L;                // levels (2^bits)
     uint8_t* idx_out;     // packed indices (or the centroid values)
     int out_row_bytes;
+    int st32;             // idx_out and out_row_bytes are 32-byte aligned: 256-bit stores
     float* s_out;         // activations: s (fp32)
     uint16_t* r_out;      // weights: r (bf16)
     float* y_out;         // test hook: x' (fp32)

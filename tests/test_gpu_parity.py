@@ -473,6 +473,17 @@ def test_tall_tiles_give_the_same_product(cuda_device, M, d, N, bw, fp8):
     assert torch.equal(y1, y2)
 
 
+def _offset16(t):
+    """An empty tensor shaped and typed like t whose data starts 16 bytes past
+    a 32-byte boundary (the rows' pitch keeps every row so)."""
+    nbytes = t.numel() * t.element_size()
+    raw = torch.empty(nbytes + 64, dtype=torch.uint8, device=t.device)
+    off = (-raw.data_ptr()) % 32 + 16
+    out = raw[off:off + nbytes].view(t.dtype).view(t.shape)
+    assert out.data_ptr() % 32 == 16
+    return out
+
+
 # (kernel family, team layout (rows per warp, slots, lanes per block) or None)
 _FAMILIES = [(B.RPBH_KERNEL_GROUPS, None), (B.RPBH_KERNEL_TEAMS, None), (B.RPBH_KERNEL_TEAMS, (1, 1, 1)),
              (B.RPBH_KERNEL_TEAMS, (8, 2, 1)), (B.RPBH_KERNEL_TEAMS, (4, 2, 2))]
@@ -499,9 +510,14 @@ def test_kernel_families_match_oracle(cuda_device, family, layout, M, d, h, ba, 
             B.debug_rpbh_layout(*layout)
         a_idx, s = B.quantize_acts(plan, cb, xg)
         w_idx, r = B.quantize_weights(plan, cb, xg)
+        # the same outputs into buffers 16 but not 32 bytes aligned (16-byte stores)
+        a_idx16 = _offset16(a_idx)
+        B.quantize_acts(plan, cb, xg, a_idx16)
         val = None
         if ba != 3:
             val, s_v = B.quantize_acts_values(plan, cb, xg)
+            val16 = _offset16(val)
+            B.quantize_acts_values(plan, cb, xg, val16)
         rows = np.arange(M)
         check_rotation(plan, x, rows, h, perm, sign, cuda_device)
         torch.cuda.synchronize()
@@ -509,6 +525,9 @@ def test_kernel_families_match_oracle(cuda_device, family, layout, M, d, h, ba, 
         B.debug_rpbh_kernel(0)
         B.debug_rpbh_layout(0, 0, 0)
     assert B.device_status() == 0
+    assert torch.equal(a_idx16, a_idx)
+    if val is not None:
+        assert torch.equal(val16, val)
     check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb, ocb, "acts")
     check_quantized_rows(w_idx, r, x, rows, h, perm, sign, cb, ocb, "weights")
     if val is not None:
