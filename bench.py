@@ -47,7 +47,11 @@ def parse():
                     help="layer schedule timed: activation codes decoded in the GEMM, or centroid values written by "
                          "the quantiser and streamed into the GEMM; auto = the one oq_qlinear takes")
     ap.add_argument("--ablation", action="store_true",
-                    help="time the rotation ablation (RPBH, Block-RHT, dense Haar) on --workload instead of the layer")
+                    help="time the rotation ablation (RPBH, Block-RHT, Full RHT, dense Haar) on --workload instead "
+                         "of the layer")
+    ap.add_argument("--quant-sweep", action="store_true",
+                    help="time the quantiser alone over a range of M at --workload's d (fixed cost against per-row "
+                         "cost) instead of the layer")
     return ap.parse_args()
 
 
@@ -607,6 +611,15 @@ def run_ours(args):
     gemm_key = ("qgemm_values" if schedule == "values" else "qgemm") + ("_fp8" if args.fp8 else "")
     rpbh_key = "rpbh_quant" + (("_values_fp8" if args.fp8 else "_values") if schedule == "values" else "")
     roof, gemm_tflops = rooflines(w, peaks, args.fp8, ms_gemm, ms_rpbh, ms_codes, schedule, (gemm_key, rpbh_key))
+    if world == 1:
+        # context for the per-launch figure: the launch floor every event time
+        # contains, and the quantiser's rate over 2x-8x the workload's rows
+        # (the slope: the cost per row once the fixed cost is amortised)
+        k_sw = max(5, min(args.steps, 10))
+        srows, per_row, _ = quant_sweep_rows(w, L.plan, L.cb_a, L.x, [2 * w.M, 4 * w.M, 8 * w.M], flush, stream,
+                                             k_sw, 3, values=False)
+        roof["roofline_rpbh_codes"]["launch_floor_us"] = launch_floor_us(flush, stream, k_sw)
+        roof["roofline_rpbh_codes"]["steady_state"] = steady_fit(srows, per_row, peaks["hbm_gbs"], 2 * w.M)
     flops = 2.0 * w.M * w.N * w.d
     out = {
         "metric": METRIC, "value": job_throughput(world, w.M, ms), "unit": "tokens/s", "n_gpus": world,
@@ -776,12 +789,120 @@ def run_ablation(args):
     print(json.dumps(out), flush=True)
 
 
+def _median_event_us(fn, flush, stream, steps, warmup):
+    """Median event time (us) of fn() over `steps` calls, L2 flushed (256 MB
+    write, outside the events) before each."""
+    import numpy as np
+    import torch
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([e0.elapsed_time(e1) for e0, e1 in ev])) * 1e3
+
+
+def launch_floor_us(flush, stream, steps):
+    """A one-element torch kernel timed like the kernels: the fixed launch
+    and event cost that every per-launch time here contains."""
+    import torch
+
+    one = torch.zeros(1, device=flush.device)
+    return _median_event_us(lambda: one.add_(1.0), flush, stream, steps, 3)
+
+
+def quant_sweep_rows(w, plan, cb, x0, Ms, flush, stream, steps, warmup, values=True):
+    """Quantiser event times at M rows each (the workload's rows repeated)."""
+    import torch
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+
+    per_row = w.d * x0.element_size() + B.packed_row_bytes(w.d, w.bits_a) + 4  # §8(d) bytes per token
+    peak = measured_peaks()["hbm_gbs"]
+    rows = []
+    for M in Ms:
+        reps = (M + x0.shape[0] - 1) // x0.shape[0]
+        x = x0.repeat(reps, 1)[:M].contiguous()
+        idx = torch.empty((M, B.packed_row_bytes(w.d, w.bits_a)), dtype=torch.uint8, device=x0.device)
+        s = torch.empty(M, dtype=torch.float32, device=x0.device)
+        tc = _median_event_us(lambda: B.quantize_acts(plan, cb, x, idx, s, stream=stream), flush, stream, steps, warmup)
+        r = {"M": M, "codes_us": tc, "codes_gbs": M * per_row / (tc * 1e-6) / 1e9}
+        r["codes_frac"] = r["codes_gbs"] / peak
+        if values:
+            val = torch.empty((M, w.d), dtype=torch.bfloat16, device=x0.device)
+            r["values_us"] = _median_event_us(lambda: B.quantize_acts_values(plan, cb, x, val, s, stream=stream),
+                                              flush, stream, steps, warmup)
+            del val
+        rows.append(r)
+        del x, idx, s
+    return rows, per_row, peak
+
+
+def steady_fit(rows, per_row, peak, m_min):
+    """Least-squares line through codes_us against M for M >= m_min: the
+    per-row cost as a rate (GB/s and fraction of the peak) and the fixed
+    cost (intercept)."""
+    import numpy as np
+
+    big = [r for r in rows if r["M"] >= m_min]
+    if len(big) < 2:
+        return None
+    k, c0 = np.polyfit(np.array([r["M"] for r in big], dtype=np.float64),
+                       np.array([r["codes_us"] for r in big], dtype=np.float64), 1)
+    gbs = per_row / (k * 1e-6) / 1e9
+    return {"us_per_row": float(k), "intercept_us": float(c0), "steady_gbs": gbs, "steady_frac": gbs / peak,
+            "fit_M": [r["M"] for r in big]}
+
+
+def run_quant_sweep(args):
+    """The quantiser alone (codes and bf16 values modes) at the workload's d,
+    h and bits over a range of M: the workload's own rows repeated.  Event
+    time per launch (median of --steps, L2 flushed before each), beside a
+    one-element torch kernel timed the same way (the launch floor of this
+    measurement).  The slope over the largest M gives the steady-state
+    rate, free of the fixed launch and ramp cost."""
+    import torch
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+    from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --quant-sweep needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    w = I.WORKLOADS[args.workload]
+    x0 = I.make_x(w).to(dev)
+    plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
+    cb = B.codebook(w.d, w.bits_a)
+    cb.upload()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    floor = launch_floor_us(flush, stream, args.steps)
+    Ms = sorted(M for M in {148, 592, 2048, w.M, 2 * w.M, 4 * w.M, 8 * w.M} if M * w.d * 2 * 3 <= (3 << 30))
+    rows, per_row, peak = quant_sweep_rows(w, plan, cb, x0, Ms, flush, stream, args.steps, args.warmup)
+    if B.device_status() != 0:
+        raise SystemExit("a kernel reported a timeout")
+    print(json.dumps({"metric": "quantiser event time against M", "workload": w.name, "d": w.d, "h": w.h,
+                      "bits_a": w.bits_a, "steps": args.steps, "launch_floor_us": floor,
+                      "bytes_per_row": per_row, "peak_gbs": peak, "rows": rows,
+                      "fit_codes": steady_fit(rows, per_row, peak, 2 * w.M),
+                      "note": "event time per launch, L2 flushed (256 MB write) before each; launch_floor_us is a "
+                              "one-element torch kernel timed the same way; fit over M >= 2x the workload's M"}))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.ablation:
         run_ablation(args)
+    elif args.quant_sweep:
+        run_quant_sweep(args)
     else:
         run_ours(args)
 
