@@ -192,7 +192,7 @@ def job_throughput(world, tokens_per_rank, ms_per_step):
 def rpbh_bytes(w):
     """Algorithmic bytes of one quantiser launch as the method defines its
     output: x read, the packed codes written (one byte per code at 6 bits),
-    and s.  The values schedule's 2-byte centroid values are this build's
+    and s.  The values schedule's 2-byte centroid values are the library's
     layout for the product, not the method's output, so they count in the
     measured traffic only."""
     esize = 4 if w.x_dtype == "f32" else 2
