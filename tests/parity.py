@@ -22,6 +22,7 @@ import torch
 
 import oracle
 from rotation_bit_quantization_rpbh_b200 import binding as B
+from stored_codebooks import stored_oracle_codebook  # noqa: F401  (re-exported for the parity tests)
 
 BAND_REL = 1e-6
 MISMATCH_FRAC = 1e-5

@@ -17,7 +17,7 @@ from rotation_bit_quantization_rpbh_b200 import binding as B
 from rotation_bit_quantization_rpbh_b200 import inputs as I
 
 from parity import (GEMM_TOL, check_product, check_quantized_rows, check_rotation, gemm_reference, rel_frob,
-                    to_f64)
+                    stored_oracle_codebook, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -534,3 +534,32 @@ def test_kernel_families_match_oracle(cuda_device, family, layout, M, d, h, ba, 
         u = B.unpack_indices(a_idx, d, ba).long()
         tab = torch.from_numpy(cb.bf16_bits().view(np.int16)).to(cuda_device)
         assert torch.equal(val.view(torch.int16), tab[u]) and torch.equal(s_v, s)
+
+
+@pytest.mark.parametrize("M,d,h,variant", [(64, 3072, 128, "rpbh"),        # warp-group kernel
+                                           (40, 12288, 128, "rpbh"),       # team kernel, 112 KB table
+                                           (48, 1536, 128, "block_rht"),   # team kernel, contiguous reads
+                                           (12, 4096, 4096, "block_rht")])  # staged kernel (Full RHT)
+def test_eight_bit_codes_in_every_kernel_family(cuda_device, M, d, h, variant):
+    """8-bit codes (256 levels: the widest table, which grows with sqrt(d))
+    through each kernel family at sizes where the table is large, against
+    the oracle; the value outputs equal the codebook at the codes."""
+    seed = 90 + M
+    v = B.OQ_ROT_BLOCK_RHT if variant == "block_rht" else B.OQ_ROT_RPBH
+    plan = B.rotation_plan(d, h, seed, v)
+    perm, sign = oracle.plan(d, h, seed, variant=oracle.BLOCK_RHT if variant == "block_rht" else 0)
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16)
+    cb, ocb = B.codebook(d, 8), stored_oracle_codebook(d, 8)
+    xg = x.to(cuda_device)
+    a_idx, s = B.quantize_acts(plan, cb, xg)
+    w_idx, r = B.quantize_weights(plan, cb, xg)
+    val, s_v = B.quantize_acts_values(plan, cb, xg)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert a_idx.shape == (M, d)
+    rows = np.arange(M)
+    check_quantized_rows(a_idx, s, x, rows, h, perm, sign, cb, ocb, "acts")
+    check_quantized_rows(w_idx, r, x, rows, h, perm, sign, cb, ocb, "weights")
+    tab = torch.from_numpy(cb.bf16_bits().view(np.int16)).to(cuda_device)
+    assert torch.equal(val.view(torch.int16), tab[a_idx.long()]) and torch.equal(s_v, s)

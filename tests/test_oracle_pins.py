@@ -454,3 +454,27 @@ def test_quantised_product_error_falls_with_bits():
         errs.append(np.linalg.norm(y - ref) / np.linalg.norm(ref))
     assert errs[0] > errs[1] > errs[2]
     assert errs[1] < 0.2 and errs[2] < 0.06
+
+
+@pytest.mark.parametrize("d", [1536, 3072, 4096, 12288])
+def test_stored_eight_bit_codebooks_satisfy_lloyd_max_conditions(d):
+    """The oracle's stored 8-bit codebooks (tests/golden, written by
+    make_oracle_codebooks.py from oracle.codebook) are pinned the same way
+    as the solved ones: ascending, antisymmetric, thresholds at midpoints,
+    each centroid the conditional mean of its cell under f_d (scipy's
+    incomplete beta for the mass, the closed-form first moment)."""
+    from stored_codebooks import stored_oracle_codebook
+
+    c, t = stored_oracle_codebook(d, 8)
+    L = 256
+    sd = math.sqrt(d)
+    assert c.shape == (L,) and t.shape == (L - 1,)
+    assert np.all(np.diff(c) > 0)
+    np.testing.assert_array_equal(c, -c[::-1])
+    np.testing.assert_allclose(t, 0.5 * (c[:-1] + c[1:]), rtol=0, atol=1e-15 / sd)
+    assert t[L // 2 - 1] == 0.0
+    edges = [-1.0] + list(t) + [1.0]
+    for j in range(0, L, 5):
+        m = fd_mass(d, edges[j], edges[j + 1])
+        f1 = fd_first_moment(d, edges[j], edges[j + 1])
+        assert abs((f1 / m - c[j]) * sd) < 1e-9, (j, f1 / m, c[j])
