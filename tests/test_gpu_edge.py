@@ -138,3 +138,45 @@ def test_binding_checks_buffers_before_the_call(layer, cuda_device):
                 torch.ones(16, dtype=torch.float16, device=cuda_device), w_idx, w_r)
     with pytest.raises(ValueError):  # an output on the host
         B.quantize_acts(plan, cb4, x, s_out=torch.empty(16))
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_layer_replays_in_a_cuda_graph(cuda_device, fp8):
+    """The layer call captured in a CUDA graph replays to the same bits as
+    the eager call, on new inputs copied into the captured buffer. One eager
+    call first uploads the tables and sets the kernels' attributes, which
+    capture cannot do. The two launches keep their programmatic dependency
+    inside the graph."""
+    M, d, N, h = 512, 1536, 768, 128
+    plan = B.rpbh_plan(d, h, 5)
+    cb_a, cb_w = B.codebook(d, 4), B.codebook(d, 4)
+    g = torch.Generator().manual_seed(5)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16).to(cuda_device)
+    x1 = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16).to(cuda_device)
+    x2 = (torch.randn(M, d, generator=g) * 3.0).to(torch.bfloat16).to(cuda_device)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W)
+    need = max(B.qlinear_workspace_values(M, d), B.qlinear_workspace(M, d, 4))
+    ws = torch.empty(need, dtype=torch.uint8, device=cuda_device)
+    xin = x1.clone()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=cuda_device)
+    B.qlinear(plan, cb_a, cb_w, xin, w_idx, w_r, y=y, workspace=ws, fp8=fp8)  # eager: uploads, attributes
+    torch.cuda.synchronize()
+    y1_eager = y.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        B.qlinear(plan, cb_a, cb_w, xin, w_idx, w_r, y=y, workspace=ws, fp8=fp8)
+    y.zero_()
+    xin.copy_(x2)
+    graph.replay()
+    torch.cuda.synchronize()
+    y2_graph = y.clone()
+    xin.copy_(x1)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    y2_eager = B.qlinear(plan, cb_a, cb_w, x2, w_idx, w_r, fp8=fp8)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y1_eager)
+    assert torch.equal(y2_graph, y2_eager)
+    assert not torch.equal(y2_graph, y1_eager)
+    del graph
