@@ -73,3 +73,28 @@ def test_noalloc_needs_the_codebook_on_the_device_first(cuda_device):
     with pytest.raises(B.OQError) as e:
         B.qlinear_noalloc(plan, cb_a, cb_w, x, w_idx, w_r, y)
     assert e.value.status == 1
+
+
+def test_noalloc_reports_too_large_for_eight_bit_values_before_any_work(cuda_device):
+    """8-bit activations have no codes schedule (no in-kernel 8-bit decoder),
+    so when their values do not fit the scratch the call must return
+    OQ_ERR_TOO_LARGE up front -- not quantise into the scratch and then find
+    that the product cannot run -- even though the 8-bit codes would fit."""
+    d, N, M = 4096, 256, 20000
+    plan = B.rpbh_plan(d, 128, 34)
+    cb_a, cb_w = B.codebook(d, 8), B.codebook(d, 4)
+    cb_a.upload()  # the call itself allocates nothing
+    assert B.qlinear_workspace_values(M, d) > B.NOALLOC_SCRATCH_BYTES
+    assert B.qlinear_workspace(M, d, 8) <= B.NOALLOC_SCRATCH_BYTES
+    x = torch.zeros((M, d), dtype=torch.bfloat16, device=cuda_device)
+    w_idx = torch.zeros((N, d // 2), dtype=torch.uint8, device=cuda_device)
+    w_r = torch.ones(N, dtype=torch.bfloat16, device=cuda_device)
+    y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device=cuda_device)
+    L = B.lib()
+    st = L.oq_qlinear_noalloc(plan.handle, cb_a.handle, cb_w.handle, ctypes.c_void_p(x.data_ptr()), B.OQ_BF16, M,
+                              ctypes.c_void_p(w_idx.data_ptr()), ctypes.c_void_p(w_r.data_ptr()), N, None,
+                              ctypes.c_void_p(y.data_ptr()), None)
+    torch.cuda.synchronize()
+    assert st == 8  # OQ_ERR_TOO_LARGE
+    assert B.device_status() == 0
+    assert bool((y == 7.0).all())  # nothing was written
