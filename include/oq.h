@@ -34,6 +34,12 @@
  *     Launch failures are reported as OQ_ERR_CUDA.  A kernel that gives up a
  *     bounded wait records OQ_ERR_TIMEOUT in a device flag read by
  *     oq_device_status().
+ *   - The quantising calls, the products and the layer calls may be
+ *     captured in a CUDA graph (stream capture) once one eager call of the
+ *     same kind has run on the device: that call uploads what is missing
+ *     and sets the kernels' launch attributes, which capture cannot do.
+ *     A quantiser followed by its product keeps their programmatic
+ *     dependency inside the graph.
  *   - Layouts are row-major.  Packed indices are K-major rows, LSB-first:
  *     bits = 4: two indices per byte (index k in bits 4*(k%2) of byte k/2);
  *     bits = 2: four per byte (bits 2*(k%4) of byte k/4);
