@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--ablation", action="store_true",
                     help="time the rotation ablation (RPBH, Block-RHT, Full RHT, dense Haar) on --workload instead "
                          "of the layer")
+    ap.add_argument("--gemm-sweep", action="store_true",
+                    help="time the A-values product alone over a range of M at --workload's d, N and bits (per-round "
+                         "rate against the fixed cost) instead of the layer")
     ap.add_argument("--quant-sweep", action="store_true",
                     help="time the quantiser alone over a range of M at --workload's d (fixed cost against per-row "
                          "cost) instead of the layer")
@@ -923,6 +926,61 @@ def run_quant_sweep(args):
                               "one-element torch kernel timed the same way; fit over M >= 2x the workload's M"}))
 
 
+def run_gemm_sweep(args):
+    """The A-values product alone (bf16, or e4m3 with --fp8) at the
+    workload's d, N and bits over a range of M: the workload's rows
+    repeated, quantised once.  Event time per launch (median of --steps, L2
+    flushed before each).  A pair of SMs takes one 256 x 256 tile at a time,
+    so the time grows in rounds of (SMs / 2) tiles; the slope over the
+    largest M gives the steady per-round rate, free of the launch floor, the
+    pipeline fill and drain and the partial last round."""
+    import numpy as np
+    import torch
+
+    from rotation_bit_quantization_rpbh_b200 import binding as B
+    from rotation_bit_quantization_rpbh_b200 import inputs as I
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --gemm-sweep needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    w = I.WORKLOADS[args.workload]
+    x0 = I.make_x(w).to(dev)
+    plan = B.rpbh_plan(w.d, w.h, w.plan_seed)
+    cb_a, cb_w = B.codebook(w.d, w.bits_a), B.codebook(w.d, w.bits_w)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, I.make_w(w).to(dev))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
+    peak = measured_peaks()["bf16_tflops"] * (2 if args.fp8 else 1)
+    rows = []
+    for M in sorted({w.M // 4, w.M // 2, w.M, 2 * w.M, 4 * w.M, 8 * w.M}):
+        if M < 256 or M * (w.d * 2 + w.N * 2) > (3 << 30):
+            continue
+        x = x0.repeat((M + w.M - 1) // w.M, 1)[:M].contiguous()
+        val, s = B.quantize_acts_values(plan, cb_a, x, fp8=args.fp8)
+        y = torch.empty((M, w.N), dtype=torch.bfloat16, device=dev)
+        us = _median_event_us(lambda: B.qgemm_values(cb_w, val, s, w_idx, w_r, y=y, stream=stream, fp8=args.fp8),
+                              flush, stream, args.steps, args.warmup)
+        tiles = ((M + 255) // 256) * ((w.N + 255) // 256)
+        tf = 2.0 * M * w.N * w.d / (us * 1e-6) / 1e12
+        rows.append({"M": M, "us": us, "tiles": tiles, "rounds": tiles / pairs, "tflops": tf, "frac": tf / peak})
+        del x, val, s, y
+    if B.device_status() != 0:
+        raise SystemExit("a kernel reported a timeout")
+    fit = None
+    big = [r for r in rows if r["M"] >= 2 * w.M]
+    if len(big) >= 2:
+        k, c0 = np.polyfit(np.array([r["rounds"] for r in big]), np.array([r["us"] for r in big]), 1)
+        flop_round = 2.0 * pairs * 256 * 256 * w.d
+        fit = {"us_per_round": float(k), "intercept_us": float(c0), "steady_tflops": flop_round / (k * 1e-6) / 1e12,
+               "steady_frac": flop_round / (k * 1e-6) / 1e12 / peak, "fit_M": [r["M"] for r in big]}
+    print(json.dumps({"metric": "A-values product event time against M", "workload": w.name, "d": w.d, "N": w.N,
+                      "bits_w": w.bits_w, "fp8": args.fp8, "sm_pairs": pairs, "steps": args.steps,
+                      "peak_tflops": peak, "rows": rows, "fit": fit,
+                      "note": "event time per launch, L2 flushed (256 MB write) before each; a round is one "
+                              "256 x 256 tile per SM pair; fit over M >= 2x the workload's M"}))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -931,6 +989,8 @@ def main():
         run_ablation(args)
     elif args.quant_sweep:
         run_quant_sweep(args)
+    elif args.gemm_sweep:
+        run_gemm_sweep(args)
     else:
         run_ours(args)
 
