@@ -563,3 +563,27 @@ def test_eight_bit_codes_in_every_kernel_family(cuda_device, M, d, h, variant):
     check_quantized_rows(w_idx, r, x, rows, h, perm, sign, cb, ocb, "weights")
     tab = torch.from_numpy(cb.bf16_bits().view(np.int16)).to(cuda_device)
     assert torch.equal(val.view(torch.int16), tab[a_idx.long()]) and torch.equal(s_v, s)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_product_gives_the_same_bits_for_every_output_alignment(cuda_device, fp8):
+    """The product's epilogue writes 32-byte sectors when y's base and row
+    pitch are 32-byte aligned, 16-byte stores otherwise: the same bits."""
+    M, d, N, h = 300, 512, 768, 128
+    plan = B.rpbh_plan(d, h, 17)
+    cb_a, cb_w = B.codebook(d, 4), B.codebook(d, 4)
+    g = torch.Generator().manual_seed(17)
+    x = (torch.randn(M, d, generator=g) * torch.exp(torch.randn(d, generator=g))).to(torch.bfloat16).to(cuda_device)
+    W = (torch.randn(N, d, generator=g) * 0.02).to(torch.bfloat16).to(cuda_device)
+    w_idx, w_r = B.quantize_weights(plan, cb_w, W)
+    val, s = B.quantize_acts_values(plan, cb_a, x, fp8=fp8)
+    y = B.qgemm_values(cb_w, val, s, w_idx, w_r, fp8=fp8)
+    y16 = _offset16(y)
+    B.qgemm_values(cb_w, val, s, w_idx, w_r, y=y16, fp8=fp8)
+    a_idx, s_c = B.quantize_acts(plan, cb_a, x)
+    yc = (B.qgemm_fp8 if fp8 else B.qgemm)(cb_a, cb_w, a_idx, s_c, w_idx, w_r)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    assert y.data_ptr() % 32 == 0
+    assert torch.equal(y16, y)
+    assert torch.equal(yc, y)
