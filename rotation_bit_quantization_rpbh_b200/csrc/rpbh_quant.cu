@@ -1,4 +1,9 @@
-// Fused RPBH rotate -> norm/direction split -> Lloyd-Max quantise -> pack.
+// Fused RPBH rotate -> norm/direction split -> Lloyd-Max quantise -> pack:
+// the team kernel, and the quantiser epilogue (store_unit) that it shares
+// with the warp-group kernel (rpbh_groups.cu).  The library runs the team
+// kernel for blocks of at most 128 when d > 8192 or when the plan has no
+// permutation (its contiguous read path); the warp-group kernel takes
+// permuted plans up to d = 8192, and rht_big.cu blocks of 256 and more.
 //
 // Method: "OrbitQuant" paper summary (hyper.ai, papers 2607.02461), section
 // 方法 (Method):
